@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the DiT-block denoising path on B200; prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dit512] [--impl reference]
+
+A step is one complete denoise of the workload: every Euler step of the configured sigma
+grid, each running every active DiT block over the joint video+audio token stream (the
+whole hot path: AdaLN LN, QKV+RoPE, attention, out-proj+gated residual, LN, FC1+GELU,
+FC2+gated residual, final AdaLN + Euler).  Inputs are synthetic (seeded, random-init
+weights of the stated architecture).  The metric is DiT block tokens per second: tokens
+processed by each executed block, summed over blocks and Euler steps, per second of
+device time; TFLOPS counts 24 N d^2 + 4 N^2 d per block.
+
+Multi-GPU (torchrun, one process per GPU): every rank denoises its own latent with the
+same weights (independent replicas, no data-path collective); value = all ranks' tokens
+/ the slowest rank's device time.
+
+--impl reference runs the CPU oracle (the plain float64 definition of the same block) on
+a bounded sample of the workload: one block over the full token count per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DiT block tokens/sec and achieved bf16 TFLOPS vs tensor peak, 1xB200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram bytes per launch from an ncu capture, keyed by kernel; only used while the kernel
+# source still hashes to the value recorded with it.
+NCU_TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="dit512")
+    ap.add_argument("--impl", default="h3b", choices=["h3b", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def block_flops(n, d, f):
+    return 2 * n * d * 3 * d + 2 * n * d * d + 4 * n * d * f + 4 * n * n * d
+
+
+def workload_counts(cfg, active):
+    """Per complete denoise: block-tokens, FLOPs and launches of each block kernel."""
+    order = [b for b in range(cfg.n_blocks) if active is None or active[b]]
+    n_full, n_red = cfg.n_tokens, cfg.n_video_reduced + cfg.n_audio
+    tokens = flops = 0
+    for k, _ in enumerate(order):
+        n = n_red if (cfg.reduce_after > 0 and k >= cfg.reduce_after) else n_full
+        tokens += n
+        flops += block_flops(n, cfg.d, cfg.d_ff)
+    per_step = {"tokens": tokens, "flops": flops, "blocks": len(order)}
+    return {k: v * cfg.run_steps for k, v in per_step.items()}, len(order)
+
+
+def src_hash(name):
+    with open(os.path.join(ROOT, "video_diffusion_transformer_03_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.path = tempfile.mktemp(prefix="h3b_clocks_", suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id, "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        sm.append(float(parts[1]))
+                        smax.append(float(parts[2]))
+                    except ValueError:
+                        continue
+                    for name, val in zip(self.NAMES, parts[5:9]):
+                        if val.lower() == "active":
+                            reasons.add(name)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(cfg, min_seconds=10.0, max_blocks=8):
+    """Time the oracle (float64 numpy, as it stands) on full-size blocks of the workload."""
+    import numpy as np
+    from oracle import workloads
+    from video_diffusion_transformer_03_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    p = {k: f64(v) for k, v in synth.block_params(cfg, 0).items()}
+    c = f64(synth.conditioning(cfg))
+    x = f64(synth.latent_noise(cfg).to(__import__("torch").bfloat16))
+    done, t0 = 0, time.perf_counter()
+    while done < max_blocks:
+        x, _ = workloads.block(cfg, p, c, x)
+        done += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": cfg.n_tokens * done / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} full block forward(s) of {cfg.name} ({cfg.n_tokens} tokens, "
+                      f"d={cfg.d}) in float64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    from video_diffusion_transformer_03_b200 import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    from oracle import workloads
+    cfg = synth.CONFIGS[args.config]
+    f64 = lambda t: t.float().numpy().astype(np.float64)
+    p = {k: f64(v) for k, v in synth.block_params(cfg, 0).items()}
+    c = f64(synth.conditioning(cfg))
+    x0 = f64(synth.latent_noise(cfg).to(__import__("torch").bfloat16))
+    for _ in range(args.warmup):
+        workloads.block(cfg, p, c, x0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        workloads.block(cfg, p, c, x0)
+    dt = time.perf_counter() - t0
+    value = cfg.n_tokens * args.steps / dt
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    flops = block_flops(cfg.n_tokens, cfg.d, cfg.d_ff)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": workload_name(cfg), "sample": "one full block forward per step"},
+            "tflops": flops * args.steps / dt / 1e12,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"one full block forward of {cfg.name} per step "
+                                       f"({cfg.n_tokens} tokens), float64 numpy"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_name(cfg):
+    t, h, w = cfg.grid
+    s = (f"{cfg.name}: {cfg.n_blocks} DiT blocks d={cfg.d} {cfg.n_heads}x{cfg.head_dim} heads "
+         f"MLP {cfg.d_ff}, video grid t{t}xh{h}xw{w}={cfg.n_video} + {cfg.n_audio} audio tokens, "
+         f"{cfg.run_steps} Euler steps")
+    if cfg.reduce_after > 0:
+        s += f", token pairing after block {cfg.reduce_after}"
+    if cfg.active_count < cfg.n_blocks:
+        s += f", {cfg.active_count} of {cfg.n_blocks} blocks active"
+    return s
+
+
+# ------------------------------------------------------------------------------ GPU arm
+def time_kernels(model, cfg, peaks, counts_per_step, reps=20):
+    """Time each kernel of the block alone (CUDA events on the launching stream), with the
+    weights rotated over all blocks so that they stream from HBM as in the step."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b
+    dev = model.device
+    n, d, f, hd, H = cfg.n_tokens, cfg.d, cfg.d_ff, cfg.head_dim, cfg.n_heads
+    g = torch.Generator(device=dev).manual_seed(7)
+    rnd = lambda *s: torch.randn(*s, generator=g, device=dev).to(torch.bfloat16)
+    h = rnd(n, d)
+    qkv = rnd(n, 3 * d)
+    attn = torch.empty(n, d, dtype=torch.bfloat16, device=dev)
+    gbuf = rnd(n, f)
+    x = rnd(n, d)
+    xs = torch.randn(n, d, device=dev)
+    cs = torch.empty((n, hd // 2, 2), dtype=torch.float32, device=dev)
+    h3b.rope_table(model.dims, model.grid, False, cs)
+    mod = model.mods[0]
+    P = model.params
+    nb = len(P)
+    kinds = {
+        "gemm_qkv_rope": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_qkv"], h3b.EPI_BIAS_ROPE,
+                                                  P[i % nb]["b_qkv"], qkv, rope_cs=cs,
+                                                  rope_cols=2 * d, head_dim=hd),
+                          "tensor", 2 * n * d * 3 * d),
+        "attention": (lambda i: h3b.attention(qkv, H, hd, attn), "tensor", 4 * n * n * d),
+        "gemm_out_gate": (lambda i: h3b.gemm_bf16(attn, P[i % nb]["w_o"], h3b.EPI_GATE_RESID,
+                                                  P[i % nb]["b_o"], x, gate=mod[2]),
+                          "tensor", 2 * n * d * d),
+        "gemm_fc1_gelu": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_fc1"], h3b.EPI_BIAS_GELU,
+                                                  P[i % nb]["b_fc1"], gbuf),
+                          "tensor", 2 * n * d * f),
+        "gemm_fc2_gate": (lambda i: h3b.gemm_bf16(gbuf, P[i % nb]["w_fc2"], h3b.EPI_GATE_RESID,
+                                                  P[i % nb]["b_fc2"], x, gate=mod[5]),
+                          "tensor", 2 * n * f * d),
+        "ln_modulate": (lambda i: h3b.ln_modulate(x, cfg.ln_eps, mod[0], mod[1], h), "hbm",
+                        4 * n * d),
+        "final_euler": (lambda i: h3b.final_euler(x, cfg.n_video, cfg.ln_eps, model.final_mod,
+                                                  1.0, 0.75, xs), "hbm", 10 * n * d),
+    }
+    blocks = counts_per_step["blocks"]
+    launches = {"gemm_qkv_rope": blocks, "attention": blocks, "gemm_out_gate": blocks,
+                "gemm_fc1_gelu": blocks, "gemm_fc2_gate": blocks, "ln_modulate": 2 * blocks,
+                "final_euler": cfg.run_steps}
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name, (fn, bound, work) in kinds.items():
+        for i in range(3):
+            fn(i)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for i in range(reps):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        h3b.sync_status()
+        ms = e0.elapsed_time(e1) / reps
+        if bound == "tensor":
+            achieved, peak, unit = work / (ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        else:
+            achieved, peak, unit = work / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        out[name] = {"bound": bound, "ms": ms, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "work_per_launch": work,
+                     "launches_per_step": launches[name],
+                     "ms_per_step": ms * launches[name]}
+    return out
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    from video_diffusion_transformer_03_b200.pipeline import DiTDenoiser
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    cfg = synth.CONFIGS[args.config]
+    model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
+    counts, n_active = workload_counts(cfg, model.active)
+    x0 = synth.latent_noise(cfg, device=str(dev))
+    x = x0.clone()
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        model.run(x)
+    h3b.sync_status()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+
+    # ---- timed region: K complete denoises, device time
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(gpu_id)
+    launches0 = h3b.launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        model.run(x)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = h3b.launch_count() - launches0
+    clk = clocks.stop()
+    barrier()
+    h3b.sync_status()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms / args.steps
+    value = counts["tokens"] * args.steps * world / (ms * 1e-3)
+    tflops = counts["flops"] * args.steps * world / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the host-buffer entry point (copies inside the timed region)
+    host_in = synth.latent_noise(cfg).pin_memory()
+    host_out = torch.empty_like(host_in).pin_memory()
+    scratch = torch.empty_like(x0)
+    for _ in range(min(args.warmup, 3)):
+        model.run_host(host_in, host_out, scratch)
+    barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, args.steps // 2)
+    torch.cuda.synchronize(dev)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        model.run_host(host_in, host_out, scratch)
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3))
+    nbytes = host_in.numel() * host_in.element_size()
+    e2e = {"value": counts["tokens"] * e2e_steps * world / (e2e_ms * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+           "ms_per_step": e2e_ms / e2e_steps}
+
+    breakdown = None
+    roofline = None
+    if not args.no_breakdown:
+        breakdown = time_kernels(model, cfg, peaks, {"blocks": n_active * cfg.run_steps})
+        dom = max(breakdown, key=lambda k: breakdown[k]["ms_per_step"])
+        b = breakdown[dom]
+        tr = NCU_TRAFFIC.get(dom)
+        traffic = tr["bytes"] if tr and tr.get("src_sha") == src_hash(tr["src"]) else None
+        roofline = {"kernel": dom, "bound": b["bound"], "achieved": b["achieved"],
+                    "peak": b["peak"], "unit": b["unit"], "frac": b["frac"], "traffic": traffic,
+                    "peak_source": f"{peak_src} burst"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random-init weights and latent noise)",
+            "config": {"workload": workload_name(cfg), "tokens": cfg.n_tokens,
+                       "blocks_executed_per_denoise": counts["blocks"],
+                       "block_tokens_per_step": counts["tokens"],
+                       "flops_per_step": counts["flops"],
+                       "l2": "no flush: each pass streams "
+                             f"{sum(p['w_qkv'].numel() + p['w_o'].numel() + p['w_fc1'].numel() + p['w_fc2'].numel() for p in model.params) * 2 / 1e9:.2f}"
+                             " GB of weights, more than the 126 MB L2",
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+            "tflops": tflops,
+            "tensor_frac": tflops / world / peaks["bf16_tflops_sustained"],
+            "tensor_frac_peak": f"{peak_src} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s",
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clk}
+    if breakdown:
+        line["kernels"] = {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
+                               for kk, vv in v.items()} for k, v in breakdown.items()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample(cfg)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

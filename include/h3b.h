@@ -1,0 +1,270 @@
+/*
+ * h3b -- B200 (sm_100a) DiT-block denoising path: public C ABI.
+ *
+ * The library computes the transformer-block forward inside the Euler denoising loop of a
+ * MiniMax-H3-style video+audio diffusion model: AdaLN-modulated LayerNorm, QKV projection,
+ * 3D RoPE over the (t, h, w) token grid, joint video+audio self-attention, an output
+ * projection whose gated residual feeds the MLP's AdaLN, a GELU MLP whose gated residual
+ * feeds the next block's AdaLN, the per-stream final AdaLN and the Euler update; plus
+ * horizontal token pairing and an int8 row-scaled FC2.
+ *
+ * Sources, cited by page title and section:
+ *   "How h3.c cuts MiniMax-H3 video inference to 3.5 seconds" (dothoosh.com), sections
+ *     "DiT fusions and memory management", "Aggressive optimisation levers",
+ *     "The powerful int8 path";
+ *   "H3-metal: running MiniMax-H3 directly on Apple Silicon" (aihot.vn, README
+ *     translation), sections 2 "First fast video", 4 "Speed/quality presets",
+ *     5 "Resolution and duration";
+ *   "h3: native MiniMax-H3 on Apple Silicon" (news.ditty.ir).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller; pointers
+ *     marked "host" are host pointers.  The library never allocates or frees device
+ *     memory except in h3b_denoise_host, which is documented below.
+ *   - Tensors are dense row-major; "[a, b]" means b is the contiguous dimension.
+ *     Every device pointer must be 16-byte aligned.
+ *   - h3b_bf16 is bfloat16 storage (IEEE-754 binary32 with the low 16 bits dropped).
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *     Calls are asynchronous on that stream; no host synchronisation happens inside
+ *     (except h3b_sync_status and h3b_denoise_host).
+ *   - Return value: H3B_OK (0) or a negative H3B_E* code.  All argument validation
+ *     happens before the first launch, so a call that fails validation launches
+ *     nothing.  h3b_last_error() returns a message for the calling thread's last error.
+ *   - Device-side waits inside the kernels give up after about two seconds; the kernel
+ *     then returns early and records the event in a per-device flag, which the next
+ *     h3b_sync_status call reports as H3B_ETIMEOUT.
+ */
+#ifndef H3B_H_
+#define H3B_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define H3B_VERSION 1
+
+enum {
+  H3B_OK = 0,
+  H3B_EINVAL = -1,        /* bad sizes, layout or alignment */
+  H3B_EWORKSPACE = -2,    /* workspace missing or smaller than the size function says */
+  H3B_ECUDA = -3,         /* a CUDA runtime call or kernel launch failed */
+  H3B_ETIMEOUT = -4,      /* a device-side wait gave up (reported by h3b_sync_status) */
+  H3B_EUNSUPPORTED = -5   /* the current device is not sm_100 */
+};
+
+typedef uint16_t h3b_bf16;
+
+/* Model dimensions.  d = n_heads * head_dim; head_dim is 64 or 128; rope_split are the
+ * widths of the (t, h, w) chunks of the head dimension (even, summing to head_dim);
+ * d % 256 == 0, d <= 4096, d_ff % 256 == 0, c_dim % 8 == 0. */
+typedef struct h3b_dims {
+  int d;
+  int n_heads;
+  int head_dim;
+  int d_ff;
+  int c_dim;
+  int rope_split[3];
+  float rope_theta;   /* RoPE base, 10000 in the workloads */
+  float ln_eps;       /* LayerNorm epsilon, 1e-6 */
+} h3b_dims;
+
+/* Token grid: video tokens (t, h, w) in raster order, then n_audio audio tokens.
+ * rope_halved != 0 halves the spatial RoPE coordinates (small-canvas variant: aihot.vn
+ * README section 5).  Audio tokens sit at RoPE position (0, 0, 0). */
+typedef struct h3b_grid {
+  int t, h, w;
+  int n_audio;
+  int rope_halved;
+} h3b_grid;
+
+/* Parameters of one block (device, bf16).  Weights are [out, in]: w_qkv [3d, d] (q rows,
+ * then k, then v; head j at rows j*head_dim), w_o [d, d], w_fc1 [d_ff, d], w_fc2 [d, d_ff];
+ * biases b_qkv [3d], b_o [d], b_fc1 [d_ff], b_fc2 [d]. */
+typedef struct h3b_block_weights {
+  const h3b_bf16* w_qkv;
+  const h3b_bf16* b_qkv;
+  const h3b_bf16* w_o;
+  const h3b_bf16* b_o;
+  const h3b_bf16* w_fc1;
+  const h3b_bf16* b_fc1;
+  const h3b_bf16* w_fc2;
+  const h3b_bf16* b_fc2;
+} h3b_block_weights;
+
+/* ---------------------------------------------------------------- library information */
+int h3b_version(void);
+const char* h3b_last_error(void);
+
+/* Number of kernels this library has launched in this process (all devices, all
+ * threads), for launch accounting by callers. */
+uint64_t h3b_launch_count(void);
+
+/* Synchronise `stream`, then read and clear this device's wait-timeout flag.
+ * Returns H3B_OK, H3B_ETIMEOUT (a kernel gave up waiting; its outputs are invalid) or
+ * H3B_ECUDA (an asynchronous CUDA error). */
+int h3b_sync_status(void* stream);
+
+/* ---------------------------------------------------------------- workspace sizes */
+/* Bytes of workspace h3b_block_forward needs for n_tokens tokens.  One arena, laid out by
+ * lifetime: the QKV and attention-output regions are reused for the MLP hidden
+ * activations (dothoosh.com, "DiT fusions and memory management": activation arenas
+ * aliased by lifetime). */
+size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens);
+
+/* Bytes of workspace h3b_denoise_step needs for this grid; reduce != 0 adds the paired
+ * stream's buffers. */
+size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce);
+
+/* ---------------------------------------------------------------- hot-path steps */
+/* AdaLN modulation vectors: mod[j] = sum_k w[j, k] c[k] + b[j], j < n_out.
+ * w [n_out, c_dim] bf16, b [n_out] bf16, c [c_dim] bf16, mod [n_out] fp32 (all device).
+ * A block's six vectors are rows of mod [6, d] in the order shift_msa, scale_msa,
+ * gate_msa, shift_mlp, scale_mlp, gate_mlp; a stream's final pair is (shift, scale).
+ * (dothoosh.com, "DiT fusions and memory management" and "Aggressive optimisation
+ * levers": per-block AdaLN gates.) */
+int h3b_adaln_modulation(const h3b_bf16* w, const h3b_bf16* b, const h3b_bf16* c,
+                         int n_out, int c_dim, float* mod, void* stream);
+
+/* RoPE cos/sin table for a grid: rope_cs [n_tokens, head_dim / 2, 2] fp32 (device),
+ * entry (i, p) = (cos a, sin a) of pair p of token i.  Pair p lies in the chunk of axis
+ * x (t, h, w in that order); with k its index inside the chunk of width D_x,
+ * a = pos_x(i) * rope_theta^(-2k / D_x).  paired != 0 builds the table of the paired
+ * grid (w / 2 columns, merged token j at w = 2j + 0.5).  n_tokens = t*h*w (or t*h*(w/2)
+ * when paired) + n_audio.  (aihot.vn README section 5: spatial RoPE coordinates.) */
+int h3b_rope_table(const h3b_dims* dims, const h3b_grid* grid, int paired, float* rope_cs,
+                   void* stream);
+
+/* LayerNorm (no affine, biased variance) + AdaLN modulation:
+ * h = LN(x) * (1 + scale) + shift.  x, h [n_tokens, d] bf16; shift, scale [d] fp32.
+ * x and h must not overlap. */
+int h3b_ln_modulate(const h3b_bf16* x, int n_tokens, int d, float eps, const float* shift,
+                    const float* scale, h3b_bf16* h, void* stream);
+
+/* One DiT block (dothoosh.com, "DiT fusions and memory management"):
+ *   h  = LN(x)(1 + scale_msa) + shift_msa          (computed here iff compute_h != 0,
+ *                                                     else h must already hold it)
+ *   qkv = h W_qkv^T + b_qkv; q, k rotated by RoPE (rope_cs from h3b_rope_table)
+ *   o  = softmax(q k^T / sqrt(head_dim)) v           per head, all tokens, no mask
+ *   x  = x + gate_msa (o W_o^T + b_o)                (in place, bf16)
+ *   h  = LN(x)(1 + scale_mlp) + shift_mlp
+ *   x  = x + gate_mlp (GELU_tanh(h W_fc1^T + b_fc1) W_fc2^T + b_fc2)
+ *   h  = LN(x)(1 + mod_next.scale_msa) + mod_next.shift_msa     iff mod_next != NULL
+ * mod, mod_next: [6, d] fp32 device; x, h: [n_tokens, d] bf16 device (in/out);
+ * ws: device workspace of at least h3b_workspace_size(dims, n_tokens) bytes. */
+int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* mod,
+                      const float* mod_next, const float* rope_cs, int n_tokens,
+                      int compute_h, h3b_bf16* x, h3b_bf16* h, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* Per-stream final AdaLN fused with the Euler update (dothoosh.com, "DiT fusions and
+ * memory management": final AdaLN bound to the video/audio offsets of one residual
+ * buffer; aihot.vn section 2: linear sigma grid):
+ *   v = LN(x_l)(1 + scale_s) + shift_s, s = video for rows < n_video, else audio;
+ *   x_state += (sigma_next - sigma) v.
+ * x_l [n_tokens, d] bf16; final_mod [2 streams, 2 (shift, scale), d] fp32;
+ * x_state [n_tokens, d] fp32 (in/out); all device. */
+int h3b_final_euler(const h3b_bf16* x_l, int n_tokens, int n_video, int d, float eps,
+                    const float* final_mod, float sigma, float sigma_next, float* x_state,
+                    void* stream);
+
+/* One Euler step of the denoising loop over all active blocks:
+ *   x = bf16(x_state); for each active block b: h3b_block_forward; after `reduce_after`
+ *   executed blocks (if > 0 and blocks remain) pair horizontal video tokens; restore
+ *   before the final AdaLN (bypass restore if unpair_bypass, else duplicate);
+ *   x_state += (sigma_next - sigma) final_adaln(x).
+ * blocks: host array of n_blocks weight sets; active: host [n_blocks] (NULL = all);
+ * mods: device [n_blocks, 6, d] fp32; final_mod: device [2, 2, d] fp32;
+ * x_state: device [n_tokens, d] fp32, n_tokens = t*h*w + n_audio;
+ * ws: device, at least h3b_denoise_workspace_size(dims, grid, reduce_after > 0).
+ * (ditty.ir and dothoosh.com "Aggressive optimisation levers": token pairing after
+ * block 3, layer thinning; aihot.vn section 2: --steps N means exactly N passes.) */
+int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                     const h3b_block_weights* blocks, const unsigned char* active,
+                     const float* mods, const float* final_mod, int reduce_after,
+                     int unpair_bypass, float sigma, float sigma_next, float* x_state,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Whole denoise from a HOST latent: copies x_host_in [n_tokens, d] fp32 to the device,
+ * runs Euler steps first_step .. first_step + n_run - 1 of the linear grid with n_steps
+ * intervals (sigma_i = 1 - i / n_steps), copies the state back into x_host_out and
+ * synchronises `stream`.  x_state_dev: device [n_tokens, d] fp32 scratch for the state.
+ * Host buffers should be pinned for full copy bandwidth. */
+int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                     const h3b_block_weights* blocks, const unsigned char* active,
+                     const float* mods, const float* final_mod, int reduce_after,
+                     int unpair_bypass, int n_steps, int first_step, int n_run,
+                     const float* x_host_in, float* x_host_out, float* x_state_dev,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Horizontal token pairing (ditty.ir; dothoosh.com "Aggressive optimisation levers").
+ * mode H3B_PAIR:   dst[t,h,j] = (src[t,h,2j] + src[t,h,2j+1]) / 2, audio rows copied;
+ *                  src [t*h*w + n_audio, d], dst [t*h*(w/2) + n_audio, d].
+ * mode H3B_UNPAIR: dst[t,h,2j+k] = saved[t,h,2j+k] + (src[t,h,j] - pair(saved)[t,h,j])
+ *                  when saved != NULL (bypass restore; pair(saved) rounded to bf16 as
+ *                  H3B_PAIR would store it), else dst[t,h,2j+k] = src[t,h,j];
+ *                  audio rows copied; src is the paired stream, dst and saved full.
+ *                  dst may equal saved (in place).
+ * All bf16 device; w must be even; averages and corrections in fp32, one rounding. */
+enum { H3B_PAIR = 0, H3B_UNPAIR = 1 };
+int h3b_token_reduce(int mode, const h3b_bf16* src, h3b_bf16* dst, const h3b_bf16* saved,
+                     int t, int h, int w, int n_audio, int d, void* stream);
+
+/* Symmetric int8 quantisation, one fp32 scale per row (aihot.vn section 4 and
+ * dothoosh.com "The powerful int8 path": one activation scale per FC2 row):
+ * absmax = max|a_row|; q = clamp(rne(a * (127 / absmax)), -127, 127) with IEEE fp32
+ * division and multiply; scale = absmax / 127; a zero row gives q = 0, scale = 0.
+ * a [rows, cols] bf16, q [rows, cols] int8, scale [rows] fp32 (device); cols % 16 == 0.
+ * Used for FC2 activations (rows = tokens) and for weights (rows = output channels). */
+int h3b_quantize_rows(const h3b_bf16* a, int rows, int cols, int8_t* q, float* scale,
+                      void* stream);
+
+/* Int8 row-scaled FC2 with gated residual (aihot.vn section 4, --use-int8-row-fc2):
+ *   act_q, row_scale = h3b_quantize_rows(act);
+ *   acc = act_q w_q^T (int32, exact);  y = float(acc) * row_scale[m] * w_scale[n] (+ bias[n]);
+ *   resid = bf16(resid + gate[n] y).
+ * act [M, K] bf16; w_q [n_out, K] int8; w_scale, gate [n_out] fp32; bias [n_out] fp32 or
+ * NULL; resid [M, n_out] bf16 in/out; act_q [M, K] int8 and row_scale [M] fp32 outputs;
+ * acc_out [M, n_out] int32 output or NULL.  All device.  K % 128 == 0,
+ * n_out % 256 == 0. */
+int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t* w_q,
+                     const float* w_scale, const float* bias, const float* gate,
+                     h3b_bf16* resid, int8_t* act_q, float* row_scale, int32_t* acc_out,
+                     void* stream);
+
+/* ---------------------------------------------------------------- single kernels */
+/* The projection GEMM used by the block: out = A B^T with an epilogue.
+ * A [M, K] bf16, B [N, K] bf16 (device), K % 64 == 0, N % 128 == 0.
+ *   H3B_EPI_BIAS:       out[M, N] = bf16(acc + bias)
+ *   H3B_EPI_BIAS_GELU:  out = bf16(GELU_tanh(acc + bias))
+ *   H3B_EPI_BIAS_ROPE:  out = bf16(rope(acc + bias)) on columns < rope_cols (pairs of
+ *                       adjacent columns, head_dim-periodic, table rope_cs), plain after
+ *   H3B_EPI_GATE_RESID: out = bf16(out + gate (acc + bias)), in place (out is the residual)
+ * bias [N] bf16; gate [N] fp32 (GATE_RESID only); rope_cs as h3b_rope_table. */
+enum { H3B_EPI_BIAS = 0, H3B_EPI_BIAS_GELU = 1, H3B_EPI_BIAS_ROPE = 2, H3B_EPI_GATE_RESID = 3 };
+int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
+                  const h3b_bf16* bias, const float* gate, const float* rope_cs,
+                  int rope_cols, int head_dim, h3b_bf16* out, void* stream);
+
+/* Joint self-attention over one packed QKV buffer: qkv [n_tokens, 3 n_heads head_dim]
+ * bf16 (q, then k, then v; head j at column j*head_dim of each), out [n_tokens,
+ * n_heads head_dim] bf16 (device).  out = softmax(q k^T / sqrt(head_dim)) v per head. */
+int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim,
+                  h3b_bf16* out, void* stream);
+
+/* ---------------------------------------------------------------- host policy */
+/* Layer thinning mask (dothoosh.com "Aggressive optimisation levers": rank blocks by
+ * their AdaLN gates, always keep the first and last block).  score_b = mean|gate_msa| +
+ * mean|gate_mlp| from mods_host [n_blocks, 6, d] fp32 (host); the n_blocks - n_active
+ * lowest-scoring interior blocks are dropped, the higher index first on ties.
+ * mask_out: host [n_blocks], 1 = active. */
+int h3b_layer_mask(const float* mods_host, int n_blocks, int d, int n_active,
+                   unsigned char* mask_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3B_H_ */

@@ -1,0 +1,299 @@
+"""Kernel-level parity: every CUDA kernel of the path alone, through the C ABI, against
+the oracle on the same seeded inputs.  Sizes span several tiles and ragged tails, up to
+the full 512x512-shaped and int8-FC2 workloads."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests.helpers import bf16_bits, max_block_rel_l2, np64, rel_l2, rnd
+
+pytestmark = pytest.mark.gpu
+
+h3b = pytest.importorskip("video_diffusion_transformer_03_b200.h3b")
+
+DEV = "cuda"
+
+
+def _sync():
+    h3b.sync_status()
+
+
+# ------------------------------------------------------------------------------ GEMM
+GEMM_SHAPES = [(40, 768, 256), (200, 256, 128), (300, 384, 192), (1600, 3072, 3072),
+               (1600, 12288, 3072), (1600, 3072, 12288)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("epi", [h3b.EPI_BIAS, h3b.EPI_BIAS_GELU, h3b.EPI_GATE_RESID])
+def test_gemm_epilogues(M, N, K, epi):
+    if (M, N, K) == (1600, 12288, 3072) and epi != h3b.EPI_BIAS_GELU:
+        pytest.skip("FC1 shape is checked with its own epilogue")
+    if (M, N, K) == (1600, 3072, 12288) and epi != h3b.EPI_GATE_RESID:
+        pytest.skip("FC2 shape is checked with its own epilogue")
+    A = rnd((M, K), 1.0, seed=1)
+    B = rnd((N, K), K ** -0.5, seed=2)
+    bias = rnd((N,), 0.1, seed=3)
+    acc = np64(A) @ np64(B).T + np64(bias)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    gate = None
+    if epi == h3b.EPI_BIAS:
+        want = acc
+    elif epi == h3b.EPI_BIAS_GELU:
+        want = O.gelu_tanh(acc)
+    else:
+        resid = rnd((M, N), 1.0, seed=4)
+        g = rnd((N,), 0.5, seed=5, dtype=torch.float32)
+        out.copy_(resid.to(DEV))
+        gate = g.to(DEV)
+        want = O.gated_residual(np64(resid), np64(g), acc)
+    h3b.gemm_bf16(A.to(DEV), B.to(DEV), epi, bias.to(DEV), out, gate=gate)
+    _sync()
+    got = np64(out)
+    assert rel_l2(got, want) < 4e-3
+    assert max_block_rel_l2(got, want) < 8e-3
+
+
+@pytest.mark.parametrize("grid,n_audio,heads,hd,split", [
+    ((2, 4, 4), 8, 4, 64, (16, 24, 24)),
+    ((6, 16, 16), 64, 24, 128, (32, 48, 48)),
+    ((3, 5, 6), 11, 2, 128, (32, 48, 48)),
+])
+def test_gemm_rope_epilogue(grid, n_audio, heads, hd, split):
+    d = heads * hd
+    M = grid[0] * grid[1] * grid[2] + n_audio
+    A = rnd((M, d), 1.0, seed=11)
+    B = rnd((3 * d, d), 0.02, seed=12)
+    bias = rnd((3 * d,), 0.02, seed=13)
+    dims = h3b.make_dims(d, heads, hd, 4 * d, 256, split)
+    g = h3b.make_grid(*grid, n_audio)
+    cs = torch.empty((M, hd // 2, 2), dtype=torch.float32, device=DEV)
+    h3b.rope_table(dims, g, False, cs)
+    out = torch.empty((M, 3 * d), dtype=torch.bfloat16, device=DEV)
+    h3b.gemm_bf16(A.to(DEV), B.to(DEV), h3b.EPI_BIAS_ROPE, bias.to(DEV), out, rope_cs=cs,
+                  rope_cols=2 * d, head_dim=hd)
+    _sync()
+    acc = np64(A) @ np64(B).T + np64(bias)
+    pos = O.rope_positions(grid, n_audio)
+    want = acc.copy()
+    for part in range(2):
+        blk = acc[:, part * d:(part + 1) * d].reshape(M, heads, hd)
+        want[:, part * d:(part + 1) * d] = O.rope_rotate(blk, pos, split, 1e4).reshape(M, d)
+    got = np64(out)
+    assert rel_l2(got, want) < 4e-3
+    assert max_block_rel_l2(got, want) < 8e-3
+
+
+# ------------------------------------------------------------------------------ attention
+ATTN_CASES = [(40, 4, 64, 1.2), (1, 2, 128, 1.0), (128, 1, 128, 1.2), (129, 2, 64, 1.2),
+              (300, 2, 128, 1.2), (300, 2, 128, 3.0), (1600, 24, 128, 1.2), (700, 3, 64, 2.0)]
+
+
+@pytest.mark.parametrize("n,heads,hd,std", ATTN_CASES)
+def test_attention(n, heads, hd, std):
+    d = heads * hd
+    qkv = rnd((n, 3 * d), std, seed=n + heads)
+    out = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.attention(qkv.to(DEV), heads, hd, out)
+    _sync()
+    x = np64(qkv)
+    q, k, v = (x[:, i * d:(i + 1) * d].reshape(n, heads, hd) for i in range(3))
+    want = O.attention(q, k, v).reshape(n, d)
+    got = np64(out)
+    assert rel_l2(got, want) < 1e-2
+    assert max_block_rel_l2(got, want) < 2e-2
+
+
+def test_attention_uniform_keys_average_values():
+    n, heads, hd = 257, 2, 128
+    d = heads * hd
+    qkv = rnd((n, 3 * d), 1.0, seed=7)
+    qkv[:, d:2 * d] = rnd((1, d), 1.0, seed=8)          # every key identical
+    out = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.attention(qkv.to(DEV), heads, hd, out)
+    _sync()
+    want = np.broadcast_to(np64(qkv[:, 2 * d:]).mean(axis=0), (n, d))
+    assert np.max(np.abs(np64(out) - want)) < 2e-2
+
+
+# ------------------------------------------------------------------------------ row kernels
+@pytest.mark.parametrize("n,d,offset", [(5, 256, 0.0), (1000, 3072, 0.0), (77, 3072, 100.0),
+                                        (33, 1024, 0.0)])
+def test_ln_modulate(n, d, offset):
+    x = (rnd((n, d), 1.0, seed=21).float() + offset).to(torch.bfloat16)
+    shift = rnd((d,), 0.3, seed=22, dtype=torch.float32)
+    scale = rnd((d,), 0.3, seed=23, dtype=torch.float32)
+    h = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.ln_modulate(x.to(DEV), 1e-6, shift.to(DEV), scale.to(DEV), h)
+    _sync()
+    want = O.modulate(O.layer_norm(np64(x), 1e-6), np64(shift), np64(scale))
+    got = np64(h)
+    assert rel_l2(got, want) < 4e-3
+    assert max_block_rel_l2(got, want, rows=1) < 8e-3
+
+
+def test_ln_modulate_constant_rows_give_shift():
+    n, d = 9, 512
+    x = torch.full((n, d), 3.25, dtype=torch.bfloat16)
+    shift = rnd((d,), 1.0, seed=24, dtype=torch.float32)
+    scale = rnd((d,), 1.0, seed=25, dtype=torch.float32)
+    h = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.ln_modulate(x.to(DEV), 1e-6, shift.to(DEV), scale.to(DEV), h)
+    _sync()
+    assert np.array_equal(np64(h), np.broadcast_to(np64(shift.to(torch.bfloat16)), (n, d)))
+
+
+@pytest.mark.parametrize("n,n_video,d", [(40, 32, 256), (1600, 1536, 3072), (11344, 11088, 3072)])
+def test_final_euler(n, n_video, d):
+    xl = rnd((n, d), 1.0, seed=31)
+    xs = rnd((n, d), 1.0, seed=32, dtype=torch.float32)
+    fm = rnd((2, 2, d), 0.3, seed=33, dtype=torch.float32)
+    xs_dev = xs.to(DEV)
+    h3b.final_euler(xl.to(DEV), n_video, 1e-6, fm.to(DEV), 0.75, 0.5, xs_dev)
+    _sync()
+    v = O.final_adaln(np64(xl), np64(fm), n_video, 1e-6)
+    want_delta = -0.25 * v
+    got_delta = np64(xs_dev) - np64(xs)
+    assert rel_l2(got_delta, want_delta) < 1e-4
+    xs2 = xs.to(DEV)
+    h3b.final_euler(xl.to(DEV), n_video, 1e-6, fm.to(DEV), 0.5, 0.5, xs2)   # sigma_next == sigma
+    _sync()
+    assert torch.equal(xs2.cpu(), xs)
+
+
+# ------------------------------------------------------------------------------ pairing
+@pytest.mark.parametrize("grid,n_audio,d", [((2, 4, 4), 8, 256), ((6, 16, 16), 64, 3072),
+                                            ((11, 24, 42), 256, 3072), ((1, 1, 2), 0, 8)])
+def test_token_pair_unpair(grid, n_audio, d):
+    t, h, w = grid
+    n = t * h * w + n_audio
+    nr = t * h * (w // 2) + n_audio
+    x = rnd((n, d), 1.0, seed=41)
+    xd = x.to(DEV)
+    red = torch.empty((nr, d), dtype=torch.bfloat16, device=DEV)
+    h3b.token_reduce(h3b.PAIR, xd, red, None, t, h, w, n_audio)
+    _sync()
+    want = O.round_to_bf16(O.token_pair(np64(x), grid, n_audio))
+    assert np.array_equal(np64(red), want.astype(np.float64))          # bit-exact
+    # duplicate restore
+    dup = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.token_reduce(h3b.UNPAIR, red, dup, None, t, h, w, n_audio)
+    _sync()
+    assert np.array_equal(np64(dup), O.token_unpair(np64(red), grid, n_audio))
+    # bypass restore of an unchanged reduced stream returns the saved stream exactly
+    back = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
+    h3b.token_reduce(h3b.UNPAIR, red, back, xd, t, h, w, n_audio)
+    _sync()
+    assert np.array_equal(bf16_bits(back), bf16_bits(x))
+    # bypass restore after an update, in place into the saved buffer
+    upd = (red.float().cpu() + rnd((nr, d), 0.1, seed=42).float()).to(torch.bfloat16)
+    want = O.token_unpair(np64(upd), grid, n_audio, saved=np64(x))
+    inplace = x.to(DEV)
+    h3b.token_reduce(h3b.UNPAIR, upd.to(DEV), inplace, inplace, t, h, w, n_audio)
+    _sync()
+    got = np64(inplace)
+    assert rel_l2(got, want) < 4e-3
+    assert np.array_equal(got[t * h * w:], np64(upd)[t * h * (w // 2):])
+
+
+# ------------------------------------------------------------------------------ int8
+def _quant_input(M, K, seed):
+    z = rnd((M, K), 1.0, seed=seed, dtype=torch.float32)
+    a = torch.nn.functional.gelu(z, approximate="tanh").to(torch.bfloat16)
+    a[0] = 0                                   # zero row
+    if M > 2:
+        a[1] = 0
+        a[1, K // 2] = -3.0                    # single non-zero
+        a[2] = torch.tensor([0.5, -1.0, 0.25, 0.0] * (K // 4), dtype=torch.bfloat16)  # ties
+    return a
+
+
+@pytest.mark.parametrize("M,K", [(5, 16), (300, 384), (64, 12288), (33, 3072)])
+def test_quantize_rows_bit_exact(M, K):
+    a = _quant_input(M, K, seed=M + K)
+    q = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    s = torch.empty((M,), dtype=torch.float32, device=DEV)
+    h3b.quantize_rows(a.to(DEV), q, s)
+    _sync()
+    wq, ws = O.quantize_rows(a.float().numpy())
+    assert np.array_equal(q.cpu().numpy(), wq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+
+
+def _fc2_case(M, K, N, with_bias, sample_rows=None, seed=50):
+    a = _quant_input(M, K, seed)
+    w = rnd((N, K), 0.02, seed=seed + 1)
+    gate = rnd((N,), 1.0, seed=seed + 2, dtype=torch.float32)
+    resid = rnd((M, N), 1.0, seed=seed + 3)
+    bias = rnd((N,), 0.02, seed=seed + 4, dtype=torch.float32) if with_bias else None
+    # weights quantised per output channel on the GPU (bit-exact with the oracle)
+    wq = torch.empty((N, K), dtype=torch.int8, device=DEV)
+    wsc = torch.empty((N,), dtype=torch.float32, device=DEV)
+    h3b.quantize_rows(w.to(DEV), wq, wsc)
+    aq = torch.empty((M, K), dtype=torch.int8, device=DEV)
+    rs = torch.empty((M,), dtype=torch.float32, device=DEV)
+    acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
+    out = resid.to(DEV)
+    h3b.fc2_int8_row(a.to(DEV), wq, wsc, None if bias is None else bias.to(DEV), gate.to(DEV),
+                     out, aq, rs, acc)
+    _sync()
+    owq, ows = O.quantize_rows(w.float().numpy())
+    assert np.array_equal(wq.cpu().numpy(), owq)
+    assert np.array_equal(wsc.cpu().numpy().view(np.uint32), ows.view(np.uint32))
+    rows = np.arange(M) if sample_rows is None else sample_rows
+    q, s_r, acc_o, out_o = O.fc2_int8_row(a.float().numpy(), owq, ows, np64(gate), np64(resid),
+                                          None if bias is None else np64(bias), rows=rows)
+    assert np.array_equal(aq.cpu().numpy()[rows], q)
+    assert np.array_equal(rs.cpu().numpy()[rows].view(np.uint32), s_r.view(np.uint32))
+    assert np.array_equal(acc.cpu().numpy()[rows].astype(np.int64), acc_o)      # bit-exact int32
+    got = np64(out)[rows]
+    assert rel_l2(got, out_o) < 4e-3
+    return acc
+
+
+@pytest.mark.parametrize("M,K,N,bias", [(300, 384, 256, False), (130, 12288, 384, True),
+                                        (257, 1024, 512, True)])
+def test_fc2_int8_row_small(M, K, N, bias):
+    _fc2_case(M, K, N, bias)
+
+
+def test_fc2_int8_row_full_size():
+    M, K, N = 8192, 12288, 3072
+    rows = np.unique(np.concatenate([np.arange(0, 4), np.linspace(5, M - 1, 40).astype(int),
+                                     np.arange(M - 4, M)]))
+    _fc2_case(M, K, N, False, sample_rows=rows, seed=4)
+
+
+# ------------------------------------------------------------------------------ setup kernels
+def test_adaln_modulation():
+    d, c = 256, 256
+    w = rnd((6 * d, c), 0.02, seed=61)
+    b = rnd((6 * d,), 0.02, seed=62)
+    cv = rnd((c,), 1.0, seed=63)
+    out = torch.empty((6, d), dtype=torch.float32, device=DEV)
+    h3b.adaln_modulation(w.to(DEV), b.to(DEV), cv.to(DEV), out)
+    _sync()
+    want = O.adaln_modulation(np64(w), np64(b), np64(cv), d)
+    assert rel_l2(np64(out), want) < 1e-5
+
+
+@pytest.mark.parametrize("grid,n_audio,halved,paired,hd,split", [
+    ((6, 16, 16), 64, False, False, 128, (32, 48, 48)),
+    ((6, 16, 16), 64, False, True, 128, (32, 48, 48)),
+    ((6, 8, 8), 64, True, False, 128, (32, 48, 48)),
+    ((2, 4, 4), 8, False, False, 64, (16, 24, 24)),
+    ((11, 24, 42), 256, False, False, 128, (32, 48, 48)),
+])
+def test_rope_table(grid, n_audio, halved, paired, hd, split):
+    heads = 256 // hd * 2
+    dims = h3b.make_dims(hd * heads, heads, hd, 1024, 256, split)
+    g = h3b.make_grid(*grid, n_audio, halved)
+    pos = O.rope_positions(grid, n_audio, halved=halved, paired=paired)
+    n = pos.shape[0]
+    cs = torch.empty((n, hd // 2, 2), dtype=torch.float32, device=DEV)
+    h3b.rope_table(dims, g, paired, cs)
+    _sync()
+    unit = np.zeros((n, 1, hd))
+    unit[..., 0::2] = 1.0
+    want = O.rope_rotate(unit, pos, split, 1e4).reshape(n, hd // 2, 2)
+    assert np.max(np.abs(cs.cpu().numpy().astype(np.float64) - want)) < 2e-6

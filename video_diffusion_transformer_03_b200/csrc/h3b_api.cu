@@ -1,0 +1,596 @@
+// C ABI of the h3b library: argument validation, workspace layout and the order of the
+// kernels inside a DiT block and an Euler step.  See include/h3b.h for the contract of
+// every entry point.
+#include "../../include/h3b.h"
+#include "kernels.h"
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+// Set (first code wins) by any kernel whose bounded wait gave up; one per device.
+__device__ uint32_t g_h3b_wait_error = 0u;
+
+namespace h3b {
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+std::atomic<uint64_t> g_launches{0};
+
+bool debug_mode() {
+  static const bool on = [] {
+    const char* v = std::getenv("H3B_DEBUG");
+    return v && v[0] && v[0] != '0';
+  }();
+  return on;
+}
+
+constexpr int kMaxDevices = 64;
+
+}  // namespace
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int check_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  if (debug_mode()) {
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess)
+      return set_error(H3B_ECUDA, "%s: kernel failed: %s", what, cudaGetErrorString(e));
+    uint32_t flag = 0;
+    cudaMemcpyFromSymbol(&flag, g_h3b_wait_error, sizeof(flag));
+    if (flag) return set_error(H3B_ETIMEOUT, "%s: device wait gave up (code %u)", what, flag);
+  }
+  return H3B_OK;
+}
+
+namespace {
+
+int get_ctx(DevCtx* ctx) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return set_error(H3B_EUNSUPPORTED, "device %d", dev);
+  static std::mutex mu;
+  static DevCtx cache[kMaxDevices];
+  static bool have[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (major != 10 || minor != 0)
+      return set_error(H3B_EUNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                       dev, major, minor);
+    void* flag = nullptr;
+    e = cudaGetSymbolAddress(&flag, g_h3b_wait_error);
+    if (e != cudaSuccess)
+      return set_error(H3B_ECUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    cache[dev] = DevCtx{dev, sms, static_cast<uint32_t*>(flag)};
+    have[dev] = true;
+  }
+  *ctx = cache[dev];
+  return H3B_OK;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t a256(size_t b) { return (b + 255) & ~size_t(255); }
+
+int check_dims(const h3b_dims* d) {
+  if (!d) return set_error(H3B_EINVAL, "dims is NULL");
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return set_error(H3B_EINVAL, "head_dim %d must be 64 or 128", d->head_dim);
+  if (d->n_heads <= 0 || d->d != d->n_heads * d->head_dim)
+    return set_error(H3B_EINVAL, "d=%d must equal n_heads*head_dim", d->d);
+  if (d->d % 256 != 0 || d->d > 4096)
+    return set_error(H3B_EINVAL, "d=%d must be a multiple of 256 and <= 4096", d->d);
+  if (d->d_ff <= 0 || d->d_ff % 256 != 0)
+    return set_error(H3B_EINVAL, "d_ff=%d must be a positive multiple of 256", d->d_ff);
+  if (d->c_dim <= 0 || d->c_dim % 8 != 0)
+    return set_error(H3B_EINVAL, "c_dim=%d must be a positive multiple of 8", d->c_dim);
+  const int* s = d->rope_split;
+  if (s[0] < 0 || s[1] < 0 || s[2] < 0 || (s[0] | s[1] | s[2]) & 1 ||
+      s[0] + s[1] + s[2] != d->head_dim)
+    return set_error(H3B_EINVAL, "rope_split (%d,%d,%d) must be even and sum to head_dim",
+                     s[0], s[1], s[2]);
+  if (!(d->ln_eps > 0.f) || !(d->rope_theta > 0.f))
+    return set_error(H3B_EINVAL, "ln_eps and rope_theta must be positive");
+  return H3B_OK;
+}
+
+int check_grid(const h3b_grid* g, bool need_even_w) {
+  if (!g) return set_error(H3B_EINVAL, "grid is NULL");
+  if (g->t < 0 || g->h < 0 || g->w < 0 || g->n_audio < 0)
+    return set_error(H3B_EINVAL, "grid sizes must be non-negative");
+  if (need_even_w && (g->w & 1)) return set_error(H3B_EINVAL, "w=%d must be even to pair tokens", g->w);
+  const long long n = 1LL * g->t * g->h * g->w + g->n_audio;
+  if (n > (1LL << 24)) return set_error(H3B_EINVAL, "too many tokens (%lld)", n);
+  return H3B_OK;
+}
+
+int check_weights(const h3b_block_weights* w) {
+  if (!w) return set_error(H3B_EINVAL, "weights NULL");
+  const void* p[8] = {w->w_qkv, w->b_qkv, w->w_o, w->b_o, w->w_fc1, w->b_fc1, w->w_fc2, w->b_fc2};
+  for (const void* q : p)
+    if (!q || !al16(q)) return set_error(H3B_EINVAL, "block weight pointer NULL or not 16-byte aligned");
+  return H3B_OK;
+}
+
+size_t arena_bytes(const h3b_dims* d, int n) {
+  return a256(size_t(n) * std::max(4 * d->d, d->d_ff) * 2);
+}
+
+// Buffers of one block inside the arena: qkv [n, 3d] then attention output [n, d]; the
+// MLP hidden activations [n, d_ff] reuse the same bytes once both are dead.
+struct BlockBufs {
+  bf16* qkv;
+  bf16* attn;
+  bf16* g;
+};
+
+BlockBufs carve_block(const h3b_dims* d, int n, void* arena) {
+  bf16* base = static_cast<bf16*>(arena);
+  return BlockBufs{base, base + size_t(n) * 3 * d->d, base};
+}
+
+int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_weights* w,
+                       const float* mod, const float* mod_next, const float* rope_cs, int n,
+                       bool compute_h, bf16* x, bf16* h, void* arena, cudaStream_t s) {
+  const int D = d->d;
+  const BlockBufs b = carve_block(d, n, arena);
+  int rc;
+  if (compute_h && (rc = launch_ln_modulate(x, n, D, d->ln_eps, mod, mod + D, h, s))) return rc;
+
+  GemmEpilogue e;
+  e.kind = kEpiRope;
+  e.bias = reinterpret_cast<const bf16*>(w->b_qkv);
+  e.rope_cs = rope_cs;
+  e.rope_cols = 2 * D;
+  e.head_dim = d->head_dim;
+  e.out = b.qkv;
+  e.ld_out = 3 * D;
+  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_qkv), n, 3 * D, D, e, s)))
+    return rc;
+  if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, s))) return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGateResid;
+  e.bias = reinterpret_cast<const bf16*>(w->b_o);
+  e.gate = mod + 2 * D;
+  e.out = x;
+  e.ld_out = D;
+  if ((rc = launch_gemm_bf16(ctx, b.attn, reinterpret_cast<const bf16*>(w->w_o), n, D, D, e, s)))
+    return rc;
+  if ((rc = launch_ln_modulate(x, n, D, d->ln_eps, mod + 3 * D, mod + 4 * D, h, s))) return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGelu;
+  e.bias = reinterpret_cast<const bf16*>(w->b_fc1);
+  e.out = b.g;
+  e.ld_out = d->d_ff;
+  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_fc1), n, d->d_ff, D, e, s)))
+    return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGateResid;
+  e.bias = reinterpret_cast<const bf16*>(w->b_fc2);
+  e.gate = mod + 5 * D;
+  e.out = x;
+  e.ld_out = D;
+  if ((rc = launch_gemm_bf16(ctx, b.g, reinterpret_cast<const bf16*>(w->w_fc2), n, D, d->d_ff, e, s)))
+    return rc;
+  if (mod_next && (rc = launch_ln_modulate(x, n, D, d->ln_eps, mod_next, mod_next + D, h, s)))
+    return rc;
+  return H3B_OK;
+}
+
+// Workspace of one denoise step.
+struct StepBufs {
+  bf16* x_res;      // [N, d] residual stream (bf16)
+  bf16* h;          // [N, d] AdaLN output feeding the next projection
+  float* rope;      // [N, hd/2, 2]
+  float* rope_red;  // [N_red, hd/2, 2]
+  bf16* x_red;      // [N_red, d]
+  void* arena;      // block arena sized for N tokens
+  size_t total;
+};
+
+StepBufs carve_step(const h3b_dims* d, const h3b_grid* g, bool reduce, void* ws) {
+  const size_t n = size_t(g->t) * g->h * g->w + g->n_audio;
+  const size_t nr = size_t(g->t) * g->h * (g->w / 2) + g->n_audio;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  StepBufs b{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* q = p ? p + off : nullptr;
+    off += a256(bytes);
+    return q;
+  };
+  b.x_res = reinterpret_cast<bf16*>(take(n * d->d * 2));
+  b.h = reinterpret_cast<bf16*>(take(n * d->d * 2));
+  b.rope = reinterpret_cast<float*>(take(n * d->head_dim * 4));
+  if (reduce) {
+    b.rope_red = reinterpret_cast<float*>(take(nr * d->head_dim * 4));
+    b.x_red = reinterpret_cast<bf16*>(take(nr * d->d * 2));
+  }
+  b.arena = take(arena_bytes(d, static_cast<int>(n)));
+  b.total = off;
+  return b;
+}
+
+int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, int n_blocks,
+                      const h3b_block_weights* blocks, const unsigned char* active,
+                      const float* mods, const float* final_mod, int reduce_after,
+                      int unpair_bypass, float sigma, float sigma_next, float* x_state,
+                      const StepBufs& b, cudaStream_t s) {
+  const int D = d->d;
+  const int nv = g->t * g->h * g->w;
+  const int n = nv + g->n_audio;
+  const int n_red = g->t * g->h * (g->w / 2) + g->n_audio;
+  const bool may_reduce = reduce_after > 0;
+  int rc;
+  if ((rc = launch_rope_table(g->t, g->h, g->w, g->n_audio, g->rope_halved, 0, d->head_dim,
+                              d->rope_split, d->rope_theta, b.rope, s)))
+    return rc;
+  if (may_reduce &&
+      (rc = launch_rope_table(g->t, g->h, g->w, g->n_audio, g->rope_halved, 1, d->head_dim,
+                              d->rope_split, d->rope_theta, b.rope_red, s)))
+    return rc;
+
+  std::vector<int> order;
+  for (int i = 0; i < n_blocks; ++i)
+    if (!active || active[i]) order.push_back(i);
+  const float* first_mod = order.empty() ? final_mod : mods + size_t(order[0]) * 6 * D;
+  if ((rc = launch_ln_modulate_from_state(x_state, n, D, d->ln_eps, first_mod, first_mod + D,
+                                          b.x_res, b.h, s)))
+    return rc;
+
+  bf16* cur = b.x_res;
+  int cur_n = n;
+  const float* rope = b.rope;
+  for (size_t k = 0; k < order.size(); ++k) {
+    const int blk = order[k];
+    const bool has_next = k + 1 < order.size();
+    const bool pair_now = may_reduce && int(k + 1) == reduce_after && has_next;
+    const float* mod = mods + size_t(blk) * 6 * D;
+    const float* mod_next = (has_next && !pair_now) ? mods + size_t(order[k + 1]) * 6 * D : nullptr;
+    if ((rc = block_forward_impl(ctx, d, &blocks[blk], mod, mod_next, rope, cur_n, false, cur,
+                                 b.h, b.arena, s)))
+      return rc;
+    if (pair_now) {
+      if ((rc = launch_token_pair(b.x_res, b.x_red, g->t, g->h, g->w, g->n_audio, D, s)))
+        return rc;
+      cur = b.x_red;
+      cur_n = n_red;
+      rope = b.rope_red;
+      const float* nm = mods + size_t(order[k + 1]) * 6 * D;
+      if ((rc = launch_ln_modulate(cur, cur_n, D, d->ln_eps, nm, nm + D, b.h, s))) return rc;
+    }
+  }
+  if (cur == b.x_red &&
+      (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
+                                g->w, g->n_audio, D, s)))
+    return rc;
+  return launch_final_euler(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma, x_state, s);
+}
+
+int check_step_args(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                    const h3b_block_weights* blocks, const unsigned char* active,
+                    const float* mods, const float* final_mod, int reduce_after,
+                    const float* x_state, void* ws, size_t ws_bytes, StepBufs* bufs) {
+  int rc;
+  if ((rc = check_dims(dims))) return rc;
+  if ((rc = check_grid(grid, reduce_after > 0))) return rc;
+  if (n_blocks < 0 || (n_blocks > 0 && !blocks)) return set_error(H3B_EINVAL, "bad block list");
+  for (int i = 0; i < n_blocks; ++i)
+    if ((!active || active[i]) && (rc = check_weights(&blocks[i]))) return rc;
+  if (!mods && n_blocks > 0) return set_error(H3B_EINVAL, "mods is NULL");
+  if (!final_mod || !x_state || !al16(mods) || !al16(final_mod) || !al16(x_state))
+    return set_error(H3B_EINVAL, "final_mod / x_state NULL or not 16-byte aligned");
+  const StepBufs need = carve_step(dims, grid, reduce_after > 0, nullptr);
+  if (!ws || !al16(ws) || ws_bytes < need.total)
+    return set_error(H3B_EWORKSPACE, "workspace of %zu bytes needed, %zu given", need.total, ws_bytes);
+  *bufs = carve_step(dims, grid, reduce_after > 0, ws);
+  return H3B_OK;
+}
+
+}  // namespace
+}  // namespace h3b
+
+using namespace h3b;
+
+// ============================================================================ C ABI
+extern "C" {
+
+int h3b_version(void) { return H3B_VERSION; }
+
+const char* h3b_last_error(void) { return g_last_error; }
+
+uint64_t h3b_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int h3b_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "stream sync: %s", cudaGetErrorString(e));
+  uint32_t flag = 0;
+  e = cudaMemcpyFromSymbol(&flag, g_h3b_wait_error, sizeof(flag));
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "read wait flag: %s", cudaGetErrorString(e));
+  if (flag) {
+    const uint32_t zero = 0;
+    cudaMemcpyToSymbol(g_h3b_wait_error, &zero, sizeof(zero));
+    return set_error(H3B_ETIMEOUT, "a device-side wait gave up (code %u)", flag);
+  }
+  return H3B_OK;
+}
+
+size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens) {
+  if (check_dims(dims) || n_tokens < 0) return 0;
+  return arena_bytes(dims, n_tokens);
+}
+
+size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce) {
+  if (check_dims(dims) || check_grid(grid, reduce != 0)) return 0;
+  return carve_step(dims, grid, reduce != 0, nullptr).total;
+}
+
+int h3b_adaln_modulation(const h3b_bf16* w, const h3b_bf16* b, const h3b_bf16* c, int n_out,
+                         int c_dim, float* mod, void* stream) {
+  if (!w || !b || !c || !mod || !al16(w) || !al16(c))
+    return set_error(H3B_EINVAL, "adaln_modulation: NULL or misaligned pointer");
+  if (n_out < 0 || c_dim <= 0 || c_dim % 8)
+    return set_error(H3B_EINVAL, "adaln_modulation: c_dim=%d must be a positive multiple of 8", c_dim);
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_adaln_gemv(reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+                           reinterpret_cast<const bf16*>(c), n_out, c_dim, mod,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int h3b_rope_table(const h3b_dims* dims, const h3b_grid* grid, int paired, float* rope_cs,
+                   void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_grid(grid, paired != 0))) return rc;
+  if (!rope_cs || !al16(rope_cs)) return set_error(H3B_EINVAL, "rope_table: bad output pointer");
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return launch_rope_table(grid->t, grid->h, grid->w, grid->n_audio, grid->rope_halved,
+                           paired != 0, dims->head_dim, dims->rope_split, dims->rope_theta,
+                           rope_cs, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_ln_modulate(const h3b_bf16* x, int n_tokens, int d, float eps, const float* shift,
+                    const float* scale, h3b_bf16* h, void* stream) {
+  if (n_tokens < 0 || d <= 0 || d % 256 || d > 4096)
+    return set_error(H3B_EINVAL, "ln_modulate: d=%d must be a multiple of 256 <= 4096", d);
+  if (!x || !h || !shift || !scale || !al16(x) || !al16(h) || !al16(shift) || !al16(scale))
+    return set_error(H3B_EINVAL, "ln_modulate: NULL or misaligned pointer");
+  if (!(eps > 0.f)) return set_error(H3B_EINVAL, "ln_modulate: eps must be positive");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_ln_modulate(reinterpret_cast<const bf16*>(x), n_tokens, d, eps, shift, scale,
+                            reinterpret_cast<bf16*>(h), static_cast<cudaStream_t>(stream));
+}
+
+int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const float* mod,
+                      const float* mod_next, const float* rope_cs, int n_tokens, int compute_h,
+                      h3b_bf16* x, h3b_bf16* h, void* ws, size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_weights(w))) return rc;
+  if (n_tokens < 0 || n_tokens > (1 << 24)) return set_error(H3B_EINVAL, "n_tokens=%d", n_tokens);
+  if (!mod || !rope_cs || !x || !h || !al16(mod) || !al16(rope_cs) || !al16(x) || !al16(h) ||
+      (mod_next && !al16(mod_next)))
+    return set_error(H3B_EINVAL, "block_forward: NULL or misaligned pointer");
+  if (!ws || !al16(ws) || ws_bytes < arena_bytes(dims, n_tokens))
+    return set_error(H3B_EWORKSPACE, "block_forward: workspace of %zu bytes needed, %zu given",
+                     arena_bytes(dims, n_tokens), ws_bytes);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return block_forward_impl(ctx, dims, w, mod, mod_next, rope_cs, n_tokens, compute_h != 0,
+                            reinterpret_cast<bf16*>(x), reinterpret_cast<bf16*>(h), ws,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int h3b_final_euler(const h3b_bf16* x_l, int n_tokens, int n_video, int d, float eps,
+                    const float* final_mod, float sigma, float sigma_next, float* x_state,
+                    void* stream) {
+  if (n_tokens < 0 || n_video < 0 || n_video > n_tokens || d <= 0 || d % 256 || d > 4096)
+    return set_error(H3B_EINVAL, "final_euler: bad sizes (n=%d n_video=%d d=%d)", n_tokens, n_video, d);
+  if (!x_l || !final_mod || !x_state || !al16(x_l) || !al16(final_mod) || !al16(x_state))
+    return set_error(H3B_EINVAL, "final_euler: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_final_euler(reinterpret_cast<const bf16*>(x_l), n_tokens, n_video, d, eps,
+                            final_mod, sigma_next - sigma, x_state,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                     const h3b_block_weights* blocks, const unsigned char* active,
+                     const float* mods, const float* final_mod, int reduce_after,
+                     int unpair_bypass, float sigma, float sigma_next, float* x_state,
+                     void* ws, size_t ws_bytes, void* stream) {
+  StepBufs b;
+  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
+                           x_state, ws, ws_bytes, &b);
+  if (rc) return rc;
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                           reduce_after, unpair_bypass, sigma, sigma_next, x_state, b,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                     const h3b_block_weights* blocks, const unsigned char* active,
+                     const float* mods, const float* final_mod, int reduce_after,
+                     int unpair_bypass, int n_steps, int first_step, int n_run,
+                     const float* x_host_in, float* x_host_out, float* x_state_dev,
+                     void* ws, size_t ws_bytes, void* stream) {
+  StepBufs b;
+  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
+                           x_state_dev, ws, ws_bytes, &b);
+  if (rc) return rc;
+  if (!x_host_in || !x_host_out) return set_error(H3B_EINVAL, "denoise_host: NULL host buffer");
+  if (n_steps <= 0 || first_step < 0 || n_run < 0 || first_step + n_run > n_steps)
+    return set_error(H3B_EINVAL, "denoise_host: steps %d..%d of %d", first_step,
+                     first_step + n_run, n_steps);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t(grid->t) * grid->h * grid->w + grid->n_audio) * dims->d * 4;
+  cudaError_t e = cudaMemcpyAsync(x_state_dev, x_host_in, bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host H2D: %s", cudaGetErrorString(e));
+  for (int i = first_step; i < first_step + n_run; ++i) {
+    const float sg = static_cast<float>(1.0 - double(i) / n_steps);
+    const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
+    if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                                reduce_after, unpair_bypass, sg, sn, x_state_dev, b, s)))
+      return rc;
+  }
+  e = cudaMemcpyAsync(x_host_out, x_state_dev, bytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host D2H: %s", cudaGetErrorString(e));
+  return h3b_sync_status(stream);
+}
+
+int h3b_token_reduce(int mode, const h3b_bf16* src, h3b_bf16* dst, const h3b_bf16* saved, int t,
+                     int h, int w, int n_audio, int d, void* stream) {
+  if (mode != H3B_PAIR && mode != H3B_UNPAIR) return set_error(H3B_EINVAL, "token_reduce: mode %d", mode);
+  if (t < 0 || h < 0 || w < 0 || (w & 1) || n_audio < 0 || d <= 0 || d % 8)
+    return set_error(H3B_EINVAL, "token_reduce: bad sizes (t=%d h=%d w=%d audio=%d d=%d)", t, h, w, n_audio, d);
+  if (!src || !dst || !al16(src) || !al16(dst) || (saved && !al16(saved)))
+    return set_error(H3B_EINVAL, "token_reduce: NULL or misaligned pointer");
+  if (mode == H3B_PAIR && saved) return set_error(H3B_EINVAL, "token_reduce: saved is for UNPAIR");
+  if (src == dst) return set_error(H3B_EINVAL, "token_reduce: src and dst must differ");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mode == H3B_PAIR)
+    return launch_token_pair(reinterpret_cast<const bf16*>(src), reinterpret_cast<bf16*>(dst), t,
+                             h, w, n_audio, d, s);
+  return launch_token_unpair(reinterpret_cast<const bf16*>(src), reinterpret_cast<bf16*>(dst),
+                             reinterpret_cast<const bf16*>(saved), t, h, w, n_audio, d, s);
+}
+
+int h3b_quantize_rows(const h3b_bf16* a, int rows, int cols, int8_t* q, float* scale,
+                      void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 || cols > 32768)
+    return set_error(H3B_EINVAL, "quantize_rows: cols=%d must be a multiple of 16 <= 32768", cols);
+  if (!a || !q || !scale || !al16(a) || !al16(q))
+    return set_error(H3B_EINVAL, "quantize_rows: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_quantize_rows(reinterpret_cast<const bf16*>(a), rows, cols, q, scale,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t* w_q,
+                     const float* w_scale, const float* bias, const float* gate, h3b_bf16* resid,
+                     int8_t* act_q, float* row_scale, int32_t* acc_out, void* stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > 32768 || n_out <= 0 || n_out % 128)
+    return set_error(H3B_EINVAL, "fc2_int8_row: K=%d must be a multiple of 128 <= 32768, n_out=%d a multiple of 128", K, n_out);
+  const void* ptrs[7] = {act, w_q, w_scale, gate, resid, act_q, row_scale};
+  for (const void* p : ptrs)
+    if (!p || !al16(p)) return set_error(H3B_EINVAL, "fc2_int8_row: NULL or misaligned pointer");
+  if ((bias && !al16(bias)) || (acc_out && !al16(acc_out)))
+    return set_error(H3B_EINVAL, "fc2_int8_row: misaligned bias / acc_out");
+  DevCtx ctx;
+  int rc;
+  if ((rc = get_ctx(&ctx))) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = launch_quantize_rows(reinterpret_cast<const bf16*>(act), M, K, act_q, row_scale, s)))
+    return rc;
+  GemmEpilogue e;
+  e.kind = kEpiInt8Deq;
+  e.bias_f32 = bias;
+  e.gate = gate;
+  e.out = reinterpret_cast<bf16*>(resid);
+  e.ld_out = n_out;
+  e.row_scale = row_scale;
+  e.col_scale = w_scale;
+  e.acc_out = acc_out;
+  return launch_gemm_i8(ctx, act_q, w_q, M, n_out, K, e, s);
+}
+
+int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
+                  const h3b_bf16* bias, const float* gate, const float* rope_cs, int rope_cols,
+                  int head_dim, h3b_bf16* out, void* stream) {
+  if (M < 0 || K <= 0 || K % 64 || N <= 0 || N % 128)
+    return set_error(H3B_EINVAL, "gemm_bf16: K=%d must be a multiple of 64, N=%d of 128", K, N);
+  if (epilogue < H3B_EPI_BIAS || epilogue > H3B_EPI_GATE_RESID)
+    return set_error(H3B_EINVAL, "gemm_bf16: epilogue %d", epilogue);
+  if (!A || !B || !bias || !out || !al16(A) || !al16(B) || !al16(bias) || !al16(out))
+    return set_error(H3B_EINVAL, "gemm_bf16: NULL or misaligned pointer");
+  if (epilogue == H3B_EPI_GATE_RESID && (!gate || !al16(gate)))
+    return set_error(H3B_EINVAL, "gemm_bf16: gate required");
+  if (epilogue == H3B_EPI_BIAS_ROPE &&
+      (!rope_cs || !al16(rope_cs) || (head_dim != 64 && head_dim != 128) || rope_cols < 0 ||
+       rope_cols % head_dim || rope_cols > N))
+    return set_error(H3B_EINVAL, "gemm_bf16: bad RoPE arguments");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  GemmEpilogue e;
+  e.kind = epilogue;
+  e.bias = reinterpret_cast<const bf16*>(bias);
+  e.gate = gate;
+  e.rope_cs = rope_cs;
+  e.rope_cols = rope_cols;
+  e.head_dim = head_dim;
+  e.out = reinterpret_cast<bf16*>(out);
+  e.ld_out = N;
+  return launch_gemm_bf16(ctx, reinterpret_cast<const bf16*>(A), reinterpret_cast<const bf16*>(B),
+                          M, N, K, e, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim, h3b_bf16* out,
+                  void* stream) {
+  if (n_tokens < 0 || n_heads <= 0 || (head_dim != 64 && head_dim != 128))
+    return set_error(H3B_EINVAL, "attention: bad sizes (n=%d heads=%d hd=%d)", n_tokens, n_heads, head_dim);
+  if (!qkv || !out || !al16(qkv) || !al16(out))
+    return set_error(H3B_EINVAL, "attention: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_attention(ctx, reinterpret_cast<const bf16*>(qkv), n_tokens, n_heads, head_dim,
+                          reinterpret_cast<bf16*>(out), static_cast<cudaStream_t>(stream));
+}
+
+int h3b_layer_mask(const float* mods_host, int n_blocks, int d, int n_active,
+                   unsigned char* mask_out) {
+  if (!mods_host || !mask_out || n_blocks <= 0 || d <= 0)
+    return set_error(H3B_EINVAL, "layer_mask: bad arguments");
+  const int n_drop = n_blocks - n_active;
+  if (n_drop > 0 && n_drop > n_blocks - 2)
+    return set_error(H3B_EINVAL, "layer_mask: the first and last blocks are always kept");
+  for (int b = 0; b < n_blocks; ++b) mask_out[b] = 1;
+  if (n_drop <= 0) return H3B_OK;
+  std::vector<std::pair<double, int>> score;
+  for (int b = 1; b < n_blocks - 1; ++b) {
+    const float* m = mods_host + size_t(b) * 6 * d;
+    double ga = 0.0, gm = 0.0;
+    for (int j = 0; j < d; ++j) {
+      ga += std::fabs(double(m[2 * d + j]));
+      gm += std::fabs(double(m[5 * d + j]));
+    }
+    score.emplace_back(ga / d + gm / d, b);
+  }
+  std::sort(score.begin(), score.end(), [](const auto& a, const auto& b) {
+    return a.first != b.first ? a.first < b.first : a.second > b.second;
+  });
+  for (int i = 0; i < n_drop; ++i) mask_out[score[i].second] = 0;
+  return H3B_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// Internal launcher interface between the C ABI (h3b_api.cu) and the kernel translation
+// units.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace h3b {
+
+using bf16 = __nv_bfloat16;
+
+// Per-device facts the launchers need.
+struct DevCtx {
+  int device;
+  int num_sms;
+  uint32_t* err_flag;  // device address of this device's wait-timeout flag
+};
+
+// Record a message for h3b_last_error (thread-local) and return `code`.
+int set_error(int code, const char* fmt, ...);
+
+// Check the launch that just happened; returns 0 or H3B_ECUDA with a message.
+int check_launch(const char* what);
+
+// ---------------------------------------------------------------- GEMM (tcgen05)
+enum GemmEpi : int {
+  kEpiBias = 0,       // out = bf16(acc + bias)
+  kEpiGelu = 1,       // out = bf16(gelu_tanh(acc + bias))
+  kEpiRope = 2,       // out = bf16(rope(acc + bias)) on columns < rope_cols
+  kEpiGateResid = 3,  // out = bf16(out + gate * (acc + bias))
+  kEpiInt8Deq = 4,    // int8 path: out = bf16(out + gate * (acc * row_scale * col_scale + bias))
+};
+
+struct GemmEpilogue {
+  int kind = kEpiBias;
+  const bf16* bias = nullptr;        // bf16 paths, [N]
+  const float* bias_f32 = nullptr;   // int8 path, [N] or null
+  const float* gate = nullptr;       // [N]
+  const float* rope_cs = nullptr;    // [M, head_dim/2, 2]
+  int rope_cols = 0;
+  int head_dim = 128;
+  bf16* out = nullptr;               // [M, ld_out]
+  int ld_out = 0;
+  const float* row_scale = nullptr;  // int8 path, [M]
+  const float* col_scale = nullptr;  // int8 path, [N]
+  int32_t* acc_out = nullptr;        // int8 path, [M, N] or null
+};
+
+// out = A[M, K] * B[N, K]^T with epilogue; bf16 inputs.  K % 64 == 0, N % 128 == 0.
+int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
+                     const GemmEpilogue& epi, cudaStream_t stream);
+// Same for int8 inputs (int32 accumulate, kEpiInt8Deq).  K % 128 == 0, N % 128 == 0.
+int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
+                   const GemmEpilogue& epi, cudaStream_t stream);
+
+// ---------------------------------------------------------------- attention (tcgen05)
+int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_heads,
+                     int head_dim, bf16* out, cudaStream_t stream);
+
+// ---------------------------------------------------------------- row kernels
+int launch_ln_modulate(const bf16* x, int n, int d, float eps, const float* shift,
+                       const float* scale, bf16* h, cudaStream_t stream);
+// x_res = bf16(x_state); h = LN(x_res)(1 + scale) + shift
+int launch_ln_modulate_from_state(const float* x_state, int n, int d, float eps,
+                                  const float* shift, const float* scale, bf16* x_res,
+                                  bf16* h, cudaStream_t stream);
+int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,
+                       const float* final_mod, float dt_sigma, float* x_state,
+                       cudaStream_t stream);
+int launch_token_pair(const bf16* src, bf16* dst, int t, int h, int w, int n_audio, int d,
+                      cudaStream_t stream);
+int launch_token_unpair(const bf16* src, bf16* dst, const bf16* saved, int t, int h, int w,
+                        int n_audio, int d, cudaStream_t stream);
+int launch_quantize_rows(const bf16* a, int rows, int cols, int8_t* q, float* scale,
+                         cudaStream_t stream);
+int launch_adaln_gemv(const bf16* w, const bf16* b, const bf16* c, int n_out, int c_dim,
+                      float* out, cudaStream_t stream);
+int launch_rope_table(int t, int h, int w, int n_audio, int halved, int paired,
+                      int head_dim, const int* split, float theta, float* rope_cs,
+                      cudaStream_t stream);
+
+}  // namespace h3b

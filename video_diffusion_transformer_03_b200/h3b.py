@@ -1,0 +1,285 @@
+"""ctypes binding of libh3b.so (argument marshalling only).
+
+Every function takes torch tensors that already live where the C ABI expects them
+(device tensors for device pointers) and passes their data pointers, sizes and the
+current CUDA stream.  All computation happens in the CUDA library; there is no fallback:
+importing this module fails if libh3b.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libh3b.so")
+
+H3B_OK, H3B_EINVAL, H3B_EWORKSPACE, H3B_ECUDA, H3B_ETIMEOUT, H3B_EUNSUPPORTED = 0, -1, -2, -3, -4, -5
+PAIR, UNPAIR = 0, 1
+EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_ROPE, EPI_GATE_RESID = 0, 1, 2, 3
+
+
+class H3BError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"h3b error {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int), ("n_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("d_ff", ctypes.c_int), ("c_dim", ctypes.c_int), ("rope_split", ctypes.c_int * 3),
+                ("rope_theta", ctypes.c_float), ("ln_eps", ctypes.c_float)]
+
+
+class Grid(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int),
+                ("n_audio", ctypes.c_int), ("rope_halved", ctypes.c_int)]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "h3b_version": (_I, []),
+    "h3b_last_error": (ctypes.c_char_p, []),
+    "h3b_launch_count": (ctypes.c_uint64, []),
+    "h3b_sync_status": (_I, [_P]),
+    "h3b_workspace_size": (_SZ, [ctypes.POINTER(Dims), _I]),
+    "h3b_denoise_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I]),
+    "h3b_adaln_modulation": (_I, [_P, _P, _P, _I, _I, _P, _P]),
+    "h3b_rope_table": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I, _P, _P]),
+    "h3b_ln_modulate": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
+    "h3b_block_forward": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _P, _P, _P,
+                               _I, _I, _P, _P, _P, _SZ, _P]),
+    "h3b_final_euler": (_I, [_P, _I, _I, _I, _F, _P, _F, _F, _P, _P]),
+    "h3b_denoise_step": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                              ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P, _P,
+                              _SZ, _P]),
+    "h3b_denoise_host": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                              ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _I, _I, _I, _P,
+                              _P, _P, _P, _SZ, _P]),
+    "h3b_token_reduce": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "h3b_quantize_rows": (_I, [_P, _I, _I, _P, _P, _P]),
+    "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P]),
+    "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P]),
+    "h3b_layer_mask": (_I, [_P, _I, _I, _I, _P]),
+}
+
+EXPORTS = tuple(_SIGS)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m video_diffusion_transformer_03_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+LIB_PATH = _LIB_PATH
+
+
+def _check(rc: int) -> None:
+    if rc != H3B_OK:
+        raise H3BError(rc, lib.h3b_last_error().decode(errors="replace"))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to h3b must be contiguous")
+    return t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if not t.is_cuda or t.dtype != dtype:
+        raise TypeError(f"{name}: expected a CUDA {dtype} tensor, got {t.device} {t.dtype}")
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------------- plumbing
+def version() -> int:
+    return lib.h3b_version()
+
+
+def launch_count() -> int:
+    return int(lib.h3b_launch_count())
+
+
+def sync_status(stream=None) -> None:
+    _check(lib.h3b_sync_status(_stream(stream)))
+
+
+def make_dims(d, n_heads, head_dim, d_ff, c_dim, rope_split, rope_theta=10000.0, ln_eps=1e-6) -> Dims:
+    return Dims(d, n_heads, head_dim, d_ff, c_dim, (ctypes.c_int * 3)(*rope_split),
+                rope_theta, ln_eps)
+
+
+def make_grid(t, h, w, n_audio, rope_halved=False) -> Grid:
+    return Grid(t, h, w, n_audio, int(bool(rope_halved)))
+
+
+def make_block_weights(p) -> BlockWeights:
+    """p: mapping with the eight bf16 CUDA tensors w_qkv, b_qkv, w_o, b_o, w_fc1, b_fc1,
+    w_fc2, b_fc2."""
+    for k in ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2"):
+        _dev(p[k], torch.bfloat16, k)
+    return BlockWeights(*[_ptr(p[k]) for k in
+                          ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")])
+
+
+def workspace_size(dims: Dims, n_tokens: int) -> int:
+    return lib.h3b_workspace_size(ctypes.byref(dims), n_tokens)
+
+
+def denoise_workspace_size(dims: Dims, grid: Grid, reduce: bool) -> int:
+    return lib.h3b_denoise_workspace_size(ctypes.byref(dims), ctypes.byref(grid), int(bool(reduce)))
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device or "cuda")
+
+
+# ---------------------------------------------------------------------- steps
+def adaln_modulation(w, b, c, out, stream=None) -> None:
+    _dev(w, torch.bfloat16, "w"); _dev(b, torch.bfloat16, "b"); _dev(c, torch.bfloat16, "c")
+    _dev(out, torch.float32, "out")
+    c_dim = w.shape[-1]
+    n_out = w.numel() // c_dim
+    _check(lib.h3b_adaln_modulation(_ptr(w), _ptr(b), _ptr(c), n_out, c_dim, _ptr(out),
+                                    _stream(stream)))
+
+
+def rope_table(dims: Dims, grid: Grid, paired: bool, out, stream=None) -> None:
+    _dev(out, torch.float32, "rope_cs")
+    _check(lib.h3b_rope_table(ctypes.byref(dims), ctypes.byref(grid), int(bool(paired)),
+                              _ptr(out), _stream(stream)))
+
+
+def ln_modulate(x, eps, shift, scale, h, stream=None) -> None:
+    _dev(x, torch.bfloat16, "x"); _dev(h, torch.bfloat16, "h")
+    _check(lib.h3b_ln_modulate(_ptr(x), x.shape[0], x.shape[1], eps, _ptr(shift), _ptr(scale),
+                               _ptr(h), _stream(stream)))
+
+
+def block_forward(dims: Dims, weights: BlockWeights, mod, mod_next, rope_cs, x, h, ws,
+                  compute_h: bool, stream=None) -> None:
+    _dev(x, torch.bfloat16, "x"); _dev(h, torch.bfloat16, "h"); _dev(mod, torch.float32, "mod")
+    _check(lib.h3b_block_forward(ctypes.byref(dims), ctypes.byref(weights), _ptr(mod),
+                                 _ptr(mod_next), _ptr(rope_cs), x.shape[0], int(bool(compute_h)),
+                                 _ptr(x), _ptr(h), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream)))
+
+
+def final_euler(x_l, n_video, eps, final_mod, sigma, sigma_next, x_state, stream=None) -> None:
+    _dev(x_l, torch.bfloat16, "x_l"); _dev(x_state, torch.float32, "x_state")
+    _check(lib.h3b_final_euler(_ptr(x_l), x_l.shape[0], n_video, x_l.shape[1], eps,
+                               _ptr(final_mod), sigma, sigma_next, _ptr(x_state), _stream(stream)))
+
+
+def _blocks_array(blocks: Sequence[BlockWeights]):
+    arr = (BlockWeights * max(len(blocks), 1))()
+    for i, b in enumerate(blocks):
+        arr[i] = b
+    return arr
+
+
+def _mask_array(active, n):
+    if active is None:
+        return None, None
+    buf = (ctypes.c_ubyte * n)(*[1 if a else 0 for a in active])
+    return buf, ctypes.cast(buf, ctypes.c_void_p)
+
+
+def denoise_step(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods, final_mod,
+                 reduce_after: int, unpair_bypass: bool, sigma: float, sigma_next: float, x_state,
+                 ws, stream=None) -> None:
+    _dev(x_state, torch.float32, "x_state")
+    arr = _blocks_array(blocks)
+    keep, mask = _mask_array(active, len(blocks))
+    _check(lib.h3b_denoise_step(ctypes.byref(dims), ctypes.byref(grid), len(blocks), arr, mask,
+                                _ptr(mods), _ptr(final_mod), reduce_after, int(bool(unpair_bypass)),
+                                sigma, sigma_next, _ptr(x_state), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def denoise_host(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods, final_mod,
+                 reduce_after: int, unpair_bypass: bool, n_steps: int, first_step: int, n_run: int,
+                 x_host_in, x_host_out, x_state_dev, ws, stream=None) -> None:
+    """x_host_in / x_host_out: CPU float32 tensors (pinned for full bandwidth)."""
+    if x_host_in.is_cuda or x_host_out.is_cuda:
+        raise TypeError("denoise_host takes host buffers")
+    arr = _blocks_array(blocks)
+    keep, mask = _mask_array(active, len(blocks))
+    _check(lib.h3b_denoise_host(ctypes.byref(dims), ctypes.byref(grid), len(blocks), arr, mask,
+                                _ptr(mods), _ptr(final_mod), reduce_after, int(bool(unpair_bypass)),
+                                n_steps, first_step, n_run, _ptr(x_host_in), _ptr(x_host_out),
+                                _ptr(x_state_dev), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)))
+    del keep
+
+
+def token_reduce(mode: int, src, dst, saved, t, h, w, n_audio, stream=None) -> None:
+    _dev(src, torch.bfloat16, "src"); _dev(dst, torch.bfloat16, "dst")
+    _check(lib.h3b_token_reduce(mode, _ptr(src), _ptr(dst), _ptr(saved), t, h, w, n_audio,
+                                src.shape[1], _stream(stream)))
+
+
+def quantize_rows(a, q, scale, stream=None) -> None:
+    _dev(a, torch.bfloat16, "a"); _dev(q, torch.int8, "q"); _dev(scale, torch.float32, "scale")
+    _check(lib.h3b_quantize_rows(_ptr(a), a.shape[0], a.shape[1], _ptr(q), _ptr(scale),
+                                 _stream(stream)))
+
+
+def fc2_int8_row(act, w_q, w_scale, bias, gate, resid, act_q, row_scale, acc_out=None,
+                 stream=None) -> None:
+    _dev(act, torch.bfloat16, "act"); _dev(w_q, torch.int8, "w_q"); _dev(resid, torch.bfloat16, "resid")
+    M, K = act.shape
+    _check(lib.h3b_fc2_int8_row(_ptr(act), M, K, w_q.shape[0], _ptr(w_q), _ptr(w_scale),
+                                _ptr(bias), _ptr(gate), _ptr(resid), _ptr(act_q), _ptr(row_scale),
+                                _ptr(acc_out), _stream(stream)))
+
+
+def gemm_bf16(A, B, epilogue, bias, out, gate=None, rope_cs=None, rope_cols=0, head_dim=128,
+              stream=None) -> None:
+    _dev(A, torch.bfloat16, "A"); _dev(B, torch.bfloat16, "B"); _dev(out, torch.bfloat16, "out")
+    M, K = A.shape
+    N = B.shape[0]
+    _check(lib.h3b_gemm_bf16(_ptr(A), _ptr(B), M, N, K, epilogue, _ptr(bias), _ptr(gate),
+                             _ptr(rope_cs), rope_cols, head_dim, _ptr(out), _stream(stream)))
+
+
+def attention(qkv, n_heads, head_dim, out, stream=None) -> None:
+    _dev(qkv, torch.bfloat16, "qkv"); _dev(out, torch.bfloat16, "out")
+    _check(lib.h3b_attention(_ptr(qkv), qkv.shape[0], n_heads, head_dim, _ptr(out),
+                             _stream(stream)))
+
+
+def layer_mask(mods_host: np.ndarray, n_active: int) -> np.ndarray:
+    """mods_host: float32 [n_blocks, 6, d] on the host; returns a bool mask."""
+    m = np.ascontiguousarray(mods_host, dtype=np.float32)
+    nb, _, d = m.shape
+    out = (ctypes.c_ubyte * nb)()
+    _check(lib.h3b_layer_mask(m.ctypes.data, nb, d, n_active, ctypes.cast(out, ctypes.c_void_p)))
+    return np.array(list(out), dtype=bool)

@@ -1,0 +1,86 @@
+"""Device-resident synthetic DiT denoiser driven through the C ABI.
+
+Holds a workload's bf16 block weights, the AdaLN modulation vectors (computed on the GPU
+by h3b_adaln_modulation), the layer-thinning mask and the step workspace, and runs Euler
+steps with h3b_denoise_step / h3b_denoise_host.  No arithmetic of the method happens in
+Python.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import h3b, synth
+from .synth import DiTConfig
+
+
+def dims_of(cfg: DiTConfig) -> h3b.Dims:
+    return h3b.make_dims(cfg.d, cfg.n_heads, cfg.head_dim, cfg.d_ff, cfg.c_dim, cfg.rope_split,
+                         cfg.rope_theta, cfg.ln_eps)
+
+
+def grid_of(cfg: DiTConfig) -> h3b.Grid:
+    t, h, w = cfg.grid
+    return h3b.make_grid(t, h, w, cfg.n_audio, cfg.rope_halved)
+
+
+class DiTDenoiser:
+    def __init__(self, cfg: DiTConfig, device: str = "cuda", gen_device: str = "cpu",
+                 keep_host_params: bool = False):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.dims = dims_of(cfg)
+        self.grid = grid_of(cfg)
+        self.host_params = [] if keep_host_params else None
+        self.params = []
+        self.mods = torch.empty((cfg.n_blocks, 6, cfg.d), dtype=torch.float32, device=self.device)
+        self.c = synth.conditioning(cfg, gen_device).to(self.device)
+        for b in range(cfg.n_blocks):
+            p = synth.block_params(cfg, b, device=gen_device)
+            if keep_host_params:
+                self.host_params.append({k: v.cpu() for k, v in p.items()})
+            pd = {k: v.to(self.device) for k, v in p.items()}
+            del p
+            h3b.adaln_modulation(pd.pop("w_ada"), pd.pop("b_ada"), self.c, self.mods[b])
+            self.params.append(pd)
+        self.weights = [h3b.make_block_weights(p) for p in self.params]
+        fin = synth.final_params(cfg, gen_device)
+        self.host_final = {k: v.cpu() for k, v in fin.items()} if keep_host_params else None
+        self.final_mod = torch.empty((2, 2, cfg.d), dtype=torch.float32, device=self.device)
+        for s in range(2):
+            h3b.adaln_modulation(fin["w_fin"][s].contiguous().to(self.device),
+                                 fin["b_fin"][s].contiguous().to(self.device), self.c,
+                                 self.final_mod[s])
+        self.active: Optional[list] = None
+        if cfg.active_count < cfg.n_blocks:
+            mask = h3b.layer_mask(self.mods.cpu().numpy(), cfg.active_count)
+            self.active = [bool(m) for m in mask]
+        self.reduce = cfg.reduce_after > 0
+        self.ws = h3b.workspace(h3b.denoise_workspace_size(self.dims, self.grid, self.reduce),
+                                self.device)
+
+    @property
+    def n_tokens(self) -> int:
+        return self.cfg.n_tokens
+
+    def sigmas(self, i: int):
+        s = self.cfg.steps
+        return 1.0 - i / s, 1.0 - (i + 1) / s
+
+    def step(self, x_state: torch.Tensor, i: int, stream=None) -> None:
+        sg, sn = self.sigmas(i)
+        h3b.denoise_step(self.dims, self.grid, self.weights, self.active, self.mods,
+                         self.final_mod, self.cfg.reduce_after, self.cfg.unpair_bypass, sg, sn,
+                         x_state, self.ws, stream)
+
+    def run(self, x_state: torch.Tensor, n_run: Optional[int] = None, stream=None) -> None:
+        for i in range(self.cfg.run_steps if n_run is None else n_run):
+            self.step(x_state, i, stream)
+
+    def run_host(self, x_host_in: torch.Tensor, x_host_out: torch.Tensor,
+                 x_state_dev: torch.Tensor, n_run: Optional[int] = None, stream=None) -> None:
+        h3b.denoise_host(self.dims, self.grid, self.weights, self.active, self.mods,
+                         self.final_mod, self.cfg.reduce_after, self.cfg.unpair_bypass,
+                         self.cfg.steps, 0, self.cfg.run_steps if n_run is None else n_run,
+                         x_host_in, x_host_out, x_state_dev, self.ws, stream)
