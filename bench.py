@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--impl", default="h3b", choices=["h3b", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--kernel", default=None,
+                    help="time one kernel of the block alone on the workload shapes (for ncu)")
+    ap.add_argument("--reps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -213,7 +216,7 @@ def workload_name(cfg):
 
 
 # ------------------------------------------------------------------------------ GPU arm
-def time_kernels(model, cfg, peaks, counts_per_step, reps=20):
+def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3):
     """Time each kernel of the block alone (CUDA events on the launching stream), with the
     weights rotated over all blocks so that they stream from HBM as in the step."""
     import torch
@@ -260,7 +263,9 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20):
     stream = torch.cuda.current_stream(dev)
     out = {}
     for name, (fn, bound, work) in kinds.items():
-        for i in range(3):
+        if only is not None and name != only:
+            continue
+        for i in range(warm):
             fn(i)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -313,6 +318,12 @@ def run_gpu(args):
     cfg = synth.CONFIGS[args.config]
     model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
     counts, n_active = workload_counts(cfg, model.active)
+    if args.kernel:
+        res = time_kernels(model, cfg, peaks, {"blocks": n_active * cfg.run_steps},
+                           reps=args.reps, only=args.kernel)
+        if rank == 0:
+            print(json.dumps({"kernel_only": args.kernel, "config": cfg.name, **res}), flush=True)
+        return
     x0 = synth.latent_noise(cfg, device=str(dev))
     x = x0.clone()
     stream = torch.cuda.current_stream(dev)

@@ -68,8 +68,6 @@ def test_block_tiny_full():
     xo, ho = oracle_block(cfg, params, nxt, c, x)
     check("x_out", np64(xg), xo, np64(x))
     check("h_next", np64(hg), ho)
-    # update itself (the residual branches) within tolerance too
-    assert rel_l2(np64(xg) - np64(x), xo - np64(x)) < 5e-2
 
 
 def _rows(cfg, k=40):
