@@ -236,20 +236,21 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3)
     mod = model.mods[0]
     P = model.params
     nb = len(P)
+    ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
     kinds = {
         "gemm_qkv_rope": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_qkv"], h3b.EPI_BIAS_ROPE,
                                                   P[i % nb]["b_qkv"], qkv, rope_cs=cs,
-                                                  rope_cols=2 * d, head_dim=hd),
+                                                  rope_cols=2 * d, head_dim=hd, ws=ws),
                           "tensor", 2 * n * d * 3 * d),
         "attention": (lambda i: h3b.attention(qkv, H, hd, attn), "tensor", 4 * n * n * d),
         "gemm_out_gate": (lambda i: h3b.gemm_bf16(attn, P[i % nb]["w_o"], h3b.EPI_GATE_RESID,
-                                                  P[i % nb]["b_o"], x, gate=mod[2]),
+                                                  P[i % nb]["b_o"], x, gate=mod[2], ws=ws),
                           "tensor", 2 * n * d * d),
         "gemm_fc1_gelu": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_fc1"], h3b.EPI_BIAS_GELU,
-                                                  P[i % nb]["b_fc1"], gbuf),
+                                                  P[i % nb]["b_fc1"], gbuf, ws=ws),
                           "tensor", 2 * n * d * f),
         "gemm_fc2_gate": (lambda i: h3b.gemm_bf16(gbuf, P[i % nb]["w_fc2"], h3b.EPI_GATE_RESID,
-                                                  P[i % nb]["b_fc2"], x, gate=mod[5]),
+                                                  P[i % nb]["b_fc2"], x, gate=mod[5], ws=ws),
                           "tensor", 2 * n * f * d),
         "ln_modulate": (lambda i: h3b.ln_modulate(x, cfg.ln_eps, mod[0], mod[1], h), "hbm",
                         4 * n * d),

@@ -114,6 +114,11 @@ int h3b_sync_status(void* stream);
  * aliased by lifetime). */
 size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens);
 
+/* Bytes of the optional scratch that lets h3b_gemm_bf16 and h3b_fc2_int8_row use the
+ * stream-K schedule (K loop split across all SMs when the output tiles do not fill the
+ * SMs evenly).  The block and step workspaces already include it. */
+size_t h3b_gemm_workspace_size(void);
+
 /* Bytes of workspace h3b_denoise_step needs for this grid; reduce != 0 adds the paired
  * stream's buffers. */
 size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce);
@@ -228,11 +233,12 @@ int h3b_quantize_rows(const h3b_bf16* a, int rows, int cols, int8_t* q, float* s
  * act [M, K] bf16; w_q [n_out, K] int8; w_scale, gate [n_out] fp32; bias [n_out] fp32 or
  * NULL; resid [M, n_out] bf16 in/out; act_q [M, K] int8 and row_scale [M] fp32 outputs;
  * acc_out [M, n_out] int32 output or NULL.  All device.  K % 128 == 0,
- * n_out % 256 == 0. */
+ * n_out % 128 == 0.  ws: NULL, or device scratch of h3b_gemm_workspace_size() bytes that
+ * enables the stream-K schedule (the result is the same either way: int32 sums are exact). */
 int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t* w_q,
                      const float* w_scale, const float* bias, const float* gate,
                      h3b_bf16* resid, int8_t* act_q, float* row_scale, int32_t* acc_out,
-                     void* stream);
+                     void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- single kernels */
 /* The projection GEMM used by the block: out = A B^T with an epilogue.
@@ -242,11 +248,13 @@ int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t*
  *   H3B_EPI_BIAS_ROPE:  out = bf16(rope(acc + bias)) on columns < rope_cols (pairs of
  *                       adjacent columns, head_dim-periodic, table rope_cs), plain after
  *   H3B_EPI_GATE_RESID: out = bf16(out + gate (acc + bias)), in place (out is the residual)
- * bias [N] bf16; gate [N] fp32 (GATE_RESID only); rope_cs as h3b_rope_table. */
+ * bias [N] bf16; gate [N] fp32 (GATE_RESID only); rope_cs as h3b_rope_table.
+ * ws: NULL, or device scratch of h3b_gemm_workspace_size() bytes enabling stream-K. */
 enum { H3B_EPI_BIAS = 0, H3B_EPI_BIAS_GELU = 1, H3B_EPI_BIAS_ROPE = 2, H3B_EPI_GATE_RESID = 3 };
 int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
                   const h3b_bf16* bias, const float* gate, const float* rope_cs,
-                  int rope_cols, int head_dim, h3b_bf16* out, void* stream);
+                  int rope_cols, int head_dim, h3b_bf16* out, void* ws, size_t ws_bytes,
+                  void* stream);
 
 /* Joint self-attention over one packed QKV buffer: qkv [n_tokens, 3 n_heads head_dim]
  * bf16 (q, then k, then v; head j at column j*head_dim of each), out [n_tokens,

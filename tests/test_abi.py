@@ -58,14 +58,14 @@ def _err(fn, *args):
 def test_validation_rejects_before_any_launch():
     L = h3b.lib
     p = ctypes.c_void_p(4096)       # aligned, never dereferenced: validation fails first
-    rc, msg = _err(L.h3b_gemm_bf16, p, p, 64, 256, 65, 0, p, None, None, 0, 128, p, None)
+    rc, msg = _err(L.h3b_gemm_bf16, p, p, 64, 256, 65, 0, p, None, None, 0, 128, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL and "K=65" in msg
-    rc, _ = _err(L.h3b_gemm_bf16, p, p, 64, 200, 64, 0, p, None, None, 0, 128, p, None)
+    rc, _ = _err(L.h3b_gemm_bf16, p, p, 64, 200, 64, 0, p, None, None, 0, 128, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL
-    rc, _ = _err(L.h3b_gemm_bf16, p, p, 64, 256, 64, 3, p, None, None, 0, 128, p, None)
+    rc, _ = _err(L.h3b_gemm_bf16, p, p, 64, 256, 64, 3, p, None, None, 0, 128, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL                                  # gate missing
     rc, _ = _err(L.h3b_gemm_bf16, ctypes.c_void_p(4097), p, 64, 256, 64, 0, p, None, None, 0,
-                 128, p, None)
+                 128, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL                                  # misaligned A
     rc, _ = _err(L.h3b_attention, p, 10, 2, 96, p, None)
     assert rc == h3b.H3B_EINVAL                                  # head_dim 96
@@ -75,7 +75,7 @@ def test_validation_rejects_before_any_launch():
     assert rc == h3b.H3B_EINVAL                                  # unknown mode
     rc, _ = _err(L.h3b_quantize_rows, p, 4, 40, p, p, None)
     assert rc == h3b.H3B_EINVAL                                  # cols % 16
-    rc, _ = _err(L.h3b_fc2_int8_row, p, 8, 100, 256, p, p, None, p, p, p, p, None, None)
+    rc, _ = _err(L.h3b_fc2_int8_row, p, 8, 100, 256, p, p, None, p, p, p, p, None, None, 0, None)
     assert rc == h3b.H3B_EINVAL                                  # K % 128
     rc, _ = _err(L.h3b_ln_modulate, p, 4, 300, ctypes.c_float(1e-6), p, p, p, None)
     assert rc == h3b.H3B_EINVAL                                  # d % 256

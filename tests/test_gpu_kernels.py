@@ -21,12 +21,24 @@ def _sync():
 
 # ------------------------------------------------------------------------------ GEMM
 GEMM_SHAPES = [(40, 768, 256), (200, 256, 128), (300, 384, 192), (1600, 3072, 3072),
-               (1600, 12288, 3072), (1600, 3072, 12288)]
+               (1600, 12288, 3072), (1600, 3072, 12288),
+               (1024, 2048, 4096), (1000, 640, 2048),
+               # long-K shapes that take the stream-K schedule, one tile spanning 3 to 5
+               # scheduling units (CTA pairs, then single CTAs with 128-wide tiles)
+               (1024, 2048, 8192), (1000, 640, 8192)]
+_SCRATCH = {}
 
 
+def gemm_scratch():
+    if "ws" not in _SCRATCH:
+        _SCRATCH["ws"] = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV)
+    return _SCRATCH["ws"]
+
+
+@pytest.mark.parametrize("sk", [True, False], ids=["scratch", "noscratch"])
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
 @pytest.mark.parametrize("epi", [h3b.EPI_BIAS, h3b.EPI_BIAS_GELU, h3b.EPI_GATE_RESID])
-def test_gemm_epilogues(M, N, K, epi):
+def test_gemm_epilogues(M, N, K, epi, sk):
     if (M, N, K) == (1600, 12288, 3072) and epi != h3b.EPI_BIAS_GELU:
         pytest.skip("FC1 shape is checked with its own epilogue")
     if (M, N, K) == (1600, 3072, 12288) and epi != h3b.EPI_GATE_RESID:
@@ -47,11 +59,18 @@ def test_gemm_epilogues(M, N, K, epi):
         out.copy_(resid.to(DEV))
         gate = g.to(DEV)
         want = O.gated_residual(np64(resid), np64(g), acc)
-    h3b.gemm_bf16(A.to(DEV), B.to(DEV), epi, bias.to(DEV), out, gate=gate)
+    Ad, Bd, bd = A.to(DEV), B.to(DEV), bias.to(DEV)
+    ws = gemm_scratch() if sk else None
+    init = out.clone()
+    h3b.gemm_bf16(Ad, Bd, epi, bd, out, gate=gate, ws=ws)
     _sync()
     got = np64(out)
     assert rel_l2(got, want) < 4e-3
     assert max_block_rel_l2(got, want) < 8e-3
+    again = init.clone()
+    h3b.gemm_bf16(Ad, Bd, epi, bd, again, gate=gate, ws=ws)        # deterministic
+    _sync()
+    assert torch.equal(again, out)
 
 
 @pytest.mark.parametrize("grid,n_audio,heads,hd,split", [
@@ -71,7 +90,7 @@ def test_gemm_rope_epilogue(grid, n_audio, heads, hd, split):
     h3b.rope_table(dims, g, False, cs)
     out = torch.empty((M, 3 * d), dtype=torch.bfloat16, device=DEV)
     h3b.gemm_bf16(A.to(DEV), B.to(DEV), h3b.EPI_BIAS_ROPE, bias.to(DEV), out, rope_cs=cs,
-                  rope_cols=2 * d, head_dim=hd)
+                  rope_cols=2 * d, head_dim=hd, ws=gemm_scratch())
     _sync()
     acc = np64(A) @ np64(B).T + np64(bias)
     pos = O.rope_positions(grid, n_audio)
@@ -220,7 +239,7 @@ def test_quantize_rows_bit_exact(M, K):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), ws.view(np.uint32))
 
 
-def _fc2_case(M, K, N, with_bias, sample_rows=None, seed=50):
+def _fc2_case(M, K, N, with_bias, sample_rows=None, seed=50, sk=True):
     a = _quant_input(M, K, seed)
     w = rnd((N, K), 0.02, seed=seed + 1)
     gate = rnd((N,), 1.0, seed=seed + 2, dtype=torch.float32)
@@ -235,7 +254,7 @@ def _fc2_case(M, K, N, with_bias, sample_rows=None, seed=50):
     acc = torch.empty((M, N), dtype=torch.int32, device=DEV)
     out = resid.to(DEV)
     h3b.fc2_int8_row(a.to(DEV), wq, wsc, None if bias is None else bias.to(DEV), gate.to(DEV),
-                     out, aq, rs, acc)
+                     out, aq, rs, acc, ws=gemm_scratch() if sk else None)
     _sync()
     owq, ows = O.quantize_rows(w.float().numpy())
     assert np.array_equal(wq.cpu().numpy(), owq)
@@ -252,9 +271,14 @@ def _fc2_case(M, K, N, with_bias, sample_rows=None, seed=50):
 
 
 @pytest.mark.parametrize("M,K,N,bias", [(300, 384, 256, False), (130, 12288, 384, True),
-                                        (257, 1024, 512, True)])
+                                        (257, 1024, 512, True), (1024, 1024, 8192, False),
+                                        (1000, 4096, 640, True), (512, 16384, 512, True)])
 def test_fc2_int8_row_small(M, K, N, bias):
     _fc2_case(M, K, N, bias)
+
+
+def test_fc2_int8_row_without_scratch():
+    _fc2_case(1024, 1024, 8192, True, sk=False)
 
 
 def test_fc2_int8_row_full_size():

@@ -20,6 +20,9 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <random>
 
 namespace h3b {
 
@@ -41,9 +44,90 @@ struct GemmCfg {
 
 struct GemmParams {
   int M, N, k_blocks, m_tiles, n_tiles;
+  // Stream-K: the tiles x k_blocks iterations are cut into one equal contiguous range per
+  // scheduling unit (CTA or CTA pair).  Each unit walks its range backwards, tile by tile
+  // (k-blocks inside a tile still run forwards), so the partial tile at the end of its
+  // range is computed first: the unit stores it in its slot and publishes sk_seq in its
+  // flag.  The unit holding the tile's last k-block reaches that tile last and adds the
+  // slots of the lower-numbered units that computed the rest of it: waits only ever point
+  // at lower-numbered units, which are dispatched first.
+  int sk;
+  long long sk_iters;
+  uint32_t* sk_slots;            // [gridDim.x][128][BN] raw accumulator words
+  unsigned long long* sk_flags;  // [gridDim.x][4]
+  unsigned long long sk_seq;
   GemmEpilogue epi;
   uint32_t* err;
 };
+
+constexpr int kMaxSkCtas = 160;  // stream-K grid cap (slots in the scratch)
+
+// Stream-K scratch: slots sized for the widest tile, then the flags (same offsets for
+// every tile width, so launches of different widths may share one scratch buffer).
+// One flag per (CTA, epilogue warp): a warp publishes the 32 slot rows it wrote, and the
+// owner's warp with the same TMEM lane quarter reads exactly those rows.
+constexpr size_t kSkFlagsOffset = size_t(kMaxSkCtas) * kBM * 256 * 4;
+constexpr size_t kSkScratchBytes = kSkFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
+
+// Scheduling units are CTAs (single-SM kernel) or CTA pairs (pair kernel): `me` is this
+// unit's index and `count` the number of units in the grid.
+__device__ __forceinline__ long long sk_begin(const GemmParams& p, int c, int count) {
+  return p.sk_iters * c / count;
+}
+
+// Unit whose range contains iteration i.
+__device__ __forceinline__ int sk_owner(const GemmParams& p, long long i, int count) {
+  int c = static_cast<int>(i * count / p.sk_iters);
+  while (c + 1 < count && sk_begin(p, c + 1, count) <= i) ++c;
+  while (c > 0 && sk_begin(p, c, count) > i) --c;
+  return c;
+}
+
+// Work items of this unit: (tile, k-block range).  Every role walks the same sequence.
+struct Sched {
+  long long it, it_end;  // stream-K
+  int tile;              // data-parallel
+  int count;
+};
+
+__device__ __forceinline__ void sched_init(const GemmParams& p, Sched& s, int me, int count) {
+  s.count = count;
+  if (p.sk) {
+    s.it = sk_begin(p, me, count);
+    s.it_end = sk_begin(p, me + 1, count);
+  } else {
+    s.tile = me;
+  }
+}
+
+__device__ __forceinline__ bool sched_next(const GemmParams& p, Sched& s, int& tile, int& kb0,
+                                           int& kb1) {
+  if (p.sk) {  // backwards over the range [it, it_end): it_end moves down
+    if (s.it_end <= s.it) return false;
+    tile = static_cast<int>((s.it_end - 1) / p.k_blocks);
+    const long long t0 = static_cast<long long>(tile) * p.k_blocks;
+    const long long start = s.it > t0 ? s.it : t0;
+    kb0 = static_cast<int>(start - t0);
+    kb1 = static_cast<int>(s.it_end - t0);
+    s.it_end = start;
+    return true;
+  }
+  if (s.tile >= p.m_tiles * p.n_tiles) return false;
+  tile = s.tile;
+  kb0 = 0;
+  kb1 = p.k_blocks;
+  s.tile += s.count;
+  return true;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
                                             int& nb) {
@@ -82,20 +166,6 @@ __device__ __forceinline__ void load_bf16x32(const bf16* src, float (&v)[32]) {
   }
 }
 
-// Same as load_bf16x32 but through the coherent path (the residual is read and written
-// by this kernel).
-__device__ __forceinline__ void load_bf16x32_rw(const bf16* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 u = s[i];
-    float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y), c = unpack_bf16x2(u.z),
-           d = unpack_bf16x2(u.w);
-    v[8 * i + 0] = a.x; v[8 * i + 1] = a.y; v[8 * i + 2] = b.x; v[8 * i + 3] = b.y;
-    v[8 * i + 4] = c.x; v[8 * i + 5] = c.y; v[8 * i + 6] = d.x; v[8 * i + 7] = d.y;
-  }
-}
-
 __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -118,10 +188,35 @@ __device__ __forceinline__ void load_f32x32(const float* src, float (&v)[32]) {
   }
 }
 
+// Row operands of one 32-column chunk that come from global memory, loaded one chunk
+// ahead of their use so that their latency overlaps the previous chunk's work.
+struct RowIn {
+  uint4 res[4];  // residual, 32 bf16 (gated-residual epilogues)
+  float4 cs[8];  // RoPE (cos, sin) of 16 pairs (RoPE epilogue)
+};
+
+template <int EPI>
+__device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int col, RowIn& in) {
+  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+    const uint4* s = reinterpret_cast<const uint4*>(e.out + size_t(row) * e.ld_out + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) in.res[i] = s[i];  // coherent: this kernel rewrites it
+  }
+  if constexpr (EPI == kEpiRope) {
+    if (col < e.rope_cols) {
+      const int half = e.head_dim >> 1;
+      const float4* cs = reinterpret_cast<const float4*>(
+          e.rope_cs + (size_t(row) * half + ((col % e.head_dim) >> 1)) * 2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) in.cs[i] = __ldg(cs + i);
+    }
+  }
+}
+
 // Epilogue of one 32-column chunk of one row.
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, int col,
-                                               const uint32_t (&r)[32]) {
+                                               const uint32_t (&r)[32], const RowIn& in) {
   float v[32];
   if constexpr (EPI == kEpiInt8Deq) {
     const float rs = __ldg(e.row_scale + row);
@@ -156,12 +251,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
   }
   if constexpr (EPI == kEpiRope) {
     if (col < e.rope_cols) {
-      const int half = e.head_dim >> 1;
-      const float4* cs = reinterpret_cast<const float4*>(
-          e.rope_cs + (size_t(row) * half + ((col % e.head_dim) >> 1)) * 2);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {  // 2 pairs per float4 (cos0, sin0, cos1, sin1)
-        const float4 c = __ldg(cs + i);
+        const float4 c = in.cs[i];
         const float x0 = v[4 * i], x1 = v[4 * i + 1], y0 = v[4 * i + 2], y1 = v[4 * i + 3];
         v[4 * i + 0] = x0 * c.x - x1 * c.y;
         v[4 * i + 1] = x0 * c.y + x1 * c.x;
@@ -172,13 +264,67 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
   }
   bf16* dst = e.out + size_t(row) * e.ld_out + col;
   if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
-    float g[32], res[32];
+    float g[32];
     load_f32x32(e.gate + col, g);
-    load_bf16x32_rw(dst, res);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = fmaf(g[j], v[j], res[j]);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {in.res[i].x, in.res[i].y, in.res[i].z, in.res[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 rr = unpack_bf16x2(w[k]);
+        v[8 * i + 2 * k] = fmaf(g[8 * i + 2 * k], v[8 * i + 2 * k], rr.x);
+        v[8 * i + 2 * k + 1] = fmaf(g[8 * i + 2 * k + 1], v[8 * i + 2 * k + 1], rr.y);
+      }
+    }
   }
   store_bf16x32(dst, v);
+}
+
+// Epilogue of one work unit for one thread (one accumulator row, BN columns starting at
+// col0): TMEM chunk by chunk, plus the stream-K partials held in slots
+// src * stride + off for src in [src_lo, src_hi), then the epilogue and the stores.
+template <int BN, bool INT8, int EPI>
+__device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbase, int row,
+                                              int row_in_tile, int col0, int src_lo,
+                                              int src_hi, int stride, int off) {
+  constexpr int NC = BN / 32;
+  const bool valid = row < p.M;
+  RowIn in[2];
+  if (valid) load_row_in<EPI>(p.epi, row, col0, in[0]);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    if (c + 1 < NC && valid) load_row_in<EPI>(p.epi, row, col0 + (c + 1) * 32, in[(c + 1) & 1]);
+    uint4 part[8];
+    if (src_lo < src_hi) {
+      const uint4* ps = reinterpret_cast<const uint4*>(
+          p.sk_slots + (size_t(src_lo * stride + off) * kBM + row_in_tile) * BN + c * 32);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) part[i] = __ldcg(ps + i);
+    }
+    tmem_wait_ld(r);
+    for (int src = src_lo; src < src_hi; ++src) {
+      if (src > src_lo) {
+        const uint4* ps = reinterpret_cast<const uint4*>(
+            p.sk_slots + (size_t(src * stride + off) * kBM + row_in_tile) * BN + c * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part[i] = __ldcg(ps + i);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t u[4] = {part[i].x, part[i].y, part[i].z, part[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if constexpr (INT8)
+            r[4 * i + k] = uint32_t(int32_t(r[4 * i + k]) + int32_t(u[k]));
+          else
+            r[4 * i + k] = __float_as_uint(__uint_as_float(r[4 * i + k]) + __uint_as_float(u[k]));
+        }
+      }
+    }
+    if (valid) epilogue_chunk<EPI>(p.epi, row, col0 + c * 32, r, in[c & 1]);
+  }
 }
 
 template <int BN, bool INT8, int EPI>
@@ -233,7 +379,6 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = p.m_tiles * p.n_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -244,10 +389,13 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      Sched sc;
+      sched_init(p, sc, blockIdx.x, gridDim.x);
+      int tile, kb0, kb1;
+      while (ok && sched_next(p, sc, tile, kb0, kb1)) {
         int mb, nb;
         tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrGemmWait)) {
             ok = false;
             break;
@@ -274,13 +422,16 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+      Sched sc;
+      sched_init(p, sc, blockIdx.x, gridDim.x);
+      int tile, kb0, kb1;
+      for (; ok && sched_next(p, sc, tile, kb0, kb1); ++local) {
         const int buf = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         if (!wait_bar(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.err, kErrGemmWait)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bar(&full[stage], phase, abort_flag, p.err, kErrGemmWait)) {
             ok = false;
             break;
@@ -292,7 +443,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int k = 0; k < K_STEPS; ++k) {
             const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
-            const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
             if constexpr (INT8)
               umma_i8(d_tmem, ad, bd, IDESC, acc);
             else
@@ -315,7 +466,10 @@ __global__ void __launch_bounds__(192, 1)
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    Sched sc;
+    sched_init(p, sc, blockIdx.x, gridDim.x);
+    int tile, kb0, kb1;
+    for (; sched_next(p, sc, tile, kb0, kb1); ++local) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       const int buf = local & 1;
@@ -325,13 +479,52 @@ __global__ void __launch_bounds__(192, 1)
       if (!ok) break;
       tc_fence_after();
       const int row = mb * kBM + row_in_tile;
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
+      if (kb1 < p.k_blocks) {
+        // stream-K contributor: park the partial tile in this CTA's slot
+        uint32_t* slot = p.sk_slots + (size_t(blockIdx.x) * kBM + row_in_tile) * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + lane_addr + static_cast<uint32_t>(buf * BN + c * 32), r);
-        tmem_wait_ld(r);
-        if (row < p.M) epilogue_chunk<EPI>(p.epi, row, nb * BN + c * 32, r);
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_wait_ld(r);
+          uint4* dst = reinterpret_cast<uint4*>(slot + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            __stcg(dst + i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+        }
+        __threadfence();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[buf]);
+          st_release_u64(p.sk_flags + blockIdx.x * 4 + quarter, p.sk_seq);
+        }
+        continue;
       }
+      // tile owner: add the partials of the CTAs that computed the rest of this tile
+      int c_lo = static_cast<int>(blockIdx.x);
+      if (kb0 > 0) {
+        c_lo = sk_owner(p, static_cast<long long>(tile) * p.k_blocks, gridDim.x);
+        for (int c = c_lo; c < static_cast<int>(blockIdx.x) && ok; ++c) {
+          const unsigned long long* f = p.sk_flags + c * 4 + quarter;
+          bool seen = ld_acquire_u64(f) == p.sk_seq;
+          if (!seen) {
+            const uint64_t t0 = global_timer_ns();
+            while (!seen) {
+              seen = ld_acquire_u64(f) == p.sk_seq;
+              if (!seen && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
+                *abort_flag = 1u;
+                atomicCAS(p.err, 0u, kErrGemmWait);
+                break;
+              }
+            }
+          }
+          ok = __all_sync(0xffffffffu, seen);
+        }
+      }
+      epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo,
+                                   static_cast<int>(blockIdx.x), 1, 0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -347,9 +540,279 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 cta_group::2): a cluster of two CTAs on two SMs computes a
+// 256 x 256 tile.  Each CTA loads its own 128 rows of A and its own 128 rows (half) of B
+// per 128-byte K slice, so per SM the operand traffic per MMA is two thirds of the
+// single-CTA 128 x 256 tile and the ring holds 6 stages.  The even CTA issues the MMAs
+// (M = 256) and signals both CTAs; each CTA's epilogue reads its own 128 accumulator
+// lanes.  Work units (tiles or stream-K ranges) are scheduled per pair.
+#ifndef H3B_PAIR_STAGES
+#define H3B_PAIR_STAGES 6
+#endif
+constexpr int kPairStages = H3B_PAIR_STAGES;
+constexpr uint32_t kPairHalfBytes = 128 * kTileBytesK;  // 16 KB: 128 rows x 128 B
+constexpr size_t kPairSmem = 1024 + size_t(kPairStages) * 2 * kPairHalfBytes + 256;
+
+template <bool INT8, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmParams p) {
+  constexpr int BN = 256;
+  constexpr int STAGES = kPairStages;
+  constexpr uint32_t HB = kPairHalfBytes;
+  constexpr uint32_t IDESC = INT8 ? idesc_s8(256, BN) : idesc_bf16(256, BN, false);
+  constexpr int BK_ELEMS = INT8 ? 128 : 64;
+  constexpr int K_STEPS = kTileBytesK / 32;
+  constexpr uint32_t kTmemCols = 512;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * HB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // four epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // the even CTA's barriers, addressed from either CTA
+  const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+  const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer (both)
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) armed[s] = -1;
+      bool ok = true;
+      Sched sc;
+      sched_init(p, sc, pair, npairs);
+      int tile, kb0, kb1;
+      while (ok && sched_next(p, sc, tile, kb0, kb1)) {
+        int mb, nb;
+        tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrGemmWait)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 4 * HB);
+          const uint32_t fb = full0 + stage * 8;
+          tma_load_2d_pair(sA + stage * HB, &tmA, fb, kb * BK_ELEMS, mb * 256 + rank * 128);
+          tma_load_2d_pair(sB + stage * HB, &tmB, fb, kb * BK_ELEMS, nb * BN + rank * 128);
+          armed[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && rank == 0) {  // the even CTA's full barriers count both CTAs' bytes
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s] >= 0) drain_wait(&full[s], static_cast<uint32_t>(armed[s]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------------- MMA issuer (even CTA)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      Sched sc;
+      sched_init(p, sc, pair, npairs);
+      int tile, kb0, kb1;
+      for (; ok && sched_next(p, sc, tile, kb0, kb1); ++local) {
+        const int buf = local & 1;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!wait_bar(&tempty[buf], (use & 1u) ^ 1u, abort_flag, p.err, kErrGemmWait)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_bar(&full[stage], phase, abort_flag, p.err, kErrGemmWait)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * HB);
+          const uint32_t b0 = smem_u32(sB + stage * HB);
+#pragma unroll
+          for (int k = 0; k < K_STEPS; ++k) {
+            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
+            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+            if constexpr (INT8)
+              umma_i8_pair(d_tmem, ad, bd, IDESC, acc);
+            else
+              umma_f16_pair(d_tmem, ad, bd, IDESC, acc);
+          }
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit_pair_mc(&tfull[buf], 0x3);
+      }
+      tc_commit_pair(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (both)
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const int slot_id = pair * 2 + static_cast<int>(rank);
+    int local = 0;
+    Sched sc;
+    sched_init(p, sc, pair, npairs);
+    int tile, kb0, kb1;
+    for (; sched_next(p, sc, tile, kb0, kb1); ++local) {
+      int mb, nb;
+      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      const int buf = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      bool ok = wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = mb * 256 + static_cast<int>(rank) * 128 + row_in_tile;
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
+      if (kb1 < p.k_blocks) {
+        // stream-K contributor: park this CTA's half of the partial tile in its slot
+        uint32_t* slot = p.sk_slots + (size_t(slot_id) * kBM + row_in_tile) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_wait_ld(r);
+          uint4* dst = reinterpret_cast<uint4*>(slot + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            __stcg(dst + i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+        }
+        __threadfence();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(&tempty[buf]);
+          else
+            mbar_arrive_cluster(tempty0 + buf * 8);
+          st_release_u64(p.sk_flags + slot_id * 4 + quarter, p.sk_seq);
+        }
+        continue;
+      }
+      int c_lo = pair;
+      if (kb0 > 0) {
+        c_lo = sk_owner(p, static_cast<long long>(tile) * p.k_blocks, npairs);
+        for (int c = c_lo; c < pair && ok; ++c) {
+          const unsigned long long* f = p.sk_flags + (c * 2 + static_cast<int>(rank)) * 4 + quarter;
+          bool seen = ld_acquire_u64(f) == p.sk_seq;
+          if (!seen) {
+            const uint64_t t0 = global_timer_ns();
+            while (!seen) {
+              seen = ld_acquire_u64(f) == p.sk_seq;
+              if (!seen && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
+                *abort_flag = 1u;
+                atomicCAS(p.err, 0u, kErrGemmWait);
+                break;
+              }
+            }
+          }
+          ok = __all_sync(0xffffffffu, seen);
+        }
+      }
+      epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo, pair, 2,
+                                   static_cast<int>(rank));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&tempty[buf]);
+        else
+          mbar_arrive_cluster(tempty0 + buf * 8);
+      }
+    }
+  }
+
+  // Neither CTA leaves while the other may still signal its barriers or read its tiles.
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+std::atomic<unsigned long long> g_sk_seq{0};
+bool trace_gemm();
+
+// A value no flag of the scratch can hold from an earlier launch: a per-process random
+// high half and a launch counter.
+unsigned long long next_sk_seq() {
+  static const unsigned long long salt =
+      (static_cast<unsigned long long>(std::random_device{}()) << 32) | 1ull;
+  return salt + (g_sk_seq.fetch_add(1) << 1);
+}
+
+// Fraction of SM-time a data-parallel schedule of `tiles` equal tiles keeps busy.
+double dp_efficiency(int tiles, int ctas) {
+  const int waves = (tiles + ctas - 1) / ctas;
+  return double(tiles) / (double(waves) * ctas);
+}
+
+// Stream-K pays a fixed cost per unit (partial-tile spill and reload, a second exposed
+// epilogue); measured on B200 it only wins when the data-parallel tail wastes a large
+// share of the SMs and the K loop is long enough to amortise it (1600 x 3072 x 12288:
+// 110 us vs 134 us; with K = 3072 it lost: 53-59 us vs 47 us).
+bool want_stream_k(int tiles, int units, int k_blocks) {
+  return dp_efficiency(tiles, std::min(units, tiles)) < 0.75 && k_blocks >= 128;
+}
+
 template <int BN, bool INT8, int EPI>
 int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, int K,
-                const GemmEpilogue& epi, cudaStream_t stream) {
+                const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
   const CUtensorMapDataType dt =
       INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -371,7 +834,7 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
     attr_done.fetch_or(bit);
   }
 
-  GemmParams p;
+  GemmParams p{};
   p.M = M;
   p.N = N;
   p.k_blocks = K / bk;
@@ -380,38 +843,199 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   p.epi = epi;
   p.err = ctx.err_flag;
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = std::min(tiles, ctx.num_sms);
-  kernel<<<grid, 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  const int sk_ctas = std::min(ctx.num_sms, kMaxSkCtas);
+  const long long iters = static_cast<long long>(tiles) * p.k_blocks;
+  const bool use_sk = scratch != nullptr && scratch_bytes >= kSkScratchBytes &&
+                      want_stream_k(tiles, ctx.num_sms, p.k_blocks) && iters >= 4LL * sk_ctas;
+  if (trace_gemm())
+    std::fprintf(stderr, "h3b gemm 1cta BN=%d M=%d N=%d K=%d tiles=%d sms=%d -> %s grid=%d\n", BN,
+                 M, N, K, tiles, ctx.num_sms, use_sk ? "stream-K" : "data-parallel",
+                 use_sk ? sk_ctas : std::min(tiles, ctx.num_sms));
+  if (!use_sk) {
+    const int grid = std::min(tiles, ctx.num_sms);
+    kernel<<<grid, 192, Cfg::kSmem, stream>>>(ta, tb, p);
+    return check_launch("gemm");
+  }
+  p.sk = 1;
+  p.sk_iters = iters;
+  p.sk_slots = static_cast<uint32_t*>(scratch);
+  p.sk_flags =
+      reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kSkFlagsOffset);
+  p.sk_seq = next_sk_seq();
+  // one CTA per SM, never more CTAs than SMs: every CTA is resident at once
+  kernel<<<sk_ctas, 192, Cfg::kSmem, stream>>>(ta, tb, p);
   return check_launch("gemm");
+}
+
+// Largest number of CTA pairs of the pair kernel that can be resident at once.
+template <bool INT8, int EPI>
+int pair_capacity(const DevCtx& ctx) {
+  static std::atomic<int> cap[64];
+  const int dev = ctx.device & 63;
+  int c = cap[dev].load();
+  if (c > 0) return c;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (ctx.num_sms / 2));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kPairSmem;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<INT8, EPI>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 0;
+  }
+  c = std::min(n, ctx.num_sms / 2);
+  if (c > 0) cap[dev].store(c);
+  return c;
+}
+
+// Returns 1 if the pair kernel is not usable here (caller falls back to single-CTA tiles).
+template <bool INT8, int EPI>
+int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, int K,
+                const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                cudaStream_t stream, int* rc) {
+  auto kernel = k_gemm_pair<INT8, EPI>;
+  static std::atomic<uint32_t> attr_done{0};
+  const uint32_t bit = 1u << (ctx.device & 31);
+  if (!(attr_done.load() & bit)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPairSmem)) != cudaSuccess) {
+      cudaGetLastError();
+      return 1;
+    }
+    attr_done.fetch_or(bit);
+  }
+  const int cap = pair_capacity<INT8, EPI>(ctx);
+  if (cap <= 0) return 1;
+  const CUtensorMapDataType dt =
+      INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int esize = INT8 ? 1 : 2;
+  const int bk = kTileBytesK / esize;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, A, dt, uint64_t(M), uint64_t(K), uint64_t(K) * esize, 128, bk) ||
+      !make_tmap_2d(&tb, B, dt, uint64_t(N), uint64_t(K), uint64_t(K) * esize, 128, bk)) {
+    *rc = set_error(-3, "gemm: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+    return 0;
+  }
+  GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.k_blocks = K / bk;
+  p.m_tiles = (M + 255) / 256;
+  p.n_tiles = N / 256;
+  p.epi = epi;
+  p.err = ctx.err_flag;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
+  const long long iters = static_cast<long long>(tiles) * p.k_blocks;
+  const bool use_sk = scratch != nullptr && scratch_bytes >= kSkScratchBytes &&
+                      want_stream_k(tiles, cap, p.k_blocks) && iters >= 4LL * sk_pairs;
+  if (trace_gemm())
+    std::fprintf(stderr, "h3b gemm pair M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n", M, N,
+                 K, tiles, cap, use_sk ? "stream-K" : "data-parallel",
+                 use_sk ? sk_pairs : std::min(tiles, cap));
+  if (use_sk) {
+    GemmParams q = p;
+    q.sk = 1;
+    q.sk_iters = iters;
+    q.sk_slots = static_cast<uint32_t*>(scratch);
+    q.sk_flags =
+        reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kSkFlagsOffset);
+    q.sk_seq = next_sk_seq();
+    // never more pairs than can be resident at once (occupancy query above)
+    kernel<<<2 * sk_pairs, 192, kPairSmem, stream>>>(ta, tb, q);
+    *rc = check_launch("gemm_pair");
+    return 0;
+  }
+  kernel<<<2 * std::min(tiles, cap), 192, kPairSmem, stream>>>(ta, tb, p);
+  *rc = check_launch("gemm_pair");
+  return 0;
+}
+
+// H3B_TRACE_GEMM=1 prints each GEMM's schedule to stderr (diagnostics only).
+bool trace_gemm() {
+  static const bool on = [] {
+    const char* v = std::getenv("H3B_TRACE_GEMM");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
+bool single_cta_forced() {
+  static const bool forced = [] {
+    const char* v = std::getenv("H3B_GEMM_SINGLE_CTA");
+    return v && v[0] == '1';
+  }();
+  return forced;
 }
 
 template <int BN>
 int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
-                  const GemmEpilogue& epi, cudaStream_t s) {
+                  const GemmEpilogue& epi, void* ws, size_t wsb, cudaStream_t s) {
   switch (epi.kind) {
-    case kEpiBias: return launch_impl<BN, false, kEpiBias>(ctx, A, B, M, N, K, epi, s);
-    case kEpiGelu: return launch_impl<BN, false, kEpiGelu>(ctx, A, B, M, N, K, epi, s);
-    case kEpiRope: return launch_impl<BN, false, kEpiRope>(ctx, A, B, M, N, K, epi, s);
+    case kEpiBias: return launch_impl<BN, false, kEpiBias>(ctx, A, B, M, N, K, epi, ws, wsb, s);
+    case kEpiGelu: return launch_impl<BN, false, kEpiGelu>(ctx, A, B, M, N, K, epi, ws, wsb, s);
+    case kEpiRope: return launch_impl<BN, false, kEpiRope>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     case kEpiGateResid:
-      return launch_impl<BN, false, kEpiGateResid>(ctx, A, B, M, N, K, epi, s);
+      return launch_impl<BN, false, kEpiGateResid>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
   }
 }
 
 }  // namespace
 
+size_t gemm_scratch_bytes() { return kSkScratchBytes; }
+
+template <int EPI>
+bool try_pair_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
+                   const GemmEpilogue& epi, void* ws, size_t wsb, cudaStream_t s, int* rc) {
+  return launch_pair<false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
+}
+
 int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
-                     const GemmEpilogue& epi, cudaStream_t stream) {
+                     const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                     cudaStream_t stream) {
   if (M <= 0) return 0;
-  if (N % 256 == 0) return dispatch_bf16<256>(ctx, A, B, M, N, K, epi, stream);
-  return dispatch_bf16<128>(ctx, A, B, M, N, K, epi, stream);
+  if (N % 256 == 0 && M >= 256 && !single_cta_forced()) {
+    int rc = 0;
+    bool done = false;
+    switch (epi.kind) {
+      case kEpiBias:
+        done = try_pair_bf16<kEpiBias>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        break;
+      case kEpiGelu:
+        done = try_pair_bf16<kEpiGelu>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        break;
+      case kEpiRope:
+        done = try_pair_bf16<kEpiRope>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        break;
+      case kEpiGateResid:
+        done = try_pair_bf16<kEpiGateResid>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                            stream, &rc);
+        break;
+      default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
+    }
+    if (done) return rc;
+  }
+  if (N % 256 == 0)
+    return dispatch_bf16<256>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+  return dispatch_bf16<128>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
 }
 
 int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
-                   const GemmEpilogue& epi, cudaStream_t stream) {
+                   const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                   cudaStream_t stream) {
   if (M <= 0) return 0;
-  if (N % 256 == 0) return launch_impl<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, stream);
-  return launch_impl<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, stream);
+  if (N % 256 == 0 && M >= 256 && !single_cta_forced()) {
+    int rc = 0;
+    if (launch_pair<true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream,
+                                       &rc) == 0)
+      return rc;
+  }
+  if (N % 256 == 0)
+    return launch_impl<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                               stream);
+  return launch_impl<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                             stream);
 }
 
 }  // namespace h3b

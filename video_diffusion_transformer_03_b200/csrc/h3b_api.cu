@@ -131,21 +131,28 @@ int check_weights(const h3b_block_weights* w) {
   return H3B_OK;
 }
 
-size_t arena_bytes(const h3b_dims* d, int n) {
+size_t activations_bytes(const h3b_dims* d, int n) {
   return a256(size_t(n) * std::max(4 * d->d, d->d_ff) * 2);
 }
 
+size_t arena_bytes(const h3b_dims* d, int n) {
+  return activations_bytes(d, n) + a256(gemm_scratch_bytes());
+}
+
 // Buffers of one block inside the arena: qkv [n, 3d] then attention output [n, d]; the
-// MLP hidden activations [n, d_ff] reuse the same bytes once both are dead.
+// MLP hidden activations [n, d_ff] reuse the same bytes once both are dead.  The GEMMs'
+// stream-K scratch follows.
 struct BlockBufs {
   bf16* qkv;
   bf16* attn;
   bf16* g;
+  void* gemm_scratch;
 };
 
 BlockBufs carve_block(const h3b_dims* d, int n, void* arena) {
   bf16* base = static_cast<bf16*>(arena);
-  return BlockBufs{base, base + size_t(n) * 3 * d->d, base};
+  return BlockBufs{base, base + size_t(n) * 3 * d->d, base,
+                   static_cast<uint8_t*>(arena) + activations_bytes(d, n)};
 }
 
 int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_weights* w,
@@ -164,7 +171,7 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   e.head_dim = d->head_dim;
   e.out = b.qkv;
   e.ld_out = 3 * D;
-  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_qkv), n, 3 * D, D, e, s)))
+  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_qkv), n, 3 * D, D, e, b.gemm_scratch, gemm_scratch_bytes(), s)))
     return rc;
   if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, s))) return rc;
 
@@ -174,7 +181,7 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   e.gate = mod + 2 * D;
   e.out = x;
   e.ld_out = D;
-  if ((rc = launch_gemm_bf16(ctx, b.attn, reinterpret_cast<const bf16*>(w->w_o), n, D, D, e, s)))
+  if ((rc = launch_gemm_bf16(ctx, b.attn, reinterpret_cast<const bf16*>(w->w_o), n, D, D, e, b.gemm_scratch, gemm_scratch_bytes(), s)))
     return rc;
   if ((rc = launch_ln_modulate(x, n, D, d->ln_eps, mod + 3 * D, mod + 4 * D, h, s))) return rc;
 
@@ -183,7 +190,7 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   e.bias = reinterpret_cast<const bf16*>(w->b_fc1);
   e.out = b.g;
   e.ld_out = d->d_ff;
-  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_fc1), n, d->d_ff, D, e, s)))
+  if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_fc1), n, d->d_ff, D, e, b.gemm_scratch, gemm_scratch_bytes(), s)))
     return rc;
 
   e = GemmEpilogue();
@@ -192,7 +199,7 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   e.gate = mod + 5 * D;
   e.out = x;
   e.ld_out = D;
-  if ((rc = launch_gemm_bf16(ctx, b.g, reinterpret_cast<const bf16*>(w->w_fc2), n, D, d->d_ff, e, s)))
+  if ((rc = launch_gemm_bf16(ctx, b.g, reinterpret_cast<const bf16*>(w->w_fc2), n, D, d->d_ff, e, b.gemm_scratch, gemm_scratch_bytes(), s)))
     return rc;
   if (mod_next && (rc = launch_ln_modulate(x, n, D, d->ln_eps, mod_next, mod_next + D, h, s)))
     return rc;
@@ -336,6 +343,8 @@ int h3b_sync_status(void* stream) {
   }
   return H3B_OK;
 }
+
+size_t h3b_gemm_workspace_size(void) { return gemm_scratch_bytes(); }
 
 size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens) {
   if (check_dims(dims) || n_tokens < 0) return 0;
@@ -499,7 +508,8 @@ int h3b_quantize_rows(const h3b_bf16* a, int rows, int cols, int8_t* q, float* s
 
 int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t* w_q,
                      const float* w_scale, const float* bias, const float* gate, h3b_bf16* resid,
-                     int8_t* act_q, float* row_scale, int32_t* acc_out, void* stream) {
+                     int8_t* act_q, float* row_scale, int32_t* acc_out, void* ws,
+                     size_t ws_bytes, void* stream) {
   if (M < 0 || K <= 0 || K % 128 || K > 32768 || n_out <= 0 || n_out % 128)
     return set_error(H3B_EINVAL, "fc2_int8_row: K=%d must be a multiple of 128 <= 32768, n_out=%d a multiple of 128", K, n_out);
   const void* ptrs[7] = {act, w_q, w_scale, gate, resid, act_q, row_scale};
@@ -522,12 +532,13 @@ int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t*
   e.row_scale = row_scale;
   e.col_scale = w_scale;
   e.acc_out = acc_out;
-  return launch_gemm_i8(ctx, act_q, w_q, M, n_out, K, e, s);
+  if (ws && !al16(ws)) return set_error(H3B_EINVAL, "fc2_int8_row: misaligned workspace");
+  return launch_gemm_i8(ctx, act_q, w_q, M, n_out, K, e, ws, ws_bytes, s);
 }
 
 int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
                   const h3b_bf16* bias, const float* gate, const float* rope_cs, int rope_cols,
-                  int head_dim, h3b_bf16* out, void* stream) {
+                  int head_dim, h3b_bf16* out, void* ws, size_t ws_bytes, void* stream) {
   if (M < 0 || K <= 0 || K % 64 || N <= 0 || N % 128)
     return set_error(H3B_EINVAL, "gemm_bf16: K=%d must be a multiple of 64, N=%d of 128", K, N);
   if (epilogue < H3B_EPI_BIAS || epilogue > H3B_EPI_GATE_RESID)
@@ -551,8 +562,9 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
   e.head_dim = head_dim;
   e.out = reinterpret_cast<bf16*>(out);
   e.ld_out = N;
+  if (ws && !al16(ws)) return set_error(H3B_EINVAL, "gemm_bf16: misaligned workspace");
   return launch_gemm_bf16(ctx, reinterpret_cast<const bf16*>(A), reinterpret_cast<const bf16*>(B),
-                          M, N, K, e, static_cast<cudaStream_t>(stream));
+                          M, N, K, e, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim, h3b_bf16* out,

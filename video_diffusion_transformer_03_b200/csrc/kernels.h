@@ -48,12 +48,19 @@ struct GemmEpilogue {
   int32_t* acc_out = nullptr;        // int8 path, [M, N] or null
 };
 
+// Bytes of stream-K scratch the GEMM can use (partial-tile slots + flags).
+size_t gemm_scratch_bytes();
+
 // out = A[M, K] * B[N, K]^T with epilogue; bf16 inputs.  K % 64 == 0, N % 128 == 0.
+// scratch (>= gemm_scratch_bytes(), or null) enables the stream-K schedule when the
+// tile count quantises badly onto the SMs.
 int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
-                     const GemmEpilogue& epi, cudaStream_t stream);
+                     const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                     cudaStream_t stream);
 // Same for int8 inputs (int32 accumulate, kEpiInt8Deq).  K % 128 == 0, N % 128 == 0.
 int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
-                   const GemmEpilogue& epi, cudaStream_t stream);
+                   const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                   cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention (tcgen05)
 int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_heads,

@@ -54,6 +54,7 @@ _SIGS = {
     "h3b_launch_count": (ctypes.c_uint64, []),
     "h3b_sync_status": (_I, [_P]),
     "h3b_workspace_size": (_SZ, [ctypes.POINTER(Dims), _I]),
+    "h3b_gemm_workspace_size": (_SZ, []),
     "h3b_denoise_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I]),
     "h3b_adaln_modulation": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "h3b_rope_table": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I, _P, _P]),
@@ -69,8 +70,8 @@ _SIGS = {
                               _P, _P, _P, _SZ, _P]),
     "h3b_token_reduce": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "h3b_quantize_rows": (_I, [_P, _I, _I, _P, _P, _P]),
-    "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P]),
+    "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P]),
     "h3b_layer_mask": (_I, [_P, _I, _I, _I, _P]),
 }
@@ -146,6 +147,16 @@ def make_block_weights(p) -> BlockWeights:
         _dev(p[k], torch.bfloat16, k)
     return BlockWeights(*[_ptr(p[k]) for k in
                           ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")])
+
+
+def gemm_workspace_size() -> int:
+    return int(lib.h3b_gemm_workspace_size())
+
+
+def _wsargs(ws):
+    if ws is None:
+        return None, 0
+    return _ptr(ws), ws.numel() * ws.element_size()
 
 
 def workspace_size(dims: Dims, n_tokens: int) -> int:
@@ -253,21 +264,24 @@ def quantize_rows(a, q, scale, stream=None) -> None:
 
 
 def fc2_int8_row(act, w_q, w_scale, bias, gate, resid, act_q, row_scale, acc_out=None,
-                 stream=None) -> None:
+                 ws=None, stream=None) -> None:
     _dev(act, torch.bfloat16, "act"); _dev(w_q, torch.int8, "w_q"); _dev(resid, torch.bfloat16, "resid")
     M, K = act.shape
+    wp, wb = _wsargs(ws)
     _check(lib.h3b_fc2_int8_row(_ptr(act), M, K, w_q.shape[0], _ptr(w_q), _ptr(w_scale),
                                 _ptr(bias), _ptr(gate), _ptr(resid), _ptr(act_q), _ptr(row_scale),
-                                _ptr(acc_out), _stream(stream)))
+                                _ptr(acc_out), wp, wb, _stream(stream)))
 
 
 def gemm_bf16(A, B, epilogue, bias, out, gate=None, rope_cs=None, rope_cols=0, head_dim=128,
-              stream=None) -> None:
+              ws=None, stream=None) -> None:
     _dev(A, torch.bfloat16, "A"); _dev(B, torch.bfloat16, "B"); _dev(out, torch.bfloat16, "out")
     M, K = A.shape
     N = B.shape[0]
+    wp, wb = _wsargs(ws)
     _check(lib.h3b_gemm_bf16(_ptr(A), _ptr(B), M, N, K, epilogue, _ptr(bias), _ptr(gate),
-                             _ptr(rope_cs), rope_cols, head_dim, _ptr(out), _stream(stream)))
+                             _ptr(rope_cs), rope_cols, head_dim, _ptr(out), wp, wb,
+                             _stream(stream)))
 
 
 def attention(qkv, n_heads, head_dim, out, stream=None) -> None:
