@@ -164,6 +164,27 @@ int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const fl
                       int compute_h, h3b_bf16* x, h3b_bf16* h, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* h3b_block_forward without a caller-supplied workspace, for callers that cannot allocate
+ * device memory: plug-in hosts that hand a module only its input and output buffers,
+ * deployments whose memory plan is fixed before launch, and latency-critical loops that
+ * must not call cudaMalloc (it can synchronise the device).  The paper has no
+ * counterpart; the block math, arguments and results are those of h3b_block_forward.
+ *
+ * The workspace is one static device array of H3B_NOALLOC_WORKSPACE_BYTES (64 MiB) inside
+ * the library; every GPU that loads the library holds it until the process exits.  A call
+ * needs h3b_workspace_size(dims, n_tokens) bytes of it (at d = 3072, d_ff = 12288 that is
+ * 1,877 tokens at most) and returns H3B_EWORKSPACE, launching nothing, when the block does
+ * not fit.  The first call on a device looks up the array's device address (make that
+ * first call before any stream capture).  All calls share the array and nothing in it has
+ * to start at zero (every region is written before it is read); calls whose executions
+ * overlap on the GPU -- concurrent streams, or threads sharing a device -- race on it, so
+ * serialise them.  Nothing here allocates or frees memory. */
+#define H3B_NOALLOC_WORKSPACE_BYTES (64u << 20)
+int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,
+                              const float* mod, const float* mod_next, const float* rope_cs,
+                              int n_tokens, int compute_h, h3b_bf16* x, h3b_bf16* h,
+                              void* stream);
+
 /* Per-stream final AdaLN fused with the Euler update (dothoosh.com, "DiT fusions and
  * memory management": final AdaLN bound to the video/audio offsets of one residual
  * buffer; aihot.vn section 2: linear sigma grid):

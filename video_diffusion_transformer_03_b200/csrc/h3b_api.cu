@@ -16,6 +16,11 @@
 // Set (first code wins) by any kernel whose bounded wait gave up; one per device.
 __device__ uint32_t g_h3b_wait_error = 0u;
 
+// Block workspace of h3b_block_forward_noalloc: a fixed array in the module's device
+// image, so that entry point never allocates.  In host code this name only stands for
+// the symbol; its device address comes from cudaGetSymbolAddress (per device).
+static __device__ __align__(256) uint8_t g_noalloc_ws[H3B_NOALLOC_WORKSPACE_BYTES];
+
 namespace h3b {
 
 namespace {
@@ -408,6 +413,46 @@ int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const fl
                      arena_bytes(dims, n_tokens), ws_bytes);
   DevCtx ctx;
   if ((rc = get_ctx(&ctx))) return rc;
+  return block_forward_impl(ctx, dims, w, mod, mod_next, rope_cs, n_tokens, compute_h != 0,
+                            reinterpret_cast<bf16*>(x), reinterpret_cast<bf16*>(h), ws,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,
+                              const float* mod, const float* mod_next, const float* rope_cs,
+                              int n_tokens, int compute_h, h3b_bf16* x, h3b_bf16* h,
+                              void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_weights(w))) return rc;
+  if (n_tokens < 0 || n_tokens > (1 << 24)) return set_error(H3B_EINVAL, "n_tokens=%d", n_tokens);
+  if (!mod || !rope_cs || !x || !h || !al16(mod) || !al16(rope_cs) || !al16(x) || !al16(h) ||
+      (mod_next && !al16(mod_next)))
+    return set_error(H3B_EINVAL, "block_forward_noalloc: NULL or misaligned pointer");
+  const size_t need = arena_bytes(dims, n_tokens);
+  if (need > H3B_NOALLOC_WORKSPACE_BYTES)
+    return set_error(H3B_EWORKSPACE,
+                     "block_forward_noalloc: %d tokens need %zu workspace bytes, the static "
+                     "workspace holds %zu",
+                     n_tokens, need, size_t(H3B_NOALLOC_WORKSPACE_BYTES));
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  // Device address of the static workspace, looked up once per device with that device
+  // current (the host-side name of a __device__ array is not a device pointer).
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[ctx.device]) {
+      void* p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_ws);
+      if (e != cudaSuccess || !p)
+        return set_error(H3B_ECUDA, "block_forward_noalloc: cudaGetSymbolAddress: %s",
+                         cudaGetErrorString(e));
+      addr[ctx.device] = p;
+    }
+    ws = addr[ctx.device];
+  }
   return block_forward_impl(ctx, dims, w, mod, mod_next, rope_cs, n_tokens, compute_h != 0,
                             reinterpret_cast<bf16*>(x), reinterpret_cast<bf16*>(h), ws,
                             static_cast<cudaStream_t>(stream));

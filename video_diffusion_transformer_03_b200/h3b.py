@@ -61,6 +61,8 @@ _SIGS = {
     "h3b_ln_modulate": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
     "h3b_block_forward": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _P, _P, _P,
                                _I, _I, _P, _P, _P, _SZ, _P]),
+    "h3b_block_forward_noalloc": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _P,
+                                       _P, _P, _I, _I, _P, _P, _P]),
     "h3b_final_euler": (_I, [_P, _I, _I, _I, _F, _P, _F, _F, _P, _P]),
     "h3b_denoise_step": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                               ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P, _P,
@@ -200,6 +202,21 @@ def block_forward(dims: Dims, weights: BlockWeights, mod, mod_next, rope_cs, x, 
                                  _ptr(mod_next), _ptr(rope_cs), x.shape[0], int(bool(compute_h)),
                                  _ptr(x), _ptr(h), _ptr(ws), ws.numel() * ws.element_size(),
                                  _stream(stream)))
+
+
+NOALLOC_WORKSPACE_BYTES = 64 << 20
+
+
+def block_forward_noalloc(dims: Dims, weights: BlockWeights, mod, mod_next, rope_cs, x, h,
+                          compute_h: bool, stream=None) -> None:
+    """h3b_block_forward with the library's static workspace instead of a caller buffer
+    (for callers that cannot allocate device memory).  Calls that overlap on the GPU
+    share that workspace and race; serialise them."""
+    _dev(x, torch.bfloat16, "x"); _dev(h, torch.bfloat16, "h"); _dev(mod, torch.float32, "mod")
+    _check(lib.h3b_block_forward_noalloc(ctypes.byref(dims), ctypes.byref(weights), _ptr(mod),
+                                         _ptr(mod_next), _ptr(rope_cs), x.shape[0],
+                                         int(bool(compute_h)), _ptr(x), _ptr(h),
+                                         _stream(stream)))
 
 
 def final_euler(x_l, n_video, eps, final_mod, sigma, sigma_next, x_state, stream=None) -> None:
