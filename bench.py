@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--kernel", default=None,
                     help="time one kernel of the block alone on the workload shapes (for ncu)")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel from the host instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -332,6 +334,15 @@ def run_gpu(args):
     for _ in range(args.warmup):
         model.run(x)
     h3b.sync_status()
+    graph = None
+    launches_per_denoise = None
+    if not args.no_graph:
+        c0 = h3b.launch_count()
+        graph = model.capture(x)
+        launches_per_denoise = h3b.launch_count() - c0
+        for _ in range(2):
+            graph.replay()
+        h3b.sync_status()
     props = torch.cuda.get_device_properties(dev)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
 
@@ -344,10 +355,15 @@ def run_gpu(args):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        model.run(x)
+        if graph is not None:
+            graph.replay()
+        else:
+            model.run(x)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     launches = h3b.launch_count() - launches0
+    if graph is not None:  # graph replays launch the captured kernels without host calls
+        launches = launches_per_denoise * args.steps
     clk = clocks.stop()
     barrier()
     h3b.sync_status()
@@ -401,7 +417,9 @@ def run_gpu(args):
                        "l2": "no flush: each pass streams "
                              f"{sum(p['w_qkv'].numel() + p['w_o'].numel() + p['w_fc1'].numel() + p['w_fc2'].numel() for p in model.params) * 2 / 1e9:.2f}"
                              " GB of weights, more than the 126 MB L2",
-                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                       "launch": "CUDA graph of one complete denoise, replayed" if graph
+                                 is not None else "host launches"},
             "tflops": tflops,
             "tensor_frac": tflops / world / peaks["bf16_tflops_sustained"],
             "tensor_frac_peak": f"{peak_src} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s",
@@ -411,6 +429,7 @@ def run_gpu(args):
                                for kk, vv in v.items()} for k, v in breakdown.items()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
+    del graph
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -525,6 +525,12 @@ __global__ void __launch_bounds__(192, 1)
       }
       epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo,
                                    static_cast<int>(blockIdx.x), 1, 0);
+      // hand the consumed flags back at zero, so a replay of this launch (same sequence
+      // value, e.g. from a CUDA graph) waits for its own contributors again
+      __syncwarp();
+      if (lane == 0)
+        for (int src = c_lo; src < static_cast<int>(blockIdx.x); ++src)
+          p.sk_flags[src * 4 + quarter] = 0ull;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -763,6 +769,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo, pair, 2,
                                    static_cast<int>(rank));
+      __syncwarp();
+      if (lane == 0)
+        for (int src = c_lo; src < pair; ++src)
+          p.sk_flags[(src * 2 + static_cast<int>(rank)) * 4 + quarter] = 0ull;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

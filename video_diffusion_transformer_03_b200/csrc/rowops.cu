@@ -12,7 +12,7 @@ namespace h3b {
 
 namespace {
 
-constexpr int kRowWarps = 8;  // rows per 256-thread block
+constexpr int kRowWarps = 4;  // rows per 128-thread block
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -70,7 +70,7 @@ __device__ __forceinline__ void row_stats(const float (&v)[NV][8], int d, float 
 // h = LN(x)(1 + scale) + shift.  FROM_STATE: x is the fp32 state; it is first rounded to
 // bf16 (the block input) and written to x_res.
 template <int NV, bool FROM_STATE>
-__global__ void __launch_bounds__(256) k_ln_modulate(const void* __restrict__ xin, int n,
+__global__ void __launch_bounds__(128) k_ln_modulate(const void* __restrict__ xin, int n,
                                                      float eps, const float* __restrict__ shift,
                                                      const float* __restrict__ scale,
                                                      bf16* __restrict__ x_res,
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(256) k_ln_modulate(const void* __restrict__ xi
 // v = LN(x_l)(1 + scale_s) + shift_s (s = video below n_video, else audio);
 // x_state += dt * v.
 template <int NV>
-__global__ void __launch_bounds__(256) k_final_euler(const bf16* __restrict__ xl, int n,
+__global__ void __launch_bounds__(128) k_final_euler(const bf16* __restrict__ xl, int n,
                                                      int n_video, float eps,
                                                      const float* __restrict__ fmod,
                                                      float dt, float* __restrict__ xs) {
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(256) k_adaln_gemv(const bf16* __restrict__ w,
                                                     const bf16* __restrict__ b,
                                                     const bf16* __restrict__ c, int n_out,
                                                     int c_dim, float* __restrict__ out) {
-  const int j = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (j >= n_out) return;
   const int lane = threadIdx.x & 31;
   const uint4* wr = reinterpret_cast<const uint4*>(w + size_t(j) * c_dim);
@@ -344,7 +344,7 @@ int launch_ln_modulate(const bf16* x, int n, int d, float eps, const float* shif
                        const float* scale, bf16* h, cudaStream_t stream) {
   if (n <= 0) return 0;
   const int grid = (n + kRowWarps - 1) / kRowWarps;
-  H3B_NV_SWITCH(d / 256, (k_ln_modulate<NV, false><<<grid, 256, 0, stream>>>(
+  H3B_NV_SWITCH(d / 256, (k_ln_modulate<NV, false><<<grid, 32 * kRowWarps, 0, stream>>>(
                              x, n, eps, shift, scale, nullptr, h)));
   return check_launch("ln_modulate");
 }
@@ -354,7 +354,7 @@ int launch_ln_modulate_from_state(const float* x_state, int n, int d, float eps,
                                   bf16* h, cudaStream_t stream) {
   if (n <= 0) return 0;
   const int grid = (n + kRowWarps - 1) / kRowWarps;
-  H3B_NV_SWITCH(d / 256, (k_ln_modulate<NV, true><<<grid, 256, 0, stream>>>(
+  H3B_NV_SWITCH(d / 256, (k_ln_modulate<NV, true><<<grid, 32 * kRowWarps, 0, stream>>>(
                              x_state, n, eps, shift, scale, x_res, h)));
   return check_launch("ln_modulate_from_state");
 }
@@ -364,7 +364,7 @@ int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,
                        cudaStream_t stream) {
   if (n <= 0) return 0;
   const int grid = (n + kRowWarps - 1) / kRowWarps;
-  H3B_NV_SWITCH(d / 256, (k_final_euler<NV><<<grid, 256, 0, stream>>>(
+  H3B_NV_SWITCH(d / 256, (k_final_euler<NV><<<grid, 32 * kRowWarps, 0, stream>>>(
                              x_l, n, n_video, eps, final_mod, dt_sigma, x_state)));
   return check_launch("final_euler");
 }
@@ -407,7 +407,7 @@ int launch_quantize_rows(const bf16* a, int rows, int cols, int8_t* q, float* sc
 int launch_adaln_gemv(const bf16* w, const bf16* b, const bf16* c, int n_out, int c_dim,
                       float* out, cudaStream_t stream) {
   if (n_out <= 0) return 0;
-  const int grid = (n_out + kRowWarps - 1) / kRowWarps;
+  const int grid = (n_out + 7) / 8;
   k_adaln_gemv<<<grid, 256, 0, stream>>>(w, b, c, n_out, c_dim, out);
   return check_launch("adaln_gemv");
 }

@@ -78,6 +78,15 @@ class DiTDenoiser:
         for i in range(self.cfg.run_steps if n_run is None else n_run):
             self.step(x_state, i, stream)
 
+    def capture(self, x_state: torch.Tensor, n_run: Optional[int] = None) -> torch.cuda.CUDAGraph:
+        """Record a whole denoise of x_state (in place) as one CUDA graph; replaying it
+        relaunches every kernel of every Euler step without host work.  Call run() once
+        first on this device (the library sets kernel attributes on first use)."""
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.run(x_state, n_run)
+        return graph
+
     def run_host(self, x_host_in: torch.Tensor, x_host_out: torch.Tensor,
                  x_state_dev: torch.Tensor, n_run: Optional[int] = None, stream=None) -> None:
         h3b.denoise_host(self.dims, self.grid, self.weights, self.active, self.mods,
