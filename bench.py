@@ -39,7 +39,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # dram bytes per launch from an ncu capture, keyed by kernel; only used while the kernel
 # source still hashes to the value recorded with it.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --set full, one launch of the dit512 shape after 3 warm-ups (profiles/)
+    "gemm_fc2_gate": {"bytes": 137959168 + 16381440, "src": "gemm_tc.cu",
+                      "src_sha": "ba40d519c5ab2266"},
+    "gemm_fc1_gelu": {"bytes": 85616896 + 15185152, "src": "gemm_tc.cu",
+                      "src_sha": "ba40d519c5ab2266"},
+}
 
 
 def parse_args():
@@ -54,6 +60,8 @@ def parse_args():
     ap.add_argument("--kernel", default=None,
                     help="time one kernel of the block alone on the workload shapes (for ncu)")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--no-also", action="store_true",
+                    help="skip the secondary measurements of the other workloads")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying a CUDA graph")
     return ap.parse_args()
@@ -291,6 +299,113 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3)
     return out
 
 
+def time_denoise(cfg_name, dev, reps, warm=1):
+    """Device time of complete denoises of another workload (graph replays)."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    from video_diffusion_transformer_03_b200.pipeline import DiTDenoiser
+    cfg = synth.CONFIGS[cfg_name]
+    model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
+    counts, _ = workload_counts(cfg, model.active)
+    x = synth.latent_noise(cfg, device=str(dev))
+    for _ in range(warm):
+        model.run(x)
+    graph = model.capture(x)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    h3b.sync_status()
+    ms = e0.elapsed_time(e1) / reps
+    del graph, model
+    torch.cuda.empty_cache()
+    return {"workload": workload_name(cfg), "ms_per_denoise": ms,
+            "tokens_per_s": counts["tokens"] / (ms * 1e-3),
+            "tflops": counts["flops"] / (ms * 1e-3) / 1e12, "denoises_timed": reps}
+
+
+def time_int8_fc2(dev, peaks, reps=10):
+    """The int8 row-scaled FC2 workload: quantise 8192 x 12288 activations, int8 GEMM
+    against 3072 x 12288 int8 weights, dequantise + gated residual."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    c = synth.INT8_CONFIG
+    inp = synth.int8_fc2_inputs(c, device=str(dev))
+    M, K, N = c.M, c.K, c.n_out
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    wsc = torch.empty((N,), dtype=torch.float32, device=dev)
+    h3b.quantize_rows(inp["w"], wq, wsc)
+    aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    rs = torch.empty((M,), dtype=torch.float32, device=dev)
+    resid = inp["resid"]
+    ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
+    run = lambda: h3b.fc2_int8_row(inp["act"], wq, wsc, None, inp["gate"], resid, aq, rs, None, ws=ws)
+    q_only = lambda: h3b.quantize_rows(inp["act"], aq, rs)
+    out = {}
+    for name, fn in (("fc2_int8_row", run), ("quantize_rows", q_only)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        out[name] = e0.elapsed_time(e1) / reps
+    h3b.sync_status()
+    q_bytes = 3 * M * K + 4 * M
+    int8_peak = 2 * peaks["bf16_tflops"]
+    gemm_ms = max(out["fc2_int8_row"] - out["quantize_rows"], 1e-6)
+    res = {"workload": f"fc2_int8_row M={M} K={K} N={N}", "ms": out["fc2_int8_row"],
+           "tops_whole_call": 2 * M * N * K / (out["fc2_int8_row"] * 1e-3) / 1e12,
+           "quantize_ms": out["quantize_rows"],
+           "quantize_gbs": q_bytes / (out["quantize_rows"] * 1e-3) / 1e9,
+           "quantize_hbm_frac": q_bytes / (out["quantize_rows"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+           "int8_gemm_tops": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12,
+           "int8_gemm_frac": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12 / int8_peak,
+           "int8_peak_tops": int8_peak, "int8_peak_note": "measured bf16 burst x 2 (nominal ratio)"}
+    del inp, wq, aq, resid
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_token_pairing(dev, peaks, reps=20):
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    cfg = synth.CONFIGS["dit768x1344"]
+    t, h, w = cfg.grid
+    n, nr, d = cfg.n_tokens, cfg.n_video_reduced + cfg.n_audio, cfg.d
+    x = torch.randn(n, d, device=dev).to(torch.bfloat16)
+    red = torch.empty(nr, d, dtype=torch.bfloat16, device=dev)
+    back = torch.empty_like(x)
+    res = {}
+    for name, fn, nbytes in (
+            ("pair", lambda: h3b.token_reduce(h3b.PAIR, x, red, None, t, h, w, cfg.n_audio),
+             2 * (n * d + nr * d)),
+            ("unpair_bypass", lambda: h3b.token_reduce(h3b.UNPAIR, red, back, x, t, h, w, cfg.n_audio),
+             2 * (nr * d + 2 * n * d))):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    h3b.sync_status()
+    res["shape"] = f"{cfg.name} stream: {n} tokens x {d} bf16 -> {nr} tokens"
+    return res
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -427,6 +542,16 @@ def run_gpu(args):
     if breakdown:
         line["kernels"] = {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv)
                                for kk, vv in v.items()} for k, v in breakdown.items()}
+    if rank == 0 and world == 1 and not args.no_also:
+        del graph
+        graph = None
+        also = {}
+        for name, reps in (("dit512_tokred", 20), ("dit768x1344", 2)):
+            if name != args.config:
+                also[name] = time_denoise(name, dev, reps)
+        also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
+        also["token_pairing"] = time_token_pairing(dev, peaks)
+        line["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
     del graph

@@ -23,6 +23,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <random>
+#include <string>
 
 namespace h3b {
 
@@ -556,27 +557,33 @@ __global__ void __launch_bounds__(192, 1)
 #ifndef H3B_PAIR_STAGES
 #define H3B_PAIR_STAGES 6
 #endif
-constexpr int kPairStages = H3B_PAIR_STAGES;
-constexpr uint32_t kPairHalfBytes = 128 * kTileBytesK;  // 16 KB: 128 rows x 128 B
-constexpr size_t kPairSmem = 1024 + size_t(kPairStages) * 2 * kPairHalfBytes + 256;
+template <int BN>
+struct PairCfg {
+  static constexpr int kStages = BN == 256 ? H3B_PAIR_STAGES : 8;
+  static constexpr uint32_t kABytes = 128 * kTileBytesK;       // this CTA's 128 rows of A
+  static constexpr uint32_t kBBytes = (BN / 2) * kTileBytesK;  // this CTA's half of B
+  static constexpr uint32_t kTmemCols = 2 * BN;
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * (kABytes + kBBytes) + 256;
+};
 
-template <bool INT8, int EPI>
+template <int BN, bool INT8, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
-  constexpr int BN = 256;
-  constexpr int STAGES = kPairStages;
-  constexpr uint32_t HB = kPairHalfBytes;
+  using Cfg = PairCfg<BN>;
+  constexpr int STAGES = Cfg::kStages;
+  constexpr uint32_t HA = Cfg::kABytes;
+  constexpr uint32_t HB = Cfg::kBBytes;
   constexpr uint32_t IDESC = INT8 ? idesc_s8(256, BN) : idesc_bf16(256, BN, false);
   constexpr int BK_ELEMS = INT8 ? 128 : 64;
   constexpr int K_STEPS = kTileBytesK / 32;
-  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kTmemCols = Cfg::kTmemCols;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * HB;
+  uint8_t* sB = smem + STAGES * HA;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -640,10 +647,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             ok = false;
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 4 * HB);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (HA + HB));
           const uint32_t fb = full0 + stage * 8;
-          tma_load_2d_pair(sA + stage * HB, &tmA, fb, kb * BK_ELEMS, mb * 256 + rank * 128);
-          tma_load_2d_pair(sB + stage * HB, &tmB, fb, kb * BK_ELEMS, nb * BN + rank * 128);
+          tma_load_2d_pair(sA + stage * HA, &tmA, fb, kb * BK_ELEMS, mb * 256 + rank * 128);
+          tma_load_2d_pair(sB + stage * HB, &tmB, fb, kb * BK_ELEMS,
+                           nb * BN + static_cast<int>(rank) * (BN / 2));
           armed[stage] = static_cast<int>(phase);
           if (++stage == STAGES) {
             stage = 0;
@@ -678,7 +686,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * HB);
+          const uint32_t a0 = smem_u32(sA + stage * HA);
           const uint32_t b0 = smem_u32(sB + stage * HB);
 #pragma unroll
           for (int k = 0; k < K_STEPS; ++k) {
@@ -878,7 +886,7 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
 }
 
 // Largest number of CTA pairs of the pair kernel that can be resident at once.
-template <bool INT8, int EPI>
+template <int BN, bool INT8, int EPI>
 int pair_capacity(const DevCtx& ctx) {
   static std::atomic<int> cap[64];
   const int dev = ctx.device & 63;
@@ -887,9 +895,10 @@ int pair_capacity(const DevCtx& ctx) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (ctx.num_sms / 2));
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.dynamicSmemBytes = PairCfg<BN>::kSmem;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<INT8, EPI>, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<BN, INT8, EPI>, &cfg) != cudaSuccess ||
+      n <= 0) {
     cudaGetLastError();
     n = 0;
   }
@@ -899,22 +908,23 @@ int pair_capacity(const DevCtx& ctx) {
 }
 
 // Returns 1 if the pair kernel is not usable here (caller falls back to single-CTA tiles).
-template <bool INT8, int EPI>
+template <int BN, bool INT8, int EPI>
 int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, int K,
                 const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                 cudaStream_t stream, int* rc) {
-  auto kernel = k_gemm_pair<INT8, EPI>;
+  using Cfg = PairCfg<BN>;
+  auto kernel = k_gemm_pair<BN, INT8, EPI>;
   static std::atomic<uint32_t> attr_done{0};
   const uint32_t bit = 1u << (ctx.device & 31);
   if (!(attr_done.load() & bit)) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kPairSmem)) != cudaSuccess) {
+                             static_cast<int>(Cfg::kSmem)) != cudaSuccess) {
       cudaGetLastError();
       return 1;
     }
     attr_done.fetch_or(bit);
   }
-  const int cap = pair_capacity<INT8, EPI>(ctx);
+  const int cap = pair_capacity<BN, INT8, EPI>(ctx);
   if (cap <= 0) return 1;
   const CUtensorMapDataType dt =
       INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -922,7 +932,7 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int bk = kTileBytesK / esize;
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, dt, uint64_t(M), uint64_t(K), uint64_t(K) * esize, 128, bk) ||
-      !make_tmap_2d(&tb, B, dt, uint64_t(N), uint64_t(K), uint64_t(K) * esize, 128, bk)) {
+      !make_tmap_2d(&tb, B, dt, uint64_t(N), uint64_t(K), uint64_t(K) * esize, BN / 2, bk)) {
     *rc = set_error(-3, "gemm: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
     return 0;
   }
@@ -931,7 +941,7 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   p.N = N;
   p.k_blocks = K / bk;
   p.m_tiles = (M + 255) / 256;
-  p.n_tiles = N / 256;
+  p.n_tiles = N / BN;
   p.epi = epi;
   p.err = ctx.err_flag;
   const int tiles = p.m_tiles * p.n_tiles;
@@ -940,8 +950,8 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const bool use_sk = scratch != nullptr && scratch_bytes >= kSkScratchBytes &&
                       want_stream_k(tiles, cap, p.k_blocks) && iters >= 4LL * sk_pairs;
   if (trace_gemm())
-    std::fprintf(stderr, "h3b gemm pair M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n", M, N,
-                 K, tiles, cap, use_sk ? "stream-K" : "data-parallel",
+    std::fprintf(stderr, "h3b gemm pair BN=%d M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n",
+                 BN, M, N, K, tiles, cap, use_sk ? "stream-K" : "data-parallel",
                  use_sk ? sk_pairs : std::min(tiles, cap));
   if (use_sk) {
     GemmParams q = p;
@@ -952,11 +962,11 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
         reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kSkFlagsOffset);
     q.sk_seq = next_sk_seq();
     // never more pairs than can be resident at once (occupancy query above)
-    kernel<<<2 * sk_pairs, 192, kPairSmem, stream>>>(ta, tb, q);
+    kernel<<<2 * sk_pairs, 192, Cfg::kSmem, stream>>>(ta, tb, q);
     *rc = check_launch("gemm_pair");
     return 0;
   }
-  kernel<<<2 * std::min(tiles, cap), 192, kPairSmem, stream>>>(ta, tb, p);
+  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
   *rc = check_launch("gemm_pair");
   return 0;
 }
@@ -970,12 +980,42 @@ bool trace_gemm() {
   return on;
 }
 
-bool single_cta_forced() {
-  static const bool forced = [] {
-    const char* v = std::getenv("H3B_GEMM_SINGLE_CTA");
-    return v && v[0] == '1';
+// Tile configurations of the bf16 / int8 GEMM.
+enum TileCfg { kPair256 = 0, kPair128 = 1, kSingle256 = 2, kSingle128 = 3, kAuto = -1 };
+
+// H3B_GEMM_TILE=pair256|pair128|single256|single128 forces one configuration where the
+// shape allows it (diagnostics and measurements only).
+int forced_tile() {
+  static const int forced = [] {
+    const char* v = std::getenv("H3B_GEMM_TILE");
+    if (!v) return int(kAuto);
+    const std::string t(v);
+    if (t == "pair256") return int(kPair256);
+    if (t == "pair128") return int(kPair128);
+    if (t == "single256") return int(kSingle256);
+    if (t == "single128") return int(kSingle128);
+    return int(kAuto);
   }();
   return forced;
+}
+
+bool tile_allowed(int cfg, int M, int N) {
+  switch (cfg) {
+    case kPair256: return N % 256 == 0 && M >= 256;
+    case kPair128: return N % 128 == 0 && M >= 256;
+    case kSingle256: return N % 256 == 0;
+    case kSingle128: return N % 128 == 0;
+    default: return false;
+  }
+}
+
+// Shape-based choice: CTA-pair 256-wide tiles unless the problem is too small for pairs.
+int choose_tile(int M, int N) {
+  const int f = forced_tile();
+  if (f != kAuto && tile_allowed(f, M, N)) return f;
+  if (tile_allowed(kPair256, M, N)) return kPair256;
+  if (tile_allowed(kSingle256, M, N)) return kSingle256;
+  return kSingle128;
 }
 
 template <int BN>
@@ -996,37 +1036,43 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
 size_t gemm_scratch_bytes() { return kSkScratchBytes; }
 
 template <int EPI>
-bool try_pair_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
+bool try_pair_bf16(int bn, const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
                    const GemmEpilogue& epi, void* ws, size_t wsb, cudaStream_t s, int* rc) {
-  return launch_pair<false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
+  if (bn == 256) return launch_pair<256, false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
+  return launch_pair<128, false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
 }
 
 int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
                      const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream) {
   if (M <= 0) return 0;
-  if (N % 256 == 0 && M >= 256 && !single_cta_forced()) {
+  const int tile = choose_tile(M, N);
+  if (tile == kPair256 || tile == kPair128) {
+    const int bn = tile == kPair256 ? 256 : 128;
     int rc = 0;
     bool done = false;
     switch (epi.kind) {
       case kEpiBias:
-        done = try_pair_bf16<kEpiBias>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        done = try_pair_bf16<kEpiBias>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                       stream, &rc);
         break;
       case kEpiGelu:
-        done = try_pair_bf16<kEpiGelu>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        done = try_pair_bf16<kEpiGelu>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                       stream, &rc);
         break;
       case kEpiRope:
-        done = try_pair_bf16<kEpiRope>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream, &rc);
+        done = try_pair_bf16<kEpiRope>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                       stream, &rc);
         break;
       case kEpiGateResid:
-        done = try_pair_bf16<kEpiGateResid>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
-                                            stream, &rc);
+        done = try_pair_bf16<kEpiGateResid>(bn, ctx, A, B, M, N, K, epi, scratch,
+                                            scratch_bytes, stream, &rc);
         break;
       default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
     }
     if (done) return rc;
   }
-  if (N % 256 == 0)
+  if (tile == kSingle256 || (tile != kSingle128 && N % 256 == 0))
     return dispatch_bf16<256>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
   return dispatch_bf16<128>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
 }
@@ -1035,12 +1081,19 @@ int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, i
                    const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                    cudaStream_t stream) {
   if (M <= 0) return 0;
-  if (N % 256 == 0 && M >= 256 && !single_cta_forced()) {
+  const int tile = choose_tile(M, N);
+  if (tile == kPair256 || tile == kPair128) {
     int rc = 0;
-    if (launch_pair<true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream,
-                                       &rc) == 0)
-      return rc;
+    const int r = tile == kPair256
+                      ? launch_pair<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch,
+                                                            scratch_bytes, stream, &rc)
+                      : launch_pair<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch,
+                                                            scratch_bytes, stream, &rc);
+    if (r == 0) return rc;
   }
+  if (tile == kSingle128 || N % 256 != 0)
+    return launch_impl<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                               stream);
   if (N % 256 == 0)
     return launch_impl<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
                                                stream);
