@@ -279,9 +279,13 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
 
 /* Joint self-attention over one packed QKV buffer: qkv [n_tokens, 3 n_heads head_dim]
  * bf16 (q, then k, then v; head j at column j*head_dim of each), out [n_tokens,
- * n_heads head_dim] bf16 (device).  out = softmax(q k^T / sqrt(head_dim)) v per head. */
+ * n_heads head_dim] bf16 (device).  out = softmax(q k^T / sqrt(head_dim)) v per head.
+ * ws: NULL, or 16-byte aligned device scratch of h3b_gemm_workspace_size() bytes (the
+ * same scratch the GEMM calls take; one kernel at a time per buffer).  With it the work
+ * is split evenly over the SMs (a query tile may be finished by two CTAs, merged through
+ * the scratch); without it, one CTA per (head, 128-query tile).  A smaller ws is ignored. */
 int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim,
-                  h3b_bf16* out, void* stream);
+                  h3b_bf16* out, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- host policy */
 /* Layer thinning mask (dothoosh.com "Aggressive optimisation levers": rank blocks by

@@ -67,8 +67,10 @@ def test_validation_rejects_before_any_launch():
     rc, _ = _err(L.h3b_gemm_bf16, ctypes.c_void_p(4097), p, 64, 256, 64, 0, p, None, None, 0,
                  128, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL                                  # misaligned A
-    rc, _ = _err(L.h3b_attention, p, 10, 2, 96, p, None)
+    rc, _ = _err(L.h3b_attention, p, 10, 2, 96, p, None, 0, None)
     assert rc == h3b.H3B_EINVAL                                  # head_dim 96
+    rc, _ = _err(L.h3b_attention, p, 10, 2, 128, p, ctypes.c_void_p(4100), 1 << 30, None)
+    assert rc == h3b.H3B_EINVAL                                  # misaligned scratch
     rc, _ = _err(L.h3b_token_reduce, 0, p, p, None, 2, 2, 3, 0, 64, None)
     assert rc == h3b.H3B_EINVAL                                  # odd w
     rc, _ = _err(L.h3b_token_reduce, 7, p, p, None, 2, 2, 4, 0, 64, None)

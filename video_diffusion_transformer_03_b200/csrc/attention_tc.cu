@@ -1,27 +1,43 @@
 // Joint video+audio self-attention, flash style, on tcgen05.
 //
-// One CTA per (128-query tile, head); full non-causal attention over all tokens of the
-// joint stream.  The q and k columns of the packed QKV buffer are already rotated by
-// 3D RoPE in the QKV projection's epilogue, so tiles are consumed as loaded.
+// Full non-causal attention over all tokens of the joint stream, per head.  The q and k
+// columns of the packed QKV buffer are already rotated by 3D RoPE in the QKV projection's
+// epilogue, so tiles are consumed as loaded.
+//
+// Work: a unit is one (head, 128-query tile) pair and has n_kv steps, one per 128-key
+// tile.  The units' steps, laid end to end (u * n_kv + j), are cut into one equal
+// contiguous range per CTA.  With a scratch buffer the grid is persistent (one CTA per
+// SM), so every SM gets the same number of steps whatever the unit count; a unit cut
+// between two CTAs is finished by the CTA holding its last key tile (the owner), which
+// merges the running state (unnormalised O, row max, row sum) that the lower CTA left in
+// the scratch.  Each CTA walks its units from last to first, so its contribution to a
+// split unit is computed first and the owner's merge, done last, does not wait in
+// practice.  Without scratch the grid has one CTA per unit (nothing is split).
 //
 // Roles (192 threads):
-//   warp 0      TMA producer: Q tile once, then K_j and V_j tiles into 2-stage rings
-//               (K stages are released as soon as S_j = Q K_j^T completes, V stages after
-//               O += P_j V_j);
-//   warp 1      MMA issuer: S_j into one of two TMEM score buffers (128 fp32 columns each),
-//               then O += P_{j-1} V_{j-1} (P from shared memory, V as an MN-major operand)
-//               into a TMEM output accumulator;
+//   warp 0      TMA producer: the Q tile of each unit (once the previous unit's last S
+//               has read the buffer), then K_j and V_j tiles into 2-stage rings (K stages are released as soon as S_j = Q K_j^T completes,
+//               V stages after O += P_j V_j);
+//   warp 1      MMA issuer: S_j into one of two TMEM score buffers (128 fp32 columns
+//               each), then O += P_{j-1} V_{j-1} (P from shared memory, V as an MN-major
+//               operand) into a TMEM output accumulator.  At the first step of a unit the
+//               previous unit's last P V goes first, so its end does not wait for the
+//               new unit's first S;
 //   warps 2..5  softmax: thread = query row; the whole 128-wide score row is in registers,
 //               so row max and row sum need no shuffles.  Exponentials are base 2 with
-//               the 1/sqrt(head_dim) scale folded in.  Rescaling of O is lazy: the
+//               the 1/sqrt(head_dim) scale folded in, all on the MUFU unit (the score
+//               row's load-exp-pack chain is latency bound, so moving a share of the
+//               exponentials to FMA-pipe polynomials only adds instructions).  Rescaling of O is lazy: the
 //               running max used for the exponentials only moves when the tile max
 //               exceeds it by more than 8 (a factor 256), and then O (in TMEM) and the
-//               row sum are multiplied by 2^(m_old - m_new).
+//               row sum are multiplied by 2^(m_old - m_new).  At the end of a unit the
+//               same warps normalise and store O, or park / merge a split unit's state.
 // TMEM map: S0 [0,128), S1 [128,256), O [256, 256 + head_dim).
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -31,41 +47,37 @@ namespace {
 
 constexpr uint32_t kBox = 128 * 128;  // [128 rows x 128 B] swizzled box
 
+// Shared memory: Q, K x 2, V x 2, P x 2 (the softmax writes P_j while P_{j-1} V_{j-1}
+// may still be running).
 template <int HD>
 struct AttnCfg {
   static constexpr int kNBox = HD / 64;
   static constexpr uint32_t kQBytes = kNBox * kBox;
   static constexpr uint32_t kKVBytes = kNBox * kBox;
   static constexpr uint32_t kPBytes = 2 * kBox;
-  static constexpr size_t kSmem = 1024 + kQBytes + 4 * size_t(kKVBytes) + 2 * kPBytes + 256;
+  static constexpr size_t kSmem =
+      1024 + size_t(kQBytes) + 4 * size_t(kKVBytes) + 2 * size_t(kPBytes) + 256;
 };
 
 struct AttnParams {
-  int n;            // tokens
-  int d;            // n_heads * head_dim
-  int n_kv;         // ceil(n / 128)
-  float scale_log2; // log2(e) / sqrt(head_dim)
-  bf16* out;        // [n, d]
+  int n;             // tokens
+  int d;             // n_heads * head_dim
+  int n_kv;          // ceil(n / 128): key tiles, and steps per unit
+  int n_qt;          // ceil(n / 128): query tiles per head
+  long long steps;   // units * n_kv
+  float scale_log2;  // log2(e) / sqrt(head_dim)
+  bf16* out;         // [n, d]
+  float4* part_o;    // [gridDim.x][head_dim / 4][128] unnormalised O of a split unit
+  float2* part_ml;   // [gridDim.x][128] (running max, row sum) of a split unit
+  unsigned long long* flags;  // [gridDim.x][4]
+  unsigned long long seq;
   uint32_t* err;
 };
 
-// 2^x on the FMA pipe, for a share of the probabilities so that the MUFU unit (16 ex2 per
-// clock per SM, the same time per 128 x 128 tile as the tile's MMAs) is not the limit.
-// Range reduction to n = round(x) by adding the 1.5 * 2^23 shifter, f = x - n in
-// [-1/2, 1/2], 2^f by a degree-3 polynomial fitted here by iteratively reweighted least
-// squares on the relative error (max 7.5e-5 over x in [-125, 8]), then 2^n added to the
-// exponent field.  x is clamped at -125 so the exponent add cannot underflow.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float shifter = 12582912.0f;
-  const float t = x + shifter;
-  const int n = __float_as_int(t) - __float_as_int(shifter);
-  const float f = x - (t - shifter);
-  float p = 0.05517259240150452f;
-  p = fmaf(p, f, 0.24261370301246643f);
-  p = fmaf(p, f, 0.6932610273361206f);
-  p = fmaf(p, f, 0.9999278783798218f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -73,6 +85,51 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > kWaitLimitNs) return;
   }
+}
+
+// This CTA's step range [begin, end) and the units it touches.
+struct Range {
+  long long begin, end;
+  int u_first, u_last;
+};
+
+__device__ __forceinline__ long long range_begin(const AttnParams& p, int c) {
+  return p.steps * c / static_cast<long long>(gridDim.x);
+}
+
+__device__ __forceinline__ Range cta_range(const AttnParams& p) {
+  Range r;
+  r.begin = range_begin(p, static_cast<int>(blockIdx.x));
+  r.end = range_begin(p, static_cast<int>(blockIdx.x) + 1);
+  r.u_first = static_cast<int>(r.begin / p.n_kv);
+  r.u_last = static_cast<int>((r.end - 1) / p.n_kv);
+  return r;
+}
+
+// Segment k of the walk (units from the last to the first): unit u_last - k, key tiles
+// [j0, j1).  j1 < n_kv: the lower part of a split unit; j0 > 0: the upper part.  A range
+// is at least n_kv steps long, so no segment is both.
+__device__ __forceinline__ void segment(const AttnParams& p, const Range& r, int k, int& unit,
+                                        int& j0, int& j1) {
+  unit = r.u_last - k;
+  const long long base = static_cast<long long>(unit) * p.n_kv;
+  j0 = static_cast<int>(r.begin > base ? r.begin - base : 0ll);
+  j1 = static_cast<int>(r.end - base < p.n_kv ? r.end - base : static_cast<long long>(p.n_kv));
+}
+
+// Wait until the flag holds `seq`; false on abort or time-out (records kErrAttnWait).
+__device__ __forceinline__ bool wait_flag(const unsigned long long* f, unsigned long long seq,
+                                          volatile uint32_t* abort_flag, uint32_t* err) {
+  if (ld_acquire_u64(f) == seq) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_u64(f) != seq) {
+    if (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1u;
+      atomicCAS(err, 0u, kErrAttnWait);
+      return false;
+    }
+  }
+  return true;
 }
 
 template <int HD>
@@ -93,26 +150,26 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sP = sV + 2 * Cfg::kKVBytes;     // 2 buffers
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * Cfg::kPBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 3;
-  uint64_t* v_full = bars + 5;
-  uint64_t* v_empty = bars + 7;
-  uint64_t* s_full = bars + 9;
-  uint64_t* s_free = bars + 11;
-  uint64_t* p_full = bars + 13;
-  uint64_t* p_free = bars + 15;
-  uint64_t* drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;   // [2]
+  uint64_t* k_empty = bars + 4;  // [2]
+  uint64_t* v_full = bars + 6;   // [2]
+  uint64_t* v_empty = bars + 8;  // [2]
+  uint64_t* s_full = bars + 10;  // [2]
+  uint64_t* s_free = bars + 12;  // [2]
+  uint64_t* p_full = bars + 14;  // [2]
+  uint64_t* p_free = bars + 16;  // [2]
+  uint64_t* o_empty = bars + 18;
+  uint64_t* drain = bars + 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x;
-  const int head = blockIdx.y;
-  const int n_kv = p.n_kv;
+  const Range rg = cta_range(p);
+  const int n_seg = rg.u_last - rg.u_first + 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -123,6 +180,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&p_full[s], 4);
       mbar_init(&p_free[s], 1);
     }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(o_empty, 4);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -140,39 +200,52 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------------ producer
-      const int xq = head * HD, xk = p.d + head * HD, xv = 2 * p.d + head * HD;
-      int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1};
-      mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
-#pragma unroll
-      for (int b = 0; b < Cfg::kNBox; ++b)
-        tma_load_2d(sQ + b * kBox, &tm, q_full, xq + 64 * b, qt * 128);
+      int k_armed[2] = {-1, -1}, v_armed[2] = {-1, -1}, q_armed = -1;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
-        if (!wait_bar(&k_empty[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait)) {
+      int t = 0;  // step counter of this CTA (ring position)
+      for (int k = 0; k < n_seg && ok; ++k) {
+        int unit, j0, j1;
+        segment(p, rg, k, unit, j0, j1);
+        const int head = unit / p.n_qt, qt = unit % p.n_qt;
+        const int xq = head * HD, xk = p.d + head * HD, xv = 2 * p.d + head * HD;
+        if (k > 0 && !wait_bar(q_empty, static_cast<uint32_t>(k - 1) & 1u, abort_flag, p.err,
+                               kErrAttnWait)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+        mbar_arrive_expect_tx(q_full, Cfg::kQBytes);
 #pragma unroll
         for (int b = 0; b < Cfg::kNBox; ++b)
-          tma_load_2d(sK + st * Cfg::kKVBytes + b * kBox, &tm, &k_full[st], xk + 64 * b,
-                      j * 128);
-        k_armed[st] = static_cast<int>(ph);
-        if (!wait_bar(&v_empty[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait)) {
-          ok = false;
-          break;
+          tma_load_2d(sQ + b * kBox, &tm, q_full, xq + 64 * b, qt * 128);
+        q_armed = k & 1;
+        for (int j = j0; j < j1; ++j, ++t) {
+          const int st = t & 1;
+          const uint32_t ph = static_cast<uint32_t>(t >> 1) & 1u;
+          if (!wait_bar(&k_empty[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[st], Cfg::kKVBytes);
+#pragma unroll
+          for (int b = 0; b < Cfg::kNBox; ++b)
+            tma_load_2d(sK + st * Cfg::kKVBytes + b * kBox, &tm, &k_full[st], xk + 64 * b,
+                        j * 128);
+          k_armed[st] = static_cast<int>(ph);
+          if (!wait_bar(&v_empty[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
+#pragma unroll
+          for (int b = 0; b < Cfg::kNBox; ++b)
+            tma_load_2d(sV + st * Cfg::kKVBytes + b * kBox, &tm, &v_full[st], xv + 64 * b,
+                        j * 128);
+          v_armed[st] = static_cast<int>(ph);
         }
-        mbar_arrive_expect_tx(&v_full[st], Cfg::kKVBytes);
-#pragma unroll
-        for (int b = 0; b < Cfg::kNBox; ++b)
-          tma_load_2d(sV + st * Cfg::kKVBytes + b * kBox, &tm, &v_full[st], xv + 64 * b,
-                      j * 128);
-        v_armed[st] = static_cast<int>(ph);
       }
       if (!ok) {
-        drain_wait(q_full, 0);
+        // let the copies in flight land before the CTA's shared memory is released
+        if (q_armed >= 0) drain_wait(q_full, static_cast<uint32_t>(q_armed));
         for (int s = 0; s < 2; ++s) {
           if (k_armed[s] >= 0) drain_wait(&k_full[s], static_cast<uint32_t>(k_armed[s]));
           if (v_armed[s] >= 0) drain_wait(&v_full[s], static_cast<uint32_t>(v_armed[s]));
@@ -182,45 +255,79 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
-      bool ok = wait_bar(q_full, 0, abort_flag, p.err, kErrAttnWait);
-      const uint32_t q0 = smem_u32(sQ);
-      for (int j = 0; j <= n_kv && ok; ++j) {
-        if (j < n_kv) {
-          const int st = j & 1;
-          const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
-          if (!wait_bar(&k_full[st], ph, abort_flag, p.err, kErrAttnWait)) break;
-          if (j >= 2 && !wait_bar(&s_free[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait))
-            break;
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(sK + st * Cfg::kKVBytes);
+      // Two cursors over the same walk: the S side (step t) runs one step ahead of the
+      // P V side (step t - 1).
+      int ks = 0, js = 0, js0 = 0, js1 = 0, unit_s = 0;  // S cursor: segment, key tile
+      int kp = 0, jp = 0, jp0 = 0, jp1 = 0, unit_p = 0;  // P V cursor
+      segment(p, rg, 0, unit_s, js0, js1);
+      js = js0;
+      segment(p, rg, 0, unit_p, jp0, jp1);
+      jp = jp0;
+      auto issue_s = [&](long long t) -> bool {
+        const int st = static_cast<int>(t & 1);
+        const uint32_t ph = static_cast<uint32_t>(t >> 1) & 1u;
+        if (js == js0 &&
+            !wait_bar(q_full, static_cast<uint32_t>(ks) & 1u, abort_flag, p.err, kErrAttnWait))
+          return false;
+        if (!wait_bar(&k_full[st], ph, abort_flag, p.err, kErrAttnWait)) return false;
+        if (t >= 2 && !wait_bar(&s_free[st], ph ^ 1u, abort_flag, p.err, kErrAttnWait))
+          return false;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ);
+        const uint32_t k0 = smem_u32(sK + st * Cfg::kKVBytes);
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_f16(tmem + st * 128, sdesc_sw128(q0 + off, 16, 1024),
-                     sdesc_sw128(k0 + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&s_full[st]);
-          tc_commit(&k_empty[st]);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+          umma_f16(tmem + st * 128, sdesc_sw128(q0 + off, 16, 1024),
+                   sdesc_sw128(k0 + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int i = j - 1;
-          const int pb = i & 1;
-          const uint32_t ph = static_cast<uint32_t>(i >> 1) & 1u;
-          if (!wait_bar(&p_full[pb], ph, abort_flag, p.err, kErrAttnWait)) break;
-          if (!wait_bar(&v_full[pb], ph, abort_flag, p.err, kErrAttnWait)) break;
-          tc_fence_after();
-          const uint32_t p0 = smem_u32(sP + pb * Cfg::kPBytes);
-          const uint32_t v0 = smem_u32(sV + pb * Cfg::kKVBytes);
+        tc_commit(&s_full[st]);
+        tc_commit(&k_empty[st]);
+        if (++js == js1) {  // last S of this unit: the Q buffer may be refilled
+          tc_commit(q_empty);
+          if (++ks < n_seg) {
+            segment(p, rg, ks, unit_s, js0, js1);
+            js = js0;
+          }
+        }
+        return true;
+      };
+      auto issue_pv = [&](long long i) -> bool {
+        const int vb = static_cast<int>(i & 1);
+        const uint32_t ph = static_cast<uint32_t>(i >> 1) & 1u;
+        const bool first = jp == jp0;
+        // the previous unit's O must have been read out before it is overwritten
+        if (first && kp > 0 &&
+            !wait_bar(o_empty, static_cast<uint32_t>(kp - 1) & 1u, abort_flag, p.err,
+                      kErrAttnWait))
+          return false;
+        if (!wait_bar(&p_full[vb], ph, abort_flag, p.err, kErrAttnWait)) return false;
+        if (!wait_bar(&v_full[vb], ph, abort_flag, p.err, kErrAttnWait)) return false;
+        tc_fence_after();
+        const uint32_t p0 = smem_u32(sP + vb * Cfg::kPBytes);
+        const uint32_t v0 = smem_u32(sV + vb * Cfg::kKVBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t poff = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_f16(tmem + kOCol, sdesc_sw128(p0 + poff, 16, 1024),
-                     sdesc_sw128(v0 + kk * 2048, kBox, 1024), IDESC_PV,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&p_free[pb]);
-          tc_commit(&v_empty[pb]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t poff = (kk >> 2) * kBox + (kk & 3) * 32;
+          umma_f16(tmem + kOCol, sdesc_sw128(p0 + poff, 16, 1024),
+                   sdesc_sw128(v0 + kk * 2048, kBox, 1024), IDESC_PV,
+                   (!first || kk > 0) ? 1u : 0u);
         }
+        tc_commit(&p_free[vb]);
+        tc_commit(&v_empty[vb]);
+        if (++jp == jp1 && ++kp < n_seg) {
+          segment(p, rg, kp, unit_p, jp0, jp1);
+          jp = jp0;
+        }
+        return true;
+      };
+      const long long total = rg.end - rg.begin;
+      for (long long t = 0; t <= total; ++t) {
+        // at a unit's first step (not the walk's first), finish the previous unit first
+        const bool pv_first = t >= 1 && t < total && js == js0;
+        if (pv_first && !issue_pv(t - 1)) break;
+        if (t < total && !issue_s(t)) break;
+        if (t >= 1 && !pv_first && !issue_pv(t - 1)) break;
       }
       tc_commit(drain);
       drain_wait(drain, 0);
@@ -231,139 +338,203 @@ __global__ void __launch_bounds__(192, 1)
     const int row = quarter * 32 + lane;  // query row within the tile
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY;
-    float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
-      ok = __all_sync(0xffffffffu, wait_bar(&s_full[sb], ph, abort_flag, p.err, kErrAttnWait));
-      if (!ok) break;
-      tc_fence_after();
-      float s[128];
+    int t = 0;
+    for (int k = 0; k < n_seg && ok; ++k) {
+      int unit, j0, j1;
+      segment(p, rg, k, unit, j0, j1);
+      float m_used = -INFINITY;
+      float l = 0.f;
+      for (int j = j0; j < j1; ++j, ++t) {
+        const int sb = t & 1;
+        const uint32_t ph = static_cast<uint32_t>(t >> 1) & 1u;
+        ok = __all_sync(0xffffffffu, wait_bar(&s_full[sb], ph, abort_flag, p.err, kErrAttnWait));
+        if (!ok) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t r[128];
+          tmem_ld128_sync(tmem + lane_addr + sb * 128, r);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + sb * 128 + c * 32, r);
-        tmem_wait_ld(r);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) s[c * 32 + t] = __uint_as_float(r[t]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-
-      if ((j + 1) * 128 > p.n) {
-        const int valid = p.n - j * 128;
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-#pragma unroll
-      for (int i = 4; i > 0; i >>= 1)
-#pragma unroll
-        for (int k = 0; k < i; ++k) m8[k] = fmaxf(m8[k], m8[k + i]);
-      const float mxs = m8[0] * sl2;
-      if (j == 0) {
-        m_used = mxs;
-      } else {
-        const bool need = mxs > m_used + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          // O must hold every earlier P V product before it is rescaled
-          const int i = j - 1;
-          ok = __all_sync(0xffffffffu,
-                          wait_bar(&p_free[i & 1], static_cast<uint32_t>(i >> 1) & 1u,
-                                   abort_flag, p.err, kErrAttnWait));
-          if (!ok) break;
-          tc_fence_after();
-          const float alpha = need ? ex2_approx(m_used - mxs) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t addr = tmem + lane_addr + kOCol + c * 32;
-            tmem_ld32(addr, r);
-            tmem_wait_ld(r);
-#pragma unroll
-            for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) * alpha);
-            tmem_st32(addr, r);
-          }
-          tmem_wait_st();
-          l *= alpha;
-          if (need) m_used = mxs;
+          for (int q = 0; q < 128; ++q) s[q] = __uint_as_float(r[q]);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+
+        if ((j + 1) * 128 > p.n) {
+          const int valid = p.n - j * 128;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        // row max: eight independent chains of three-input maxima
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          m8[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+          for (int c = 16; c < 128; c += 16) m8[i] = max3(m8[i], s[c + i], s[c + 8 + i]);
+        }
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
+                              fmaxf(m8[6], m8[7]));
+        const float mxs = mx * sl2;
+        if (j == j0) {
+          m_used = mxs;
+        } else {
+          const bool need = mxs > m_used + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            // O must hold every earlier P V product of this unit before it is rescaled
+            const int i = t - 1;
+            ok = __all_sync(0xffffffffu,
+                            wait_bar(&p_free[i & 1], static_cast<uint32_t>(i >> 1) & 1u,
+                                     abort_flag, p.err, kErrAttnWait));
+            if (!ok) break;
+            tc_fence_after();
+            const float alpha = need ? ex2_approx(m_used - mxs) : 1.0f;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+              uint32_t r[32];
+              const uint32_t addr = tmem + lane_addr + kOCol + c * 32;
+              tmem_ld32(addr, r);
+              tmem_wait_ld(r);
+#pragma unroll
+              for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+              tmem_st32(addr, r);
+            }
+            tmem_wait_st();
+            l *= alpha;
+            if (need) m_used = mxs;
+          }
+        }
+        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float x = fmaf(s[c], sl2, -m_used);
+          const float e = ex2_approx(x);
+          sum8[c & 7] += e;
+          s[c] = e;
+        }
+#pragma unroll
+        for (int i = 4; i > 0; i >>= 1)
+#pragma unroll
+          for (int q = 0; q < i; ++q) sum8[q] += sum8[q + i];
+        l += sum8[0];
+        if (t >= 2) {  // P buffer sb is free once P_{t-2} V_{t-2} has completed
+          ok = __all_sync(0xffffffffu,
+                          wait_bar(&p_free[sb], ph ^ 1u, abort_flag, p.err, kErrAttnWait));
+          if (!ok) break;
+        }
+        uint8_t* pbuf = sP + sb * Cfg::kPBytes + row * 128;
+#pragma unroll
+        for (int c16 = 0; c16 < 16; ++c16) {
+          uint4 u;
+          u.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
+          u.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
+          u.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
+          u.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
+          const int chunk = (c16 & 7) ^ (row & 7);
+          *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kBox + chunk * 16) = u;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float x = fmaf(s[c], sl2, -m_used);
-        const float e = (c & 3) == 3 ? exp2_fma(x) : ex2_approx(x);
-        sum8[c & 7] += e;
-        s[c] = e;
-      }
-#pragma unroll
-      for (int i = 4; i > 0; i >>= 1)
-#pragma unroll
-        for (int k = 0; k < i; ++k) sum8[k] += sum8[k + i];
-      l += sum8[0];
-      if (j >= 2) {
+      if (!ok) break;
+      // ---- end of the unit: O holds every P V product once the last one completes
+      {
+        const int last = t - 1;
         ok = __all_sync(0xffffffffu,
-                        wait_bar(&p_free[sb], ph ^ 1u, abort_flag, p.err, kErrAttnWait));
+                        wait_bar(&p_free[last & 1], static_cast<uint32_t>(last >> 1) & 1u,
+                                 abort_flag, p.err, kErrAttnWait));
         if (!ok) break;
       }
-      uint8_t* pbuf = sP + sb * Cfg::kPBytes + row * 128;
-#pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        uint4 u;
-        u.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
-        u.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
-        u.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
-        u.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
-        const int chunk = (c16 & 7) ^ (row & 7);
-        *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kBox + chunk * 16) = u;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-    }
-    if (ok) {
-      const int last = n_kv - 1;
-      ok = __all_sync(0xffffffffu,
-                      wait_bar(&p_free[last & 1], static_cast<uint32_t>(last >> 1) & 1u,
-                               abort_flag, p.err, kErrAttnWait));
-    }
-    if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
-      const int grow = qt * 128 + row;
+      const int head = unit / p.n_qt, qt = unit % p.n_qt;
+      const uint32_t o_addr = tmem + lane_addr + kOCol;
+      if (j1 < p.n_kv) {
+        // lower part of a split unit: park the running state for the owner (next CTA)
+        float4* po = p.part_o + size_t(blockIdx.x) * (HD / 4) * 128 + row;
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c * 32, r);
+          tmem_wait_ld(r);
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kOCol + c * 32, r);
-        tmem_wait_ld(r);
-        if (grow < p.n) {
-          uint4* dst =
-              reinterpret_cast<uint4*>(p.out + size_t(grow) * p.d + head * HD + c * 32);
+          for (int i = 0; i < 8; ++i)
+            __stcg(po + size_t(c * 8 + i) * 128,
+                   make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
+        }
+        __stcg(p.part_ml + size_t(blockIdx.x) * 128 + row, make_float2(m_used, l));
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_u64(p.flags + blockIdx.x * 4 + quarter, p.seq);
+      } else {
+        // whole unit, or upper part of a split unit: merge the lower CTA's state, then
+        // normalise and store
+        float wa = 0.f, wb = 1.f;
+        const float4* po = nullptr;
+        if (j0 > 0) {
+          const int src = static_cast<int>(blockIdx.x) - 1;
+          ok = __all_sync(0xffffffffu, wait_flag(p.flags + src * 4 + quarter, p.seq,
+                                                 abort_flag, p.err));
+          if (!ok) break;
+          const float2 ml = __ldcg(p.part_ml + size_t(src) * 128 + row);
+          const float m = fmaxf(ml.x, m_used);
+          wa = ex2_approx(ml.x - m);
+          wb = ex2_approx(m_used - m);
+          l = ml.y * wa + l * wb;
+          po = p.part_o + size_t(src) * (HD / 4) * 128 + row;
+        }
+        const float inv_l = 1.0f / l;
+        wa *= inv_l;
+        wb *= inv_l;
+        const int grow = qt * 128 + row;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l,
-                              __uint_as_float(r[8 * i + 1]) * inv_l);
-            u.y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l,
-                              __uint_as_float(r[8 * i + 3]) * inv_l);
-            u.z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l,
-                              __uint_as_float(r[8 * i + 5]) * inv_l);
-            u.w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l,
-                              __uint_as_float(r[8 * i + 7]) * inv_l);
-            dst[i] = u;
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + c * 32, r);
+          tmem_wait_ld(r);
+          float o[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(r[q]) * wb;
+          if (po != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 a = __ldcg(po + size_t(c * 8 + i) * 128);
+              o[4 * i + 0] = fmaf(a.x, wa, o[4 * i + 0]);
+              o[4 * i + 1] = fmaf(a.y, wa, o[4 * i + 1]);
+              o[4 * i + 2] = fmaf(a.z, wa, o[4 * i + 2]);
+              o[4 * i + 3] = fmaf(a.w, wa, o[4 * i + 3]);
+            }
+          }
+          if (grow < p.n) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(p.out + size_t(grow) * p.d + head * HD + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16x2(o[8 * i + 0], o[8 * i + 1]);
+              u.y = pack_bf16x2(o[8 * i + 2], o[8 * i + 3]);
+              u.z = pack_bf16x2(o[8 * i + 4], o[8 * i + 5]);
+              u.w = pack_bf16x2(o[8 * i + 6], o[8 * i + 7]);
+              dst[i] = u;
+            }
           }
         }
+        if (po != nullptr) {
+          // hand the flag back at zero, so a replay of this launch (same sequence value,
+          // e.g. from a CUDA graph) waits for the lower CTA again
+          __syncwarp();
+          if (lane == 0) p.flags[(blockIdx.x - 1) * 4 + quarter] = 0ull;
+        }
       }
+      // O may now be overwritten by the next unit's first P V
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
     }
   }
 
@@ -377,8 +548,8 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int HD>
-int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out,
-              cudaStream_t stream) {
+int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, void* scratch,
+              size_t scratch_bytes, cudaStream_t stream) {
   using Cfg = AttnCfg<HD>;
   const int d = heads * HD;
   CUtensorMap tm;
@@ -395,25 +566,45 @@ int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out,
       return set_error(-3, "attention: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     attr_done.fetch_or(bit);
   }
-  AttnParams p;
+  AttnParams p = {};
   p.n = n;
   p.d = d;
   p.n_kv = (n + 127) / 128;
+  p.n_qt = p.n_kv;
+  const long long units = static_cast<long long>(p.n_qt) * heads;
+  p.steps = units * p.n_kv;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(HD)));
   p.out = out;
   p.err = ctx.err_flag;
-  dim3 grid((n + 127) / 128, heads);
-  kernel<<<grid, 192, Cfg::kSmem, stream>>>(tm, p);
+  // Split schedule: one CTA per SM, never more CTAs than units, so a range is at least
+  // n_kv steps long: a unit is cut at most once and each CTA parks at most one partial
+  // state.  Without scratch: one CTA per unit.
+  long long grid = units;
+  if (scratch != nullptr && scratch_bytes >= kScratchBytes) {
+    static_assert(size_t(kMaxSkCtas) * 128 * (128 + 2) * 4 <= kSkFlagsOffset,
+                  "attention partial states must fit the slot area");
+    grid = std::min<long long>(units, std::min(ctx.num_sms, kMaxSkCtas));
+    uint8_t* base = static_cast<uint8_t*>(scratch);
+    p.part_o = reinterpret_cast<float4*>(base);
+    p.part_ml = reinterpret_cast<float2*>(base + size_t(kMaxSkCtas) * 128 * HD * 4);
+    p.flags = reinterpret_cast<unsigned long long*>(base + kAttnFlagsOffset);
+    p.seq = next_scratch_seq();
+  }
+  if (grid > 0x7fffffffll) return set_error(-1, "attention: %lld units", units);
+  kernel<<<static_cast<unsigned>(grid), 192, Cfg::kSmem, stream>>>(tm, p);
   return check_launch("attention");
 }
 
 }  // namespace
 
 int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_heads,
-                     int head_dim, bf16* out, cudaStream_t stream) {
+                     int head_dim, bf16* out, void* scratch, size_t scratch_bytes,
+                     cudaStream_t stream) {
   if (n_tokens <= 0) return 0;
-  if (head_dim == 128) return launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, stream);
-  if (head_dim == 64) return launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, stream);
+  if (head_dim == 128)
+    return launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+  if (head_dim == 64)
+    return launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
   return set_error(-1, "attention: head_dim %d unsupported (64 or 128)", head_dim);
 }
 

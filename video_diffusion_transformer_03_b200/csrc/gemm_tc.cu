@@ -61,14 +61,12 @@ struct GemmParams {
   uint32_t* err;
 };
 
-constexpr int kMaxSkCtas = 160;  // stream-K grid cap (slots in the scratch)
-
-// Stream-K scratch: slots sized for the widest tile, then the flags (same offsets for
-// every tile width, so launches of different widths may share one scratch buffer).
-// One flag per (CTA, epilogue warp): a warp publishes the 32 slot rows it wrote, and the
-// owner's warp with the same TMEM lane quarter reads exactly those rows.
-constexpr size_t kSkFlagsOffset = size_t(kMaxSkCtas) * kBM * 256 * 4;
-constexpr size_t kSkScratchBytes = kSkFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
+// Stream-K slots are sized for the widest tile (same offsets for every tile width, so
+// launches of different widths may share one scratch buffer).  One flag per (CTA,
+// epilogue warp): a warp publishes the 32 slot rows it wrote, and the owner's warp with
+// the same TMEM lane quarter reads exactly those rows.
+static_assert(kSkFlagsOffset >= size_t(kMaxSkCtas) * kBM * 256 * 4,
+              "stream-K slots must hold the widest tile");
 
 // Scheduling units are CTAs (single-SM kernel) or CTA pairs (pair kernel): `me` is this
 // unit's index and `count` the number of units in the grid.
@@ -119,15 +117,6 @@ __device__ __forceinline__ bool sched_next(const GemmParams& p, Sched& s, int& t
   kb1 = p.k_blocks;
   s.tile += s.count;
   return true;
-}
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
@@ -863,7 +852,7 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_ctas = std::min(ctx.num_sms, kMaxSkCtas);
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
-  const bool use_sk = scratch != nullptr && scratch_bytes >= kSkScratchBytes &&
+  const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
                       want_stream_k(tiles, ctx.num_sms, p.k_blocks) && iters >= 4LL * sk_ctas;
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm 1cta BN=%d M=%d N=%d K=%d tiles=%d sms=%d -> %s grid=%d\n", BN,
@@ -947,7 +936,7 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
-  const bool use_sk = scratch != nullptr && scratch_bytes >= kSkScratchBytes &&
+  const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
                       want_stream_k(tiles, cap, p.k_blocks) && iters >= 4LL * sk_pairs;
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm pair BN=%d M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n",
@@ -1033,7 +1022,9 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
 
 }  // namespace
 
-size_t gemm_scratch_bytes() { return kSkScratchBytes; }
+size_t gemm_scratch_bytes() { return kScratchBytes; }
+
+unsigned long long next_scratch_seq() { return next_sk_seq(); }
 
 template <int EPI>
 bool try_pair_bf16(int bn, const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,

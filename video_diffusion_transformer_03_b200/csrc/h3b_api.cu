@@ -178,7 +178,9 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   e.ld_out = 3 * D;
   if ((rc = launch_gemm_bf16(ctx, h, reinterpret_cast<const bf16*>(w->w_qkv), n, 3 * D, D, e, b.gemm_scratch, gemm_scratch_bytes(), s)))
     return rc;
-  if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, s))) return rc;
+  if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, b.gemm_scratch,
+                             gemm_scratch_bytes(), s)))
+    return rc;
 
   e = GemmEpilogue();
   e.kind = kEpiGateResid;
@@ -613,15 +615,16 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
 }
 
 int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim, h3b_bf16* out,
-                  void* stream) {
+                  void* ws, size_t ws_bytes, void* stream) {
   if (n_tokens < 0 || n_heads <= 0 || (head_dim != 64 && head_dim != 128))
     return set_error(H3B_EINVAL, "attention: bad sizes (n=%d heads=%d hd=%d)", n_tokens, n_heads, head_dim);
-  if (!qkv || !out || !al16(qkv) || !al16(out))
+  if (!qkv || !out || !al16(qkv) || !al16(out) || (ws && !al16(ws)))
     return set_error(H3B_EINVAL, "attention: NULL or misaligned pointer");
   DevCtx ctx;
   if (int rc = get_ctx(&ctx)) return rc;
   return launch_attention(ctx, reinterpret_cast<const bf16*>(qkv), n_tokens, n_heads, head_dim,
-                          reinterpret_cast<bf16*>(out), static_cast<cudaStream_t>(stream));
+                          reinterpret_cast<bf16*>(out), ws, ws_bytes,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int h3b_layer_mask(const float* mods_host, int n_blocks, int d, int n_active,

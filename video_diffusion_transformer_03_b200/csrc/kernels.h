@@ -48,8 +48,24 @@ struct GemmEpilogue {
   int32_t* acc_out = nullptr;        // int8 path, [M, N] or null
 };
 
-// Bytes of stream-K scratch the GEMM can use (partial-tile slots + flags).
+// Kernel scratch: one caller buffer per stream, used by one kernel at a time.  Layout:
+//   [0, kSkFlagsOffset)                 partial tiles: the GEMM's stream-K slots
+//                                       ([CTA][128][256] words), or the attention's split
+//                                       query tiles ([CTA][head_dim/4][128] float4, then
+//                                       [CTA][128] (m, l) pairs)
+//   [kSkFlagsOffset, kAttnFlagsOffset)  GEMM flags, [CTA][4 epilogue warps]
+//   [kAttnFlagsOffset, kScratchBytes)   attention flags, [CTA][4 softmax warps]
+// A flag holds the launch's sequence number (next_scratch_seq) once the 32 partial rows
+// of that warp are written, and is put back to zero by the reader.
+constexpr int kMaxSkCtas = 160;  // grid cap of the split schedules
+constexpr size_t kSkFlagsOffset = size_t(kMaxSkCtas) * 128 * 256 * 4;
+constexpr size_t kAttnFlagsOffset = kSkFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
+constexpr size_t kScratchBytes = kAttnFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
+
+// Bytes of kernel scratch (kScratchBytes).
 size_t gemm_scratch_bytes();
+// A value no flag can hold from an earlier launch of this process.
+unsigned long long next_scratch_seq();
 
 // out = A[M, K] * B[N, K]^T with epilogue; bf16 inputs.  K % 64 == 0, N % 128 == 0.
 // scratch (>= gemm_scratch_bytes(), or null) enables the stream-K schedule when the
@@ -63,8 +79,11 @@ int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, i
                    cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention (tcgen05)
+// scratch (>= gemm_scratch_bytes(), or null) enables the persistent split schedule:
+// one CTA per SM, each taking an equal share of the (query tile, KV tile) steps.
 int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_heads,
-                     int head_dim, bf16* out, cudaStream_t stream);
+                     int head_dim, bf16* out, void* scratch, size_t scratch_bytes,
+                     cudaStream_t stream);
 
 // ---------------------------------------------------------------- row kernels
 int launch_ln_modulate(const bf16* x, int n, int d, float eps, const float* shift,

@@ -74,7 +74,7 @@ _SIGS = {
     "h3b_quantize_rows": (_I, [_P, _I, _I, _P, _P, _P]),
     "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P]),
-    "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P]),
+    "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P, _SZ, _P]),
     "h3b_layer_mask": (_I, [_P, _I, _I, _I, _P]),
 }
 
@@ -301,9 +301,10 @@ def gemm_bf16(A, B, epilogue, bias, out, gate=None, rope_cs=None, rope_cols=0, h
                              _stream(stream)))
 
 
-def attention(qkv, n_heads, head_dim, out, stream=None) -> None:
+def attention(qkv, n_heads, head_dim, out, ws=None, stream=None) -> None:
     _dev(qkv, torch.bfloat16, "qkv"); _dev(out, torch.bfloat16, "out")
-    _check(lib.h3b_attention(_ptr(qkv), qkv.shape[0], n_heads, head_dim, _ptr(out),
+    wp, wb = _wsargs(ws)
+    _check(lib.h3b_attention(_ptr(qkv), qkv.shape[0], n_heads, head_dim, _ptr(out), wp, wb,
                              _stream(stream)))
 
 
