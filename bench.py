@@ -296,7 +296,76 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3)
                      "frac": achieved / peak, "work_per_launch": work,
                      "launches_per_step": launches[name],
                      "ms_per_step": ms * launches[name]}
+        if bound == "hbm":
+            # the same launch with the L2 flushed before each one (its inputs come from HBM)
+            cold = time_cold(lambda: fn(0), dev)
+            out[name]["cold_ms"] = cold
+            out[name]["cold_frac"] = work / (cold * 1e-3) / 1e9 / peaks["hbm_gbs"]
     return out
+
+
+_FLUSH = {}
+
+
+def flush_l2(dev):
+    """Overwrite a buffer twice the size of the 126 MB L2."""
+    import torch
+    buf = _FLUSH.get(dev)
+    if buf is None:
+        buf = _FLUSH[dev] = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    buf.zero_()
+
+
+def time_cold(fn, dev, reps=10):
+    """Average device time of single launches, each after an L2 flush (CUDA events around
+    the launch only)."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    fn()
+    for a, b in ev:
+        flush_l2(dev)
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return sum(a.elapsed_time(b) for a, b in ev) / reps
+
+
+def time_gemm_widths(dev, peaks, reps=10):
+    """bf16 GEMMs at the model widths the pages name (5376, 7168), M = 1600 and 2048 rows:
+    out = A[M, d] W[d, d]^T + bias (an out-projection shape) and the QKV shape N = 3 d."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b
+    g = torch.Generator(device=dev).manual_seed(11)
+    ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
+    res = []
+    for d in (5376, 7168):
+        for M in (1600, 2048):
+            for N in (d, 3 * d):
+                A = (torch.randn(M, d, generator=g, device=dev) * 0.5).to(torch.bfloat16)
+                W = (torch.randn(N, d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+                b = torch.zeros(N, dtype=torch.bfloat16, device=dev)
+                out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                f = lambda: h3b.gemm_bf16(A, W, h3b.EPI_BIAS, b, out, ws=ws)
+                for _ in range(3):
+                    f()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize(dev)
+                e0.record()
+                for _ in range(reps):
+                    f()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                ms = e0.elapsed_time(e1) / reps
+                tf = 2 * M * N * d / (ms * 1e-3) / 1e12
+                res.append({"M": M, "N": N, "K": d, "ms": ms, "tflops": tf,
+                            "frac": tf / peaks["bf16_tflops"]})
+                del A, W, out
+    h3b.sync_status()
+    torch.cuda.empty_cache()
+    return res
 
 
 def time_denoise(cfg_name, dev, reps, warm=1):
@@ -357,6 +426,7 @@ def time_int8_fc2(dev, peaks, reps=10):
         e1.record()
         torch.cuda.synchronize(dev)
         out[name] = e0.elapsed_time(e1) / reps
+    q_cold = time_cold(q_only, dev)
     h3b.sync_status()
     q_bytes = 3 * M * K + 4 * M
     int8_peak = 2 * peaks["bf16_tflops"]
@@ -366,6 +436,8 @@ def time_int8_fc2(dev, peaks, reps=10):
            "quantize_ms": out["quantize_rows"],
            "quantize_gbs": q_bytes / (out["quantize_rows"] * 1e-3) / 1e9,
            "quantize_hbm_frac": q_bytes / (out["quantize_rows"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+           "quantize_cold_ms": q_cold,
+           "quantize_cold_hbm_frac": q_bytes / (q_cold * 1e-3) / 1e9 / peaks["hbm_gbs"],
            "int8_gemm_tops": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12,
            "int8_gemm_frac": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12 / int8_peak,
            "int8_peak_tops": int8_peak, "int8_peak_note": "measured bf16 burst x 2 (nominal ratio)"}
@@ -399,8 +471,11 @@ def time_token_pairing(dev, peaks, reps=20):
         e1.record()
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / reps
+        cold = time_cold(fn, dev)
         res[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
-                     "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                     "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "cold_ms": cold,
+                     "cold_hbm_frac": nbytes / (cold * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     h3b.sync_status()
     res["shape"] = f"{cfg.name} stream: {n} tokens x {d} bf16 -> {nr} tokens"
     return res
@@ -551,6 +626,7 @@ def run_gpu(args):
                 also[name] = time_denoise(name, dev, reps)
         also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
+        also["gemm_widths"] = time_gemm_widths(dev, peaks)
         line["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
