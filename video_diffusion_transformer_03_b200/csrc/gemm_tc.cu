@@ -54,7 +54,7 @@ struct GemmParams {
   // at lower-numbered units, which are dispatched first.
   int sk;
   long long sk_iters;
-  uint32_t* sk_slots;            // [gridDim.x][128][BN] raw accumulator words
+  uint32_t* sk_slots;            // [gridDim.x][BN / 4][128] uint4 of raw accumulator words
   unsigned long long* sk_flags;  // [gridDim.x][4]
   unsigned long long sk_seq;
   GemmEpilogue epi;
@@ -270,47 +270,85 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
   store_bf16x32(dst, v);
 }
 
-// Epilogue of one work unit for one thread (one accumulator row, BN columns starting at
-// col0): TMEM chunk by chunk, plus the stream-K partials held in slots
-// src * stride + off for src in [src_lo, src_hi), then the epilogue and the stores.
+// Stream-K slot of a unit: BN / 4 column groups of 128 rows, so that the 32 rows of a warp
+// read or write 512 contiguous bytes per column group.
+template <int BN>
+__device__ __forceinline__ uint4* sk_slot(const GemmParams& p, int slot_id) {
+  return reinterpret_cast<uint4*>(p.sk_slots) + size_t(slot_id) * (BN / 4) * kBM;
+}
+
+// Park a 128 x BN partial accumulator (this thread's row from TMEM) in a slot.
+template <int BN>
+__device__ __forceinline__ void sk_park(const GemmParams& p, int slot_id, uint32_t tbase,
+                                        int row_in_tile) {
+  uint4* slot = sk_slot<BN>(p, slot_id) + row_in_tile;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    tmem_wait_ld(r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      __stcg(slot + size_t(c * 8 + i) * kBM,
+             make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+  }
+}
+
+template <bool INT8>
+__device__ __forceinline__ void add_part(uint32_t (&r)[32], const uint4 (&part)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t u[4] = {part[i].x, part[i].y, part[i].z, part[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (INT8)
+        r[4 * i + k] = uint32_t(int32_t(r[4 * i + k]) + int32_t(u[k]));
+      else
+        r[4 * i + k] = __float_as_uint(__uint_as_float(r[4 * i + k]) + __uint_as_float(u[k]));
+    }
+  }
+}
+
+// Epilogue of one output tile row (BN columns): accumulator from TMEM, plus the partial
+// tiles parked by units [src_lo, src_hi) (slot src * stride + off), then the fused
+// epilogue.  The next column chunk's row inputs and first partial are fetched while the
+// current chunk is finished.
 template <int BN, bool INT8, int EPI>
 __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbase, int row,
                                               int row_in_tile, int col0, int src_lo,
                                               int src_hi, int stride, int off) {
   constexpr int NC = BN / 32;
   const bool valid = row < p.M;
+  const bool has_part = src_lo < src_hi;
+  const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
   RowIn in[2];
+  uint4 part[2][8];
   if (valid) load_row_in<EPI>(p.epi, row, col0, in[0]);
+  if (has_part) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[0][i] = __ldcg(first + size_t(i) * kBM);
+  }
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
-    if (c + 1 < NC && valid) load_row_in<EPI>(p.epi, row, col0 + (c + 1) * 32, in[(c + 1) & 1]);
-    uint4 part[8];
-    if (src_lo < src_hi) {
-      const uint4* ps = reinterpret_cast<const uint4*>(
-          p.sk_slots + (size_t(src_lo * stride + off) * kBM + row_in_tile) * BN + c * 32);
+    if (c + 1 < NC) {
+      if (valid) load_row_in<EPI>(p.epi, row, col0 + (c + 1) * 32, in[(c + 1) & 1]);
+      if (has_part) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) part[i] = __ldcg(ps + i);
+        for (int i = 0; i < 8; ++i)
+          part[(c + 1) & 1][i] = __ldcg(first + size_t((c + 1) * 8 + i) * kBM);
+      }
     }
     tmem_wait_ld(r);
-    for (int src = src_lo; src < src_hi; ++src) {
-      if (src > src_lo) {
-        const uint4* ps = reinterpret_cast<const uint4*>(
-            p.sk_slots + (size_t(src * stride + off) * kBM + row_in_tile) * BN + c * 32);
+    if (has_part) {
+      add_part<INT8>(r, part[c & 1]);
+      for (int src = src_lo + 1; src < src_hi; ++src) {
+        const uint4* ps = sk_slot<BN>(p, src * stride + off) + row_in_tile;
+        uint4 more[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) part[i] = __ldcg(ps + i);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t u[4] = {part[i].x, part[i].y, part[i].z, part[i].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if constexpr (INT8)
-            r[4 * i + k] = uint32_t(int32_t(r[4 * i + k]) + int32_t(u[k]));
-          else
-            r[4 * i + k] = __float_as_uint(__uint_as_float(r[4 * i + k]) + __uint_as_float(u[k]));
-        }
+        for (int i = 0; i < 8; ++i) more[i] = __ldcg(ps + size_t(c * 8 + i) * kBM);
+        add_part<INT8>(r, more);
       }
     }
     if (valid) epilogue_chunk<EPI>(p.epi, row, col0 + c * 32, r, in[c & 1]);
@@ -472,17 +510,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
       if (kb1 < p.k_blocks) {
         // stream-K contributor: park the partial tile in this CTA's slot
-        uint32_t* slot = p.sk_slots + (size_t(blockIdx.x) * kBM + row_in_tile) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c * 32, r);
-          tmem_wait_ld(r);
-          uint4* dst = reinterpret_cast<uint4*>(slot + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            __stcg(dst + i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
-        }
+        sk_park<BN>(p, static_cast<int>(blockIdx.x), tbase, row_in_tile);
         __threadfence();
         tc_fence_before();
         __syncwarp();
@@ -721,17 +749,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
       if (kb1 < p.k_blocks) {
         // stream-K contributor: park this CTA's half of the partial tile in its slot
-        uint32_t* slot = p.sk_slots + (size_t(slot_id) * kBM + row_in_tile) * BN;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c * 32, r);
-          tmem_wait_ld(r);
-          uint4* dst = reinterpret_cast<uint4*>(slot + c * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            __stcg(dst + i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
-        }
+        sk_park<BN>(p, slot_id, tbase, row_in_tile);
         __threadfence();
         tc_fence_before();
         __syncwarp();
@@ -793,6 +811,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
 std::atomic<unsigned long long> g_sk_seq{0};
 bool trace_gemm();
+int forced_sched();
 
 // A value no flag of the scratch can hold from an earlier launch: a per-process random
 // high half and a launch counter.
@@ -802,18 +821,16 @@ unsigned long long next_sk_seq() {
   return salt + (g_sk_seq.fetch_add(1) << 1);
 }
 
-// Fraction of SM-time a data-parallel schedule of `tiles` equal tiles keeps busy.
-double dp_efficiency(int tiles, int ctas) {
-  const int waves = (tiles + ctas - 1) / ctas;
-  return double(tiles) / (double(waves) * ctas);
-}
-
-// Stream-K pays a fixed cost per unit (partial-tile spill and reload, a second exposed
-// epilogue); measured on B200 it only wins when the data-parallel tail wastes a large
-// share of the SMs and the K loop is long enough to amortise it (1600 x 3072 x 12288:
-// 110 us vs 134 us; with K = 3072 it lost: 53-59 us vs 47 us).
+// Schedule choice from a cost model in units of one K slice of one tile on one scheduling
+// unit.  Data-parallel: ceil(tiles / units) waves of k_blocks slices.  Stream-K: the even
+// share tiles * k_blocks / units, times 1.24, plus 23 (partial-tile parking and merging,
+// the exposed epilogue of the merged tile).  The two constants fit the CTA-pair kernel on
+// B200 at M = 832 and 1600, N = 3072, K = 3072 and 12288 (stream-K / data-parallel time
+// 0.94, 1.28, 0.76, 0.94 measured; the model gives 0.94, 1.28, 0.76, 0.92).
 bool want_stream_k(int tiles, int units, int k_blocks) {
-  return dp_efficiency(tiles, std::min(units, tiles)) < 0.75 && k_blocks >= 128;
+  const double dp = double((tiles + units - 1) / units) * k_blocks;
+  const double sk = 1.24 * double(tiles) * k_blocks / units + 23.0;
+  return sk < dp;
 }
 
 template <int BN, bool INT8, int EPI>
@@ -852,8 +869,10 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_ctas = std::min(ctx.num_sms, kMaxSkCtas);
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
-  const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
-                      want_stream_k(tiles, ctx.num_sms, p.k_blocks) && iters >= 4LL * sk_ctas;
+  const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
+                     iters >= 4LL * sk_ctas;
+  const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() == 1
+                                                    : want_stream_k(tiles, ctx.num_sms, p.k_blocks));
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm 1cta BN=%d M=%d N=%d K=%d tiles=%d sms=%d -> %s grid=%d\n", BN,
                  M, N, K, tiles, ctx.num_sms, use_sk ? "stream-K" : "data-parallel",
@@ -936,8 +955,10 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
-  const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
-                      want_stream_k(tiles, cap, p.k_blocks) && iters >= 4LL * sk_pairs;
+  const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
+                     iters >= 4LL * sk_pairs;
+  const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() == 1
+                                                    : want_stream_k(tiles, cap, p.k_blocks));
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm pair BN=%d M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n",
                  BN, M, N, K, tiles, cap, use_sk ? "stream-K" : "data-parallel",
@@ -958,6 +979,18 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
   *rc = check_launch("gemm_pair");
   return 0;
+}
+
+// H3B_GEMM_SCHED=sk|dp forces the stream-K or the data-parallel schedule where the
+// scratch allows it (diagnostics and measurements only).
+int forced_sched() {
+  static const int forced = [] {
+    const char* v = std::getenv("H3B_GEMM_SCHED");
+    if (!v) return -1;
+    const std::string t(v);
+    return t == "sk" ? 1 : t == "dp" ? 0 : -1;
+  }();
+  return forced;
 }
 
 // H3B_TRACE_GEMM=1 prints each GEMM's schedule to stderr (diagnostics only).
