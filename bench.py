@@ -45,8 +45,8 @@ NCU_TRAFFIC = {
                       "src_sha": "d8d12281faaa06e2"},
     "gemm_out_gate": {"bytes": 38645504 + 1378816, "src": "gemm_tc.cu",
                       "src_sha": "d8d12281faaa06e2"},
-    "gemm_fc1_gelu": {"bytes": 85552896 + 14709248, "src": "gemm_tc.cu",
-                      "src_sha": "84edba3bedaede90"},
+    "gemm_fc1_gelu": {"bytes": 85510912 + 14807808, "src": "gemm_tc.cu",
+                      "src_sha": "d8d12281faaa06e2"},
 }
 
 
@@ -229,8 +229,9 @@ def workload_name(cfg):
 
 # ------------------------------------------------------------------------------ GPU arm
 def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3):
-    """Time each kernel of the block alone (CUDA events on the launching stream), with the
-    weights rotated over all blocks so that they stream from HBM as in the step."""
+    """Time each kernel of the block alone (CUDA events around a CUDA-graph replay of
+    `reps` launches, as the denoise runs them), with the weights rotated over all blocks
+    so that they stream from HBM as in the step."""
     import torch
     from video_diffusion_transformer_03_b200 import h3b
     dev = model.device
@@ -273,21 +274,29 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3)
     launches = {"gemm_qkv_rope": blocks, "attention": blocks, "gemm_out_gate": blocks,
                 "gemm_fc1_gelu": blocks, "gemm_fc2_gate": blocks, "ln_modulate": 2 * blocks,
                 "final_euler": cfg.run_steps}
-    stream = torch.cuda.current_stream(dev)
     out = {}
     for name, (fn, bound, work) in kinds.items():
         if only is not None and name != only:
             continue
         for i in range(warm):
             fn(i)
+        torch.cuda.synchronize(dev)
+        # the reps are captured as one CUDA graph and replayed, so the device time is not
+        # bounded by the host's per-call cost (short kernels would otherwise measure it)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(reps):
+                fn(i)
+        graph.replay()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        stream = torch.cuda.current_stream(dev)
         torch.cuda.synchronize(dev)
         e0.record(stream)
-        for i in range(reps):
-            fn(i)
+        graph.replay()
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        del graph
         h3b.sync_status()
         ms = e0.elapsed_time(e1) / reps
         if bound == "tensor":
