@@ -492,31 +492,59 @@ def time_token_pairing(dev, peaks, reps=20):
     return res
 
 
+class Replicas:
+    """The N-GPU run: one process per GPU (torchrun sets RANK / WORLD_SIZE), each an
+    independent replica of the whole denoise; nothing crosses GPUs on the data path.  The
+    only collectives are the timing barrier and the max of the device times over ranks."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=300):
+        import datetime
+        import torch.distributed as dist
+        self.dist = dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.backend = backend
+        self.device = device
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            if self.backend == "nccl":
+                self.dist.barrier(device_ids=[self.device.index])
+            else:
+                self.dist.barrier()
+
+    def max(self, v):
+        """Max of a per-rank float over all ranks (the slowest replica sets the time)."""
+        if self.world == 1:
+            return float(v)
+        import torch
+        t = torch.tensor([float(v)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def throughput(self, units_per_step, steps, ms_max):
+        """Whole-job rate: every rank processed units_per_step per step."""
+        return units_per_step * steps * self.world / (ms_max * 1e-3)
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
 def run_gpu(args):
     import torch
-    import torch.distributed as dist
     from video_diffusion_transformer_03_b200 import h3b, synth
     from video_diffusion_transformer_03_b200.pipeline import DiTDenoiser
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
-
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    reps = Replicas("nccl", dev)
+    world, rank = reps.world, reps.rank
+    barrier, max_over_ranks = reps.barrier, reps.max
 
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.config]
@@ -570,7 +598,7 @@ def run_gpu(args):
     h3b.sync_status()
     ms = max_over_ranks(e0.elapsed_time(e1))
     ms_step = ms / args.steps
-    value = counts["tokens"] * args.steps * world / (ms * 1e-3)
+    value = reps.throughput(counts["tokens"], args.steps, ms)
     tflops = counts["flops"] * args.steps * world / (ms * 1e-3) / 1e12
 
     # ---- end to end through the host-buffer entry point (copies inside the timed region)
@@ -591,7 +619,7 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e2.elapsed_time(e3))
     nbytes = host_in.numel() * host_in.element_size()
-    e2e = {"value": counts["tokens"] * e2e_steps * world / (e2e_ms * 1e-3), "unit": UNIT,
+    e2e = {"value": reps.throughput(counts["tokens"], e2e_steps, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
            "ms_per_step": e2e_ms / e2e_steps}
 
@@ -642,8 +670,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
     del graph
-    if world > 1:
-        dist.destroy_process_group()
+    reps.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
