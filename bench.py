@@ -542,9 +542,9 @@ def run_gpu(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    reps = Replicas("nccl", dev)
-    world, rank = reps.world, reps.rank
-    barrier, max_over_ranks = reps.barrier, reps.max
+    replicas = Replicas("nccl", dev)
+    world, rank = replicas.world, replicas.rank
+    barrier, max_over_ranks = replicas.barrier, replicas.max
 
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.config]
@@ -598,30 +598,35 @@ def run_gpu(args):
     h3b.sync_status()
     ms = max_over_ranks(e0.elapsed_time(e1))
     ms_step = ms / args.steps
-    value = reps.throughput(counts["tokens"], args.steps, ms)
+    value = replicas.throughput(counts["tokens"], args.steps, ms)
     tflops = counts["flops"] * args.steps * world / (ms * 1e-3) / 1e12
 
-    # ---- end to end through the host-buffer entry point (copies inside the timed region)
-    host_in = synth.latent_noise(cfg).pin_memory()
+    # ---- end to end through the host-buffer entry point (copies inside the timed region):
+    # batches of requests, each uploaded from pinned host memory and its result downloaded,
+    # the copies overlapped with the neighbouring requests' compute
+    e2e_steps = max(1, args.steps // 2)
+    batch = min(10, e2e_steps)
+    n_batches = (e2e_steps + batch - 1) // batch
+    e2e_steps = n_batches * batch
+    host_in = torch.stack([synth.latent_noise(cfg)] * batch).pin_memory()
     host_out = torch.empty_like(host_in).pin_memory()
-    scratch = torch.empty_like(x0)
-    for _ in range(min(args.warmup, 3)):
-        model.run_host(host_in, host_out, scratch)
+    state2 = torch.empty((2,) + tuple(x0.shape), dtype=torch.float32, device=dev)
+    model.run_host_pipelined(host_in[:2], host_out[:2], state2)
     barrier()
     e2 = torch.cuda.Event(enable_timing=True)
     e3 = torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, args.steps // 2)
     torch.cuda.synchronize(dev)
     e2.record(stream)
-    for _ in range(e2e_steps):
-        model.run_host(host_in, host_out, scratch)
+    for _ in range(n_batches):
+        model.run_host_pipelined(host_in, host_out, state2)
     e3.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e2.elapsed_time(e3))
-    nbytes = host_in.numel() * host_in.element_size()
-    e2e = {"value": reps.throughput(counts["tokens"], e2e_steps, e2e_ms), "unit": UNIT,
+    nbytes = host_in[0].numel() * host_in.element_size()
+    e2e = {"value": replicas.throughput(counts["tokens"], e2e_steps, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
-           "ms_per_step": e2e_ms / e2e_steps}
+           "ms_per_step": e2e_ms / e2e_steps,
+           "api": f"h3b_denoise_host_pipelined, {batch} requests per call"}
 
     breakdown = None
     roofline = None
@@ -670,7 +675,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
     del graph
-    reps.close()
+    replicas.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
 

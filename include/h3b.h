@@ -20,13 +20,14 @@
  * Conventions for every entry point:
  *   - Pointers marked "device" are CUDA device pointers owned by the caller; pointers
  *     marked "host" are host pointers.  The library never allocates or frees device
- *     memory except in h3b_denoise_host, which is documented below.
+ *     memory (h3b_denoise_host_pipelined creates two copy streams and a few events per
+ *     device on its first call and keeps them).
  *   - Tensors are dense row-major; "[a, b]" means b is the contiguous dimension.
  *     Every device pointer must be 16-byte aligned.
  *   - h3b_bf16 is bfloat16 storage (IEEE-754 binary32 with the low 16 bits dropped).
  *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
  *     Calls are asynchronous on that stream; no host synchronisation happens inside
- *     (except h3b_sync_status and h3b_denoise_host).
+ *     (except h3b_sync_status, h3b_denoise_host and h3b_denoise_host_pipelined).
  *   - Return value: H3B_OK (0) or a negative H3B_E* code.  All argument validation
  *     happens before the first launch, so a call that fails validation launches
  *     nothing.  h3b_last_error() returns a message for the calling thread's last error.
@@ -224,6 +225,23 @@ int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                      int unpair_bypass, int n_steps, int first_step, int n_run,
                      const float* x_host_in, float* x_host_out, float* x_state_dev,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* Serving form of h3b_denoise_host: n_requests independent whole denoises of HOST
+ * latents, request r read from x_host_in + r * n_tokens * d and written to
+ * x_host_out + r * n_tokens * d ([n_requests, n_tokens, d] fp32, pinned for full copy
+ * bandwidth).  Request r computes on `stream` while the library's copy streams upload
+ * request r + 1 and download request r - 1, so the copies overlap the compute; every
+ * request still makes its own host-to-device and device-to-host trip.  x_state_dev:
+ * device [2, n_tokens, d] fp32 (two state buffers, alternating).  The work is ordered
+ * after what `stream` already holds, and `stream` is synchronised before returning.
+ * Calls on one device must not overlap (the copy streams are shared).  No counterpart
+ * on the pages: the host-side pipelining of a serving loop around the denoise. */
+int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                               const h3b_block_weights* blocks, const unsigned char* active,
+                               const float* mods, const float* final_mod, int reduce_after,
+                               int unpair_bypass, int n_steps, int first_step, int n_run,
+                               int n_requests, const float* x_host_in, float* x_host_out,
+                               float* x_state_dev, void* ws, size_t ws_bytes, void* stream);
 
 /* Horizontal token pairing (ditty.ir; dothoosh.com "Aggressive optimisation levers").
  * mode H3B_PAIR:   dst[t,h,j] = (src[t,h,2j] + src[t,h,2j+1]) / 2, audio rows copied;

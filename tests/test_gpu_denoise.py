@@ -83,6 +83,26 @@ def test_host_entry_matches_device_steps(name):
     assert torch.equal(host_out, xd.cpu())          # same kernels, same order: bit-equal
 
 
+@pytest.mark.parametrize("name,requests", [("tiny", 5), ("dit512", 3), ("dit512_tokred", 2)])
+def test_pipelined_host_entry_matches_device_runs(name, requests):
+    cfg = synth.CONFIGS[name]
+    m = DiTDenoiser(cfg)
+    g = torch.Generator().manual_seed(5)
+    x0 = torch.randn((requests, cfg.n_tokens, cfg.d), generator=g).to(torch.bfloat16).float()
+    want = []
+    for r in range(requests):
+        xd = x0[r].to(DEV)
+        m.run(xd)
+        want.append(xd.cpu())
+    h3b.sync_status()
+    host_in = x0.pin_memory()
+    host_out = torch.full_like(host_in, float("nan")).pin_memory()
+    state2 = torch.empty((2, cfg.n_tokens, cfg.d), dtype=torch.float32, device=DEV)
+    m.run_host_pipelined(host_in, host_out, state2)
+    for r in range(requests):        # same kernels, same order per request: bit-equal
+        assert torch.equal(host_out[r], want[r]), f"request {r}"
+
+
 def test_768x1344_full_denoise_is_finite_and_deterministic():
     cfg = synth.CONFIGS["dit768x1344"]
     m = DiTDenoiser(cfg, gen_device="cuda")

@@ -522,6 +522,100 @@ int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
   return h3b_sync_status(stream);
 }
 
+namespace {
+
+// Copy streams and events of the pipelined host entry point, created once per device.
+struct CopyLanes {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t start = nullptr, in[2] = {}, done[2] = {}, out[2] = {};
+};
+
+int copy_lanes(int device, CopyLanes** out) {
+  static std::mutex mu;
+  static CopyLanes lanes[kMaxDevices];
+  static bool ready[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  CopyLanes& l = lanes[device];
+  if (!ready[device]) {
+    cudaError_t e = cudaStreamCreateWithFlags(&l.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&l.down, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&l.start, &l.in[0], &l.in[1], &l.done[0], &l.done[1], &l.out[0],
+                          &l.out[1]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess)
+      return set_error(H3B_ECUDA, "denoise_host_pipelined: stream/event creation: %s",
+                       cudaGetErrorString(e));
+    ready[device] = true;
+  }
+  *out = &l;
+  return 0;
+}
+
+}  // namespace
+
+int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                               const h3b_block_weights* blocks, const unsigned char* active,
+                               const float* mods, const float* final_mod, int reduce_after,
+                               int unpair_bypass, int n_steps, int first_step, int n_run,
+                               int n_requests, const float* x_host_in, float* x_host_out,
+                               float* x_state_dev, void* ws, size_t ws_bytes, void* stream) {
+  StepBufs b;
+  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
+                           x_state_dev, ws, ws_bytes, &b);
+  if (rc) return rc;
+  if (!x_host_in || !x_host_out || n_requests < 0)
+    return set_error(H3B_EINVAL, "denoise_host_pipelined: NULL host buffer or %d requests",
+                     n_requests);
+  if (n_steps <= 0 || first_step < 0 || n_run < 0 || first_step + n_run > n_steps)
+    return set_error(H3B_EINVAL, "denoise_host_pipelined: steps %d..%d of %d", first_step,
+                     first_step + n_run, n_steps);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  CopyLanes* l = nullptr;
+  if ((rc = copy_lanes(ctx.device, &l))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t elems = (size_t(grid->t) * grid->h * grid->w + grid->n_audio) * dims->d;
+  const size_t bytes = elems * sizeof(float);
+  auto fail = [](cudaError_t e, const char* what) {
+    return set_error(H3B_ECUDA, "denoise_host_pipelined: %s: %s", what, cudaGetErrorString(e));
+  };
+  cudaError_t e;
+  // everything below is ordered after the work already on `stream`
+  if ((e = cudaEventRecord(l->start, s)) != cudaSuccess) return fail(e, "record");
+  if ((e = cudaStreamWaitEvent(l->up, l->start, 0)) != cudaSuccess) return fail(e, "wait");
+  for (int r = 0; r < n_requests; ++r) {
+    const int k = r & 1;
+    float* state = x_state_dev + k * elems;
+    // upload r into state buffer k once request r - 2 has been downloaded from it
+    if (r >= 2 && (e = cudaStreamWaitEvent(l->up, l->out[k], 0)) != cudaSuccess)
+      return fail(e, "wait");
+    if ((e = cudaMemcpyAsync(state, x_host_in + r * elems, bytes, cudaMemcpyHostToDevice,
+                             l->up)) != cudaSuccess)
+      return fail(e, "H2D");
+    if ((e = cudaEventRecord(l->in[k], l->up)) != cudaSuccess) return fail(e, "record");
+    if ((e = cudaStreamWaitEvent(s, l->in[k], 0)) != cudaSuccess) return fail(e, "wait");
+    for (int i = first_step; i < first_step + n_run; ++i) {
+      const float sg = static_cast<float>(1.0 - double(i) / n_steps);
+      const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
+      if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                                  reduce_after, unpair_bypass, sg, sn, state, b, s)))
+        return rc;
+    }
+    if ((e = cudaEventRecord(l->done[k], s)) != cudaSuccess) return fail(e, "record");
+    if ((e = cudaStreamWaitEvent(l->down, l->done[k], 0)) != cudaSuccess) return fail(e, "wait");
+    if ((e = cudaMemcpyAsync(x_host_out + r * elems, state, bytes, cudaMemcpyDeviceToHost,
+                             l->down)) != cudaSuccess)
+      return fail(e, "D2H");
+    if ((e = cudaEventRecord(l->out[k], l->down)) != cudaSuccess) return fail(e, "record");
+  }
+  // the call ends on `stream` after the last download
+  for (int k = 0; k < 2 && k < n_requests; ++k)
+    if ((e = cudaStreamWaitEvent(s, l->out[(n_requests - 1 - k) & 1], 0)) != cudaSuccess)
+      return fail(e, "wait");
+  return h3b_sync_status(stream);
+}
+
 int h3b_token_reduce(int mode, const h3b_bf16* src, h3b_bf16* dst, const h3b_bf16* saved, int t,
                      int h, int w, int n_audio, int d, void* stream) {
   if (mode != H3B_PAIR && mode != H3B_UNPAIR) return set_error(H3B_EINVAL, "token_reduce: mode %d", mode);

@@ -70,6 +70,9 @@ _SIGS = {
     "h3b_denoise_host": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                               ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _I, _I, _I, _P,
                               _P, _P, _P, _SZ, _P]),
+    "h3b_denoise_host_pipelined": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                                        ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _I,
+                                        _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "h3b_token_reduce": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "h3b_quantize_rows": (_I, [_P, _I, _I, _P, _P, _P]),
     "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -265,6 +268,26 @@ def denoise_host(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active,
                                 n_steps, first_step, n_run, _ptr(x_host_in), _ptr(x_host_out),
                                 _ptr(x_state_dev), _ptr(ws), ws.numel() * ws.element_size(),
                                 _stream(stream)))
+    del keep
+
+
+def denoise_host_pipelined(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods,
+                           final_mod, reduce_after: int, unpair_bypass: bool, n_steps: int,
+                           first_step: int, n_run: int, x_host_in, x_host_out, x_state_dev2,
+                           ws, stream=None) -> None:
+    """x_host_in / x_host_out: CPU float32 [requests, n_tokens, d] (pinned);
+    x_state_dev2: device float32 [2, n_tokens, d]."""
+    if x_host_in.is_cuda or x_host_out.is_cuda:
+        raise TypeError("denoise_host_pipelined takes host buffers")
+    if x_host_in.shape != x_host_out.shape or x_state_dev2.shape[0] != 2:
+        raise ValueError("denoise_host_pipelined: shapes")
+    arr = _blocks_array(blocks)
+    keep, mask = _mask_array(active, len(blocks))
+    _check(lib.h3b_denoise_host_pipelined(
+        ctypes.byref(dims), ctypes.byref(grid), len(blocks), arr, mask, _ptr(mods),
+        _ptr(final_mod), reduce_after, int(bool(unpair_bypass)), n_steps, first_step, n_run,
+        x_host_in.shape[0], _ptr(x_host_in), _ptr(x_host_out), _ptr(x_state_dev2), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
     del keep
 
 

@@ -87,6 +87,17 @@ class DiTDenoiser:
             self.run(x_state, n_run)
         return graph
 
+    def run_host_pipelined(self, x_host_in: torch.Tensor, x_host_out: torch.Tensor,
+                           x_state_dev2: torch.Tensor, n_run: Optional[int] = None,
+                           stream=None) -> None:
+        """Whole denoises of a batch of host latents [requests, n_tokens, d], copies
+        overlapped with compute (h3b_denoise_host_pipelined)."""
+        h3b.denoise_host_pipelined(self.dims, self.grid, self.weights, self.active, self.mods,
+                                   self.final_mod, self.cfg.reduce_after,
+                                   self.cfg.unpair_bypass, self.cfg.steps, 0,
+                                   self.cfg.run_steps if n_run is None else n_run, x_host_in,
+                                   x_host_out, x_state_dev2, self.ws, stream)
+
     def run_host(self, x_host_in: torch.Tensor, x_host_out: torch.Tensor,
                  x_state_dev: torch.Tensor, n_run: Optional[int] = None, stream=None) -> None:
         h3b.denoise_host(self.dims, self.grid, self.weights, self.active, self.mods,
