@@ -234,6 +234,8 @@ int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
  * request still makes its own host-to-device and device-to-host trip.  x_state_dev:
  * device [2, n_tokens, d] fp32 (two state buffers, alternating).  The work is ordered
  * after what `stream` already holds, and `stream` is synchronised before returning.
+ * Each request's Euler steps run as a CUDA graph captured on the first call with these
+ * arguments (the library keeps the last four per device; H3B_DEBUG=1 launches directly).
  * Calls on one device must not overlap (the copy streams are shared).  No counterpart
  * on the pages: the host-side pipelining of a serving loop around the denoise. */
 int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,

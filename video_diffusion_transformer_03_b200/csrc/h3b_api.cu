@@ -554,6 +554,98 @@ int copy_lanes(int device, CopyLanes** out) {
 
 }  // namespace
 
+namespace {
+
+// Captured whole denoises (the Euler steps of one request on one state buffer), kept per
+// device and keyed by every argument that shapes the launches: a replay relaunches the
+// same kernels with the same arguments (the split schedules' flags are handed back at zero
+// by their readers, so replays stay correct).  Captured on a stream of the library's and
+// launched on the caller's.
+struct DenoiseGraph {
+  std::vector<uint8_t> key;
+  cudaGraphExec_t exec = nullptr;
+};
+
+constexpr size_t kGraphCacheSize = 4;
+
+void key_bytes(std::vector<uint8_t>& k, const void* v, size_t n) {
+  const uint8_t* b = static_cast<const uint8_t*>(v);
+  k.insert(k.end(), b, b + n);
+}
+#define H3B_KEY_PUT(k, v) key_bytes((k), &(v), sizeof(v))
+
+int denoise_graph(const DevCtx& ctx, const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                  const h3b_block_weights* blocks, const unsigned char* active,
+                  const float* mods, const float* final_mod, int reduce_after,
+                  int unpair_bypass, int n_steps, int first_step, int n_run, float* state,
+                  const StepBufs& b, void* ws, size_t ws_bytes, cudaGraphExec_t* out) {
+  static std::mutex mu;
+  static std::vector<DenoiseGraph> cache[kMaxDevices];
+  static cudaStream_t capture_stream[kMaxDevices] = {};
+  std::vector<uint8_t> key;
+  H3B_KEY_PUT(key, *dims);
+  H3B_KEY_PUT(key, *grid);
+  H3B_KEY_PUT(key, n_blocks);
+  for (int i = 0; i < n_blocks; ++i) {
+    H3B_KEY_PUT(key, blocks[i]);
+    const unsigned char on = active ? active[i] : 1;
+    H3B_KEY_PUT(key, on);
+  }
+  H3B_KEY_PUT(key, mods);
+  H3B_KEY_PUT(key, final_mod);
+  H3B_KEY_PUT(key, reduce_after);
+  H3B_KEY_PUT(key, unpair_bypass);
+  H3B_KEY_PUT(key, n_steps);
+  H3B_KEY_PUT(key, first_step);
+  H3B_KEY_PUT(key, n_run);
+  H3B_KEY_PUT(key, state);
+  H3B_KEY_PUT(key, ws);
+  H3B_KEY_PUT(key, ws_bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  auto& c = cache[ctx.device];
+  for (const DenoiseGraph& gph : c)
+    if (gph.key == key) {
+      *out = gph.exec;
+      return 0;
+    }
+  cudaError_t e = cudaSuccess;
+  if (!capture_stream[ctx.device])
+    e = cudaStreamCreateWithFlags(&capture_stream[ctx.device], cudaStreamNonBlocking);
+  if (e != cudaSuccess)
+    return set_error(H3B_ECUDA, "denoise graph: stream: %s", cudaGetErrorString(e));
+  cudaStream_t cs = capture_stream[ctx.device];
+  if ((e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal)) != cudaSuccess)
+    return set_error(H3B_ECUDA, "denoise graph: begin capture: %s", cudaGetErrorString(e));
+  int rc = 0;
+  for (int i = first_step; i < first_step + n_run && rc == 0; ++i) {
+    const float sg = static_cast<float>(1.0 - double(i) / n_steps);
+    const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
+    rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                           reduce_after, unpair_bypass, sg, sn, state, b, cs);
+  }
+  cudaGraph_t graph = nullptr;
+  e = cudaStreamEndCapture(cs, &graph);
+  if (rc != 0 || e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return rc ? rc : set_error(H3B_ECUDA, "denoise graph: capture: %s", cudaGetErrorString(e));
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess)
+    return set_error(H3B_ECUDA, "denoise graph: instantiate: %s", cudaGetErrorString(e));
+  if (c.size() >= kGraphCacheSize) {
+    cudaGraphExecDestroy(c.front().exec);
+    c.erase(c.begin());
+  }
+  c.push_back({std::move(key), exec});
+  *out = exec;
+  return 0;
+}
+
+}  // namespace
+
 int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                                const h3b_block_weights* blocks, const unsigned char* active,
                                const float* mods, const float* final_mod, int reduce_after,
@@ -581,6 +673,15 @@ int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n
     return set_error(H3B_ECUDA, "denoise_host_pipelined: %s: %s", what, cudaGetErrorString(e));
   };
   cudaError_t e;
+  // one captured denoise per state buffer (reused across calls with the same arguments);
+  // with H3B_DEBUG the steps are launched directly so that each launch is checked
+  cudaGraphExec_t graphs[2] = {nullptr, nullptr};
+  if (!debug_mode())
+    for (int k = 0; k < 2 && k < n_requests; ++k)
+      if ((rc = denoise_graph(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                              reduce_after, unpair_bypass, n_steps, first_step, n_run,
+                              x_state_dev + k * elems, b, ws, ws_bytes, &graphs[k])))
+        return rc;
   // everything below is ordered after the work already on `stream`
   if ((e = cudaEventRecord(l->start, s)) != cudaSuccess) return fail(e, "record");
   if ((e = cudaStreamWaitEvent(l->up, l->start, 0)) != cudaSuccess) return fail(e, "wait");
@@ -595,12 +696,16 @@ int h3b_denoise_host_pipelined(const h3b_dims* dims, const h3b_grid* grid, int n
       return fail(e, "H2D");
     if ((e = cudaEventRecord(l->in[k], l->up)) != cudaSuccess) return fail(e, "record");
     if ((e = cudaStreamWaitEvent(s, l->in[k], 0)) != cudaSuccess) return fail(e, "wait");
-    for (int i = first_step; i < first_step + n_run; ++i) {
-      const float sg = static_cast<float>(1.0 - double(i) / n_steps);
-      const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
-      if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
-                                  reduce_after, unpair_bypass, sg, sn, state, b, s)))
-        return rc;
+    if (graphs[k]) {
+      if ((e = cudaGraphLaunch(graphs[k], s)) != cudaSuccess) return fail(e, "graph launch");
+    } else {
+      for (int i = first_step; i < first_step + n_run; ++i) {
+        const float sg = static_cast<float>(1.0 - double(i) / n_steps);
+        const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
+        if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                                    reduce_after, unpair_bypass, sg, sn, state, b, s)))
+          return rc;
+      }
     }
     if ((e = cudaEventRecord(l->done[k], s)) != cudaSuccess) return fail(e, "record");
     if ((e = cudaStreamWaitEvent(l->down, l->done[k], 0)) != cudaSuccess) return fail(e, "wait");
