@@ -60,7 +60,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="time one kernel of the block alone on the workload shapes (for ncu)")
+                    help="time one kernel of the block alone on the workload shapes, or the "
+                         "fc2_int8_row / token_pairing workload (for ncu)")
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--no-also", action="store_true",
                     help="skip the secondary measurements of the other workloads")
@@ -547,6 +548,12 @@ def run_gpu(args):
     barrier, max_over_ranks = replicas.barrier, replicas.max
 
     peaks, peak_src = load_peaks()
+    if args.kernel in ("fc2_int8_row", "token_pairing"):  # workloads outside the block
+        res = (time_int8_fc2(dev, peaks, reps=args.reps) if args.kernel == "fc2_int8_row"
+               else time_token_pairing(dev, peaks, reps=args.reps))
+        if rank == 0:
+            print(json.dumps({"kernel_only": args.kernel, **res}), flush=True)
+        return
     cfg = synth.CONFIGS[args.config]
     model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
     counts, n_active = workload_counts(cfg, model.active)
