@@ -213,23 +213,27 @@ __global__ void k_token_unpair(const bf16* __restrict__ src, bf16* dst, const bf
 
 // One block per row; the row stays in registers (cols <= 256 * 8 * MAXV).
 template <int MAXV>
-__global__ void __launch_bounds__(256) k_quantize_rows(const bf16* __restrict__ a, int cols,
-                                                       int8_t* __restrict__ q,
-                                                       float* __restrict__ scale) {
+__global__ void __launch_bounds__(256, 3) k_quantize_rows(const bf16* __restrict__ a, int cols,
+                                                          int8_t* __restrict__ q,
+                                                          float* __restrict__ scale) {
   __shared__ float red[8];
   const int row = blockIdx.x;
   const int nvec = cols >> 3;
   const uint4* src = reinterpret_cast<const uint4*>(a + size_t(row) * cols);
-  float v[MAXV][8];
+  // the row stays packed (4 registers per 8 values) so that three blocks fit on an SM
+  uint4 raw[MAXV];
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int vi = i * 256 + threadIdx.x;
-    if (vi < nvec) {
-      unpack8(__ldg(src + vi), v[i]);
+    raw[i] = vi < nvec ? __ldg(src + vi) : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[i][k]));
-    }
+  for (int i = 0; i < MAXV; ++i) {
+    float v[8];
+    unpack8(raw[i], v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[k]));
   }
   amax = warp_max(amax);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
@@ -243,10 +247,12 @@ __global__ void __launch_bounds__(256) k_quantize_rows(const bf16* __restrict__ 
   for (int i = 0; i < MAXV; ++i) {
     const int vi = i * 256 + threadIdx.x;
     if (vi < nvec) {
+      float v[8];
+      unpack8(raw[i], v);
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        int qi = __float2int_rn(__fmul_rn(v[i][k], inv));
+        int qi = __float2int_rn(__fmul_rn(v[k], inv));
         qi = max(-127, min(127, qi));
         w[k >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (k & 3));
       }
