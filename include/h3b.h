@@ -218,7 +218,8 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
  * runs Euler steps first_step .. first_step + n_run - 1 of the linear grid with n_steps
  * intervals (sigma_i = 1 - i / n_steps), copies the state back into x_host_out and
  * synchronises `stream`.  x_state_dev: device [n_tokens, d] fp32 scratch for the state.
- * Host buffers should be pinned for full copy bandwidth. */
+ * Host buffers should be pinned for full copy bandwidth.  The steps run as a CUDA graph
+ * captured on the first call with these arguments (see h3b_denoise_host_pipelined). */
 int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                      const h3b_block_weights* blocks, const unsigned char* active,
                      const float* mods, const float* final_mod, int reduce_after,

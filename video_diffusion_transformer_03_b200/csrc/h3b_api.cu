@@ -490,70 +490,6 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                            static_cast<cudaStream_t>(stream));
 }
 
-int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
-                     const h3b_block_weights* blocks, const unsigned char* active,
-                     const float* mods, const float* final_mod, int reduce_after,
-                     int unpair_bypass, int n_steps, int first_step, int n_run,
-                     const float* x_host_in, float* x_host_out, float* x_state_dev,
-                     void* ws, size_t ws_bytes, void* stream) {
-  StepBufs b;
-  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
-                           x_state_dev, ws, ws_bytes, &b);
-  if (rc) return rc;
-  if (!x_host_in || !x_host_out) return set_error(H3B_EINVAL, "denoise_host: NULL host buffer");
-  if (n_steps <= 0 || first_step < 0 || n_run < 0 || first_step + n_run > n_steps)
-    return set_error(H3B_EINVAL, "denoise_host: steps %d..%d of %d", first_step,
-                     first_step + n_run, n_steps);
-  DevCtx ctx;
-  if ((rc = get_ctx(&ctx))) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t bytes = (size_t(grid->t) * grid->h * grid->w + grid->n_audio) * dims->d * 4;
-  cudaError_t e = cudaMemcpyAsync(x_state_dev, x_host_in, bytes, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host H2D: %s", cudaGetErrorString(e));
-  for (int i = first_step; i < first_step + n_run; ++i) {
-    const float sg = static_cast<float>(1.0 - double(i) / n_steps);
-    const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
-    if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
-                                reduce_after, unpair_bypass, sg, sn, x_state_dev, b, s)))
-      return rc;
-  }
-  e = cudaMemcpyAsync(x_host_out, x_state_dev, bytes, cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host D2H: %s", cudaGetErrorString(e));
-  return h3b_sync_status(stream);
-}
-
-namespace {
-
-// Copy streams and events of the pipelined host entry point, created once per device.
-struct CopyLanes {
-  cudaStream_t up = nullptr, down = nullptr;
-  cudaEvent_t start = nullptr, in[2] = {}, done[2] = {}, out[2] = {};
-};
-
-int copy_lanes(int device, CopyLanes** out) {
-  static std::mutex mu;
-  static CopyLanes lanes[kMaxDevices];
-  static bool ready[kMaxDevices] = {};
-  std::lock_guard<std::mutex> lock(mu);
-  CopyLanes& l = lanes[device];
-  if (!ready[device]) {
-    cudaError_t e = cudaStreamCreateWithFlags(&l.up, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&l.down, cudaStreamNonBlocking);
-    cudaEvent_t* evs[] = {&l.start, &l.in[0], &l.in[1], &l.done[0], &l.done[1], &l.out[0],
-                          &l.out[1]};
-    for (cudaEvent_t* ev : evs)
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
-    if (e != cudaSuccess)
-      return set_error(H3B_ECUDA, "denoise_host_pipelined: stream/event creation: %s",
-                       cudaGetErrorString(e));
-    ready[device] = true;
-  }
-  *out = &l;
-  return 0;
-}
-
-}  // namespace
-
 namespace {
 
 // Captured whole denoises (the Euler steps of one request on one state buffer), kept per
@@ -641,6 +577,82 @@ int denoise_graph(const DevCtx& ctx, const h3b_dims* dims, const h3b_grid* grid,
   }
   c.push_back({std::move(key), exec});
   *out = exec;
+  return 0;
+}
+
+}  // namespace
+
+int h3b_denoise_host(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                     const h3b_block_weights* blocks, const unsigned char* active,
+                     const float* mods, const float* final_mod, int reduce_after,
+                     int unpair_bypass, int n_steps, int first_step, int n_run,
+                     const float* x_host_in, float* x_host_out, float* x_state_dev,
+                     void* ws, size_t ws_bytes, void* stream) {
+  StepBufs b;
+  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
+                           x_state_dev, ws, ws_bytes, &b);
+  if (rc) return rc;
+  if (!x_host_in || !x_host_out) return set_error(H3B_EINVAL, "denoise_host: NULL host buffer");
+  if (n_steps <= 0 || first_step < 0 || n_run < 0 || first_step + n_run > n_steps)
+    return set_error(H3B_EINVAL, "denoise_host: steps %d..%d of %d", first_step,
+                     first_step + n_run, n_steps);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the Euler steps as one cached CUDA graph (direct launches with H3B_DEBUG)
+  cudaGraphExec_t graph = nullptr;
+  if (!debug_mode() &&
+      (rc = denoise_graph(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                          reduce_after, unpair_bypass, n_steps, first_step, n_run, x_state_dev,
+                          b, ws, ws_bytes, &graph)))
+    return rc;
+  const size_t bytes = (size_t(grid->t) * grid->h * grid->w + grid->n_audio) * dims->d * 4;
+  cudaError_t e = cudaMemcpyAsync(x_state_dev, x_host_in, bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host H2D: %s", cudaGetErrorString(e));
+  if (graph) {
+    if ((e = cudaGraphLaunch(graph, s)) != cudaSuccess)
+      return set_error(H3B_ECUDA, "denoise_host graph launch: %s", cudaGetErrorString(e));
+  } else {
+    for (int i = first_step; i < first_step + n_run; ++i) {
+      const float sg = static_cast<float>(1.0 - double(i) / n_steps);
+      const float sn = static_cast<float>(1.0 - double(i + 1) / n_steps);
+      if ((rc = denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                                  reduce_after, unpair_bypass, sg, sn, x_state_dev, b, s)))
+        return rc;
+    }
+  }
+  e = cudaMemcpyAsync(x_host_out, x_state_dev, bytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return set_error(H3B_ECUDA, "denoise_host D2H: %s", cudaGetErrorString(e));
+  return h3b_sync_status(stream);
+}
+
+namespace {
+
+// Copy streams and events of the pipelined host entry point, created once per device.
+struct CopyLanes {
+  cudaStream_t up = nullptr, down = nullptr;
+  cudaEvent_t start = nullptr, in[2] = {}, done[2] = {}, out[2] = {};
+};
+
+int copy_lanes(int device, CopyLanes** out) {
+  static std::mutex mu;
+  static CopyLanes lanes[kMaxDevices];
+  static bool ready[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  CopyLanes& l = lanes[device];
+  if (!ready[device]) {
+    cudaError_t e = cudaStreamCreateWithFlags(&l.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&l.down, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&l.start, &l.in[0], &l.in[1], &l.done[0], &l.done[1], &l.out[0],
+                          &l.out[1]};
+    for (cudaEvent_t* ev : evs)
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess)
+      return set_error(H3B_ECUDA, "denoise_host_pipelined: stream/event creation: %s",
+                       cudaGetErrorString(e));
+    ready[device] = true;
+  }
+  *out = &l;
   return 0;
 }
 
