@@ -30,6 +30,7 @@ namespace h3b {
 namespace {
 
 constexpr int kBM = 128;
+constexpr int kTransBN = 160;  // token tile of the transposed pair kernel
 constexpr int kTileBytesK = 128;  // bytes of K per smem tile row (one swizzle span)
 constexpr int kGroupM = 16;
 
@@ -45,6 +46,7 @@ struct GemmCfg {
 
 struct GemmParams {
   int M, N, k_blocks, m_tiles, n_tiles;
+  int tokens;  // transposed pair kernel: output rows (the B operand's rows); else unused
   // Stream-K: the tiles x k_blocks iterations are cut into one equal contiguous range per
   // scheduling unit (CTA or CTA pair).  Each unit walks its range backwards, tile by tile
   // (k-blocks inside a tile still run forwards), so the partial tile at the end of its
@@ -355,6 +357,38 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
   }
 }
 
+// Epilogue of the transposed pair kernel (A = weights, B = activations, so the TMEM lane
+// is an output feature and the column a token).  For each 32-token chunk the warp turns
+// its 32 features x 32 tokens around in its own 4 KB of shared memory (rotated columns:
+// conflict-free both ways), after which lane L owns token L's 32 consecutive features and
+// runs the same row epilogue as the untransposed kernel.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_t tbase,
+                                                    int lane, int feat0, int tok0,
+                                                    float* stage) {
+  constexpr int NC = BN / 32;
+  RowIn in[2];
+  if (tok0 + lane < p.tokens) load_row_in<EPI>(p.epi, tok0 + lane, feat0, in[0]);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    const int tok_next = tok0 + (c + 1) * 32 + lane;
+    if (c + 1 < NC && tok_next < p.tokens)
+      load_row_in<EPI>(p.epi, tok_next, feat0, in[(c + 1) & 1]);
+    tmem_wait_ld(r);
+#pragma unroll
+    for (int t = 0; t < 32; ++t) stage[t * 32 + ((lane + t) & 31)] = __uint_as_float(r[t]);
+    __syncwarp();
+    uint32_t v[32];
+#pragma unroll
+    for (int f = 0; f < 32; ++f) v[f] = __float_as_uint(stage[lane * 32 + ((f + lane) & 31)]);
+    __syncwarp();
+    const int tok = tok0 + c * 32 + lane;
+    if (tok < p.tokens) epilogue_chunk<EPI>(p.epi, tok, feat0, v, in[c & 1]);
+  }
+}
+
 template <int BN, bool INT8, int EPI>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -574,20 +608,23 @@ __global__ void __launch_bounds__(192, 1)
 #ifndef H3B_PAIR_STAGES
 #define H3B_PAIR_STAGES 6
 #endif
-template <int BN>
+template <int BN, bool TRANS = false>
 struct PairCfg {
-  static constexpr int kStages = BN == 256 ? H3B_PAIR_STAGES : 8;
+  static constexpr int kStages = BN == 256 ? H3B_PAIR_STAGES : BN == 160 ? 7 : 8;
   static constexpr uint32_t kABytes = 128 * kTileBytesK;       // this CTA's 128 rows of A
   static constexpr uint32_t kBBytes = (BN / 2) * kTileBytesK;  // this CTA's half of B
-  static constexpr uint32_t kTmemCols = 2 * BN;
-  static constexpr size_t kSmem = 1024 + size_t(kStages) * (kABytes + kBBytes) + 256;
+  static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;  // two accumulators
+  // transposed epilogue: a 32 x 32 fp32 staging block per epilogue warp
+  static constexpr uint32_t kStageOut = TRANS ? 4 * 32 * 32 * 4 : 0;
+  static constexpr size_t kSmem =
+      1024 + size_t(kStages) * (kABytes + kBBytes) + kStageOut + 256;
 };
 
-template <int BN, bool INT8, int EPI>
+template <int BN, bool INT8, int EPI, bool TRANS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
-  using Cfg = PairCfg<BN>;
+  using Cfg = PairCfg<BN, TRANS>;
   constexpr int STAGES = Cfg::kStages;
   constexpr uint32_t HA = Cfg::kABytes;
   constexpr uint32_t HB = Cfg::kBBytes;
@@ -601,7 +638,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * HA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB);
+  float* sOut = reinterpret_cast<float*>(sB + STAGES * HB);  // transposed epilogue staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB + Cfg::kStageOut);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -782,8 +820,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           ok = __all_sync(0xffffffffu, seen);
         }
       }
-      epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo, pair, 2,
-                                   static_cast<int>(rank));
+      if constexpr (TRANS)
+        epilogue_unit_trans<BN, EPI>(p, tbase, lane, mb * 256 + static_cast<int>(rank) * 128 +
+                                     quarter * 32, nb * BN, sOut + quarter * 1024);
+      else
+        epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo, pair, 2,
+                                     static_cast<int>(rank));
       __syncwarp();
       if (lane == 0)
         for (int src = c_lo; src < pair; ++src)
@@ -894,7 +936,7 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
 }
 
 // Largest number of CTA pairs of the pair kernel that can be resident at once.
-template <int BN, bool INT8, int EPI>
+template <int BN, bool INT8, int EPI, bool TRANS = false>
 int pair_capacity(const DevCtx& ctx) {
   static std::atomic<int> cap[64];
   const int dev = ctx.device & 63;
@@ -903,9 +945,10 @@ int pair_capacity(const DevCtx& ctx) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (ctx.num_sms / 2));
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = PairCfg<BN>::kSmem;
+  cfg.dynamicSmemBytes = PairCfg<BN, TRANS>::kSmem;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<BN, INT8, EPI>, &cfg) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<BN, INT8, EPI, TRANS>, &cfg) !=
+          cudaSuccess ||
       n <= 0) {
     cudaGetLastError();
     n = 0;
@@ -921,7 +964,7 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
                 const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                 cudaStream_t stream, int* rc) {
   using Cfg = PairCfg<BN>;
-  auto kernel = k_gemm_pair<BN, INT8, EPI>;
+  auto kernel = k_gemm_pair<BN, INT8, EPI, false>;
   static std::atomic<uint32_t> attr_done{0};
   const uint32_t bit = 1u << (ctx.device & 31);
   if (!(attr_done.load() & bit)) {
@@ -978,6 +1021,54 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   }
   kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
   *rc = check_launch("gemm_pair");
+  return 0;
+}
+
+// Transposed CTA-pair GEMM, out[M, N] = X[M, K] W[N, K]^T computed as W X^T: the weight
+// rows fill the 256-row MMA side and the M activation rows (tokens) the 160-wide N side,
+// so a token count that is not a multiple of 256 wastes little (1,600 = 10 x 160).
+// Data-parallel only.  Returns 1 if the kernel cannot run here.
+template <int EPI>
+int launch_pair_trans(const DevCtx& ctx, const bf16* X, const bf16* W, int M, int N, int K,
+                      const GemmEpilogue& epi, cudaStream_t stream, int* rc) {
+  constexpr int BN = kTransBN;
+  using Cfg = PairCfg<BN, true>;
+  auto kernel = k_gemm_pair<BN, false, EPI, true>;
+  static std::atomic<uint32_t> attr_done{0};
+  const uint32_t bit = 1u << (ctx.device & 31);
+  if (!(attr_done.load() & bit)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Cfg::kSmem)) != cudaSuccess) {
+      cudaGetLastError();
+      return 1;
+    }
+    attr_done.fetch_or(bit);
+  }
+  const int cap = pair_capacity<BN, false, EPI, true>(ctx);
+  if (cap <= 0) return 1;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint64_t(N), uint64_t(K),
+                    uint64_t(K) * 2, 128, 64) ||
+      !make_tmap_2d(&tb, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint64_t(M), uint64_t(K),
+                    uint64_t(K) * 2, BN / 2, 64)) {
+    *rc = set_error(-3, "gemm: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+    return 0;
+  }
+  GemmParams p{};
+  p.M = N;
+  p.N = M;
+  p.tokens = M;
+  p.k_blocks = K / 64;
+  p.m_tiles = N / 256;
+  p.n_tiles = (M + BN - 1) / BN;
+  p.epi = epi;
+  p.err = ctx.err_flag;
+  const int tiles = p.m_tiles * p.n_tiles;
+  if (trace_gemm())
+    std::fprintf(stderr, "h3b gemm pair transposed BN=%d M=%d N=%d K=%d tiles=%d cap=%d\n", BN,
+                 M, N, K, tiles, cap);
+  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  *rc = check_launch("gemm_pair_trans");
   return 0;
 }
 
@@ -1066,11 +1157,58 @@ bool try_pair_bf16(int bn, const DevCtx& ctx, const bf16* A, const bf16* B, int 
   return launch_pair<128, false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
 }
 
+// H3B_GEMM_TRANS=0|1 forbids or forces the transposed pair kernel where the shape allows
+// it (diagnostics and measurements only).
+int forced_trans() {
+  static const int forced = [] {
+    const char* v = std::getenv("H3B_GEMM_TRANS");
+    if (!v || !v[0]) return -1;
+    return v[0] == '1' ? 1 : 0;
+  }();
+  return forced;
+}
+
+// Transposed (tokens on the 160-wide side) or not, from the same cost reasoning as the
+// stream-K choice, in units of one 256 x 256 tile on one CTA pair: the untransposed
+// kernel's best schedule against ceil(tiles / pairs) waves of 160 / 256 of a tile, times
+// kTransCost for the narrower tile's lower efficiency.  Measured on B200 (CUDA graphs of
+// 20 launches): the 160-wide tile does ~1.5x the time per FLOP of the 256-wide one, so the
+// transposed kernel is picked only where it wins: the out-projection at 1,600 tokens
+// (42.1 vs 44.7 us) and 832 tokens (28.0 vs 30.2 us); QKV, FC1 and FC2 stay untransposed.
+constexpr double kTransCost = 1.5;
+
+bool want_trans(const DevCtx& ctx, int M, int N, int K, bool sk_possible) {
+  if (N % 256 != 0 || M < kTransBN || forced_tile() != kAuto) return false;
+  if (forced_trans() >= 0) return forced_trans() == 1;
+  const int pairs = std::max(1, ctx.num_sms / 2);
+  const double kb = K / 64;
+  const int tiles_n = ((M + 255) / 256) * (N / 256);
+  double best_n = double((tiles_n + pairs - 1) / pairs);
+  if (sk_possible) best_n = std::min(best_n, (1.24 * tiles_n * kb / pairs + 23.0) / kb);
+  const int tiles_t = (N / 256) * ((M + kTransBN - 1) / kTransBN);
+  const double t = double((tiles_t + pairs - 1) / pairs) * kTransBN / 256.0 * kTransCost;
+  return t < best_n;
+}
+
 int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
                      const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream) {
   if (M <= 0) return 0;
   const int tile = choose_tile(M, N);
+  if (tile == kPair256 &&
+      want_trans(ctx, M, N, K, scratch != nullptr && scratch_bytes >= kScratchBytes)) {
+    int rc = 0, r = 1;
+    switch (epi.kind) {
+      case kEpiBias: r = launch_pair_trans<kEpiBias>(ctx, A, B, M, N, K, epi, stream, &rc); break;
+      case kEpiGelu: r = launch_pair_trans<kEpiGelu>(ctx, A, B, M, N, K, epi, stream, &rc); break;
+      case kEpiRope: r = launch_pair_trans<kEpiRope>(ctx, A, B, M, N, K, epi, stream, &rc); break;
+      case kEpiGateResid:
+        r = launch_pair_trans<kEpiGateResid>(ctx, A, B, M, N, K, epi, stream, &rc);
+        break;
+      default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
+    }
+    if (r == 0) return rc;
+  }
   if (tile == kPair256 || tile == kPair128) {
     const int bn = tile == kPair256 ? 256 : 128;
     int rc = 0;
