@@ -103,6 +103,37 @@ def test_pipelined_host_entry_matches_device_runs(name, requests):
         assert torch.equal(host_out[r], want[r]), f"request {r}"
 
 
+def test_host_entries_without_graphs_match_device_runs():
+    # H3B_DEBUG=1 makes the host entry points launch the steps directly (no cached graph)
+    # and check every launch; run in a child process, since the switch is read once
+    import subprocess
+    import sys
+    code = (
+        "import torch\n"
+        "from video_diffusion_transformer_03_b200 import synth, h3b\n"
+        "from video_diffusion_transformer_03_b200.pipeline import DiTDenoiser\n"
+        "cfg = synth.CONFIGS['tiny']\n"
+        "m = DiTDenoiser(cfg)\n"
+        "g = torch.Generator().manual_seed(9)\n"
+        "x0 = torch.randn((3, cfg.n_tokens, cfg.d), generator=g).to(torch.bfloat16).float()\n"
+        "want = []\n"
+        "for r in range(3):\n"
+        "    xd = x0[r].to('cuda'); m.run(xd); want.append(xd.cpu())\n"
+        "h3b.sync_status()\n"
+        "hi, ho = x0.pin_memory(), torch.empty_like(x0).pin_memory()\n"
+        "m.run_host_pipelined(hi, ho, torch.empty((2, cfg.n_tokens, cfg.d), device='cuda'))\n"
+        "one = torch.empty_like(x0[0]).pin_memory()\n"
+        "m.run_host(x0[1].pin_memory(), one, torch.empty_like(x0[0], device='cuda'))\n"
+        "assert all(torch.equal(ho[r], want[r]) for r in range(3))\n"
+        "assert torch.equal(one, want[1])\n"
+        "print('ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, H3B_DEBUG="1", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=600, cwd=root)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
 def test_768x1344_full_denoise_is_finite_and_deterministic():
     cfg = synth.CONFIGS["dit768x1344"]
     m = DiTDenoiser(cfg, gen_device="cuda")
