@@ -357,25 +357,239 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
   }
 }
 
-// Epilogue of the transposed pair kernel (A = weights, B = activations, so the TMEM lane
-// is an output feature and the column a token).  For each 32-token chunk the warp turns
-// its 32 features x 32 tokens around in its own 4 KB of shared memory (rotated columns:
-// conflict-free both ways), after which lane L owns token L's 32 consecutive features and
-// runs the same row epilogue as the untransposed kernel.
-template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_t tbase,
-                                                    int lane, int feat0, int tok0,
-                                                    float* stage) {
+// ---------------------------------------------------------------- staged pair epilogue
+// Each epilogue warp of the pair kernels owns kWarpStage bytes of shared memory: a 4 KB
+// block through which a 32 x 32 chunk passes between the row-per-lane form of the TMEM
+// accumulator and the coalesced form of global memory, and the tile's column vectors as
+// fp32, which all lanes read at the same address.  With one row per lane a warp-wide
+// 16-byte access touches 32 cache lines; through the block it touches 8 (bf16 rows of 64
+// bytes) or 4 (fp32 rows of 128 bytes), and the vectors cost one global round trip per
+// tile, issued while the warp waits for the accumulator, instead of one per chunk.
+constexpr int kVecLen = 256;                               // widest tile
+constexpr uint32_t kWarpStage = 4096 + 3 * kVecLen * 4;   // block + 3 vectors
+constexpr int kVecBias = 0, kVecGate = kVecLen, kVecScale = 2 * kVecLen;
+
+// 16-byte piece j of row r of a 32 x 32 block: bf16 rows hold 4 pieces, fp32 rows 8.  The
+// XOR keeps both access forms (one row per lane; 8 or 4 whole rows per instruction) free of
+// bank conflicts within each quarter warp.
+__device__ __forceinline__ int blk16(int r, int j) { return r * 4 + (j ^ ((r >> 1) & 3)); }
+__device__ __forceinline__ int blk32(int r, int j) { return r * 8 + (j ^ (r & 7)); }
+
+// The NV column vectors starting at col0 into vec (fp32): bias (int8: the fp32 bias, zero
+// when absent), gate, int8 column scales.
+template <int EPI, int NV>
+__device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, float* vec,
+                                              int lane) {
+#pragma unroll
+  for (int k = 0; k < NV / 32; ++k) {
+    const int i = k * 32 + lane;
+    const int col = col0 + i;
+    if constexpr (EPI == kEpiInt8Deq) {
+      vec[kVecBias + i] = e.bias_f32 ? __ldg(e.bias_f32 + col) : 0.0f;
+      vec[kVecScale + i] = __ldg(e.col_scale + col);
+    } else {
+      const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(e.bias) + col);
+      vec[kVecBias + i] = __uint_as_float(b << 16);
+    }
+    if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq)
+      vec[kVecGate + i] = __ldg(e.gate + col);
+  }
+}
+
+// Global inputs of the 32 x 32 chunk (rows row0 + [0, nrows), columns col + [0, 32)) in
+// coalesced form: residual pieces (row k * 8 + lane / 4, piece lane % 4) and RoPE (cos, sin)
+// pieces (row k * 4 + lane / 8, piece lane % 8).
+template <int EPI>
+__device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, int nrows,
+                                              int col, int lane, RowIn& in) {
+  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = k * 8 + (lane >> 2);
+      in.res[k] = r < nrows ? *reinterpret_cast<const uint4*>(
+                                  e.out + size_t(row0 + r) * e.ld_out + col + (lane & 3) * 8)
+                            : make_uint4(0u, 0u, 0u, 0u);  // coherent: this kernel rewrites it
+    }
+  }
+  if constexpr (EPI == kEpiRope) {
+    if (col < e.rope_cols) {
+      const int half = e.head_dim >> 1;
+      const int pair0 = (col % e.head_dim) >> 1;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int r = k * 4 + (lane >> 3);
+        in.cs[k] = r < nrows ? __ldg(reinterpret_cast<const float4*>(
+                                         e.rope_cs + (size_t(row0 + r) * half + pair0) * 2) +
+                                     (lane & 7))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+}
+
+// Epilogue of one 32 x 32 chunk held one row per lane (lane L: row row0 + L, columns col +
+// [0, 32)); vec points at the chunk's first column in the staged vectors.
+template <int EPI>
+__device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, int nrows,
+                                               int col, const uint32_t (&r)[32],
+                                               const RowIn& in, uint4* blk, const float* vec,
+                                               int lane) {
+  const bool valid = lane < nrows;
+  float v[32];
+  if constexpr (EPI == kEpiInt8Deq) {
+    const float rs = valid ? __ldg(e.row_scale + row0 + lane) : 0.0f;
+    if (e.acc_out && valid) {
+      int4* dst = reinterpret_cast<int4*>(e.acc_out + size_t(row0 + lane) * e.ld_out + col);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        dst[i] = make_int4(int(r[4 * i]), int(r[4 * i + 1]), int(r[4 * i + 2]),
+                           int(r[4 * i + 3]));
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), rs),
+                       vec[kVecScale + j]);
+    if (e.bias_f32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += vec[kVecBias + j];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + vec[kVecBias + j];
+  }
+  if constexpr (EPI == kEpiGelu) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+  }
+  if constexpr (EPI == kEpiRope) {
+    if (col < e.rope_cols) {
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 c = in.cs[k];
+        blk[blk32(k * 4 + (lane >> 3), lane & 7)] =
+            make_uint4(__float_as_uint(c.x), __float_as_uint(c.y), __float_as_uint(c.z),
+                       __float_as_uint(c.w));
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {  // 2 pairs per piece (cos0, sin0, cos1, sin1)
+        const uint4 u = blk[blk32(lane, i)];
+        const float cx = __uint_as_float(u.x), sx = __uint_as_float(u.y);
+        const float cy = __uint_as_float(u.z), sy = __uint_as_float(u.w);
+        const float x0 = v[4 * i], x1 = v[4 * i + 1], y0 = v[4 * i + 2], y1 = v[4 * i + 3];
+        v[4 * i + 0] = x0 * cx - x1 * sx;
+        v[4 * i + 1] = x0 * sx + x1 * cx;
+        v[4 * i + 2] = y0 * cy - y1 * sy;
+        v[4 * i + 3] = y0 * sy + y1 * cy;
+      }
+    }
+  }
+  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) blk[blk16(k * 8 + (lane >> 2), lane & 3)] = in.res[k];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = blk[blk16(lane, i)];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 rr = unpack_bf16x2(w[k]);
+        v[8 * i + 2 * k] = fmaf(vec[kVecGate + 8 * i + 2 * k], v[8 * i + 2 * k], rr.x);
+        v[8 * i + 2 * k + 1] =
+            fmaf(vec[kVecGate + 8 * i + 2 * k + 1], v[8 * i + 2 * k + 1], rr.y);
+      }
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    blk[blk16(lane, i)] =
+        make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                   pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int rr = k * 8 + (lane >> 2);
+    if (rr < nrows)
+      *reinterpret_cast<uint4*>(e.out + size_t(row0 + rr) * e.ld_out + col + (lane & 3) * 8) =
+          blk[blk16(rr, lane & 3)];
+  }
+  __syncwarp();  // the block is free for the next chunk
+}
+
+// Epilogue of one 128-row half tile of the pair kernel, this warp's 32 rows (row0 + lane):
+// accumulator from TMEM, plus the partial tiles parked by units [src_lo, src_hi) (slot
+// src * stride + off), then the staged epilogue chunk by chunk.  The next chunk's global
+// inputs and first partial are fetched while the current chunk is finished.
+template <int BN, bool INT8, int EPI>
+__device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t tbase,
+                                                   int row0, int row_in_tile, int col0,
+                                                   int src_lo, int src_hi, int stride,
+                                                   int off, uint4* blk, const float* vec,
+                                                   int lane) {
   constexpr int NC = BN / 32;
+  const int nrows = p.M - row0;
+  const bool has_part = src_lo < src_hi;
+  const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
   RowIn in[2];
-  if (tok0 + lane < p.tokens) load_row_in<EPI>(p.epi, tok0 + lane, feat0, in[0]);
+  uint4 part[2][8];
+  load_block_in<EPI>(p.epi, row0, nrows, col0, lane, in[0]);
+  if (has_part) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[0][i] = __ldcg(first + size_t(i) * kBM);
+  }
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
-    const int tok_next = tok0 + (c + 1) * 32 + lane;
-    if (c + 1 < NC && tok_next < p.tokens)
-      load_row_in<EPI>(p.epi, tok_next, feat0, in[(c + 1) & 1]);
+    if (c + 1 < NC) {
+      load_block_in<EPI>(p.epi, row0, nrows, col0 + (c + 1) * 32, lane, in[(c + 1) & 1]);
+      if (has_part) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          part[(c + 1) & 1][i] = __ldcg(first + size_t((c + 1) * 8 + i) * kBM);
+      }
+    }
+    tmem_wait_ld(r);
+    if (has_part) {
+      add_part<INT8>(r, part[c & 1]);
+      for (int src = src_lo + 1; src < src_hi; ++src) {
+        const uint4* ps = sk_slot<BN>(p, src * stride + off) + row_in_tile;
+        uint4 more[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) more[i] = __ldcg(ps + size_t(c * 8 + i) * kBM);
+        add_part<INT8>(r, more);
+      }
+    }
+    epilogue_block<EPI>(p.epi, row0, nrows, col0 + c * 32, r, in[c & 1], blk, vec + c * 32,
+                        lane);
+  }
+}
+
+// Epilogue of the transposed pair kernel (A = weights, B = activations, so the TMEM lane
+// is an output feature and the column a token).  For each 32-token chunk the warp turns
+// its 32 features x 32 tokens around in its block (rotated columns: conflict-free both
+// ways), after which lane L owns token L's 32 consecutive features and the chunk takes the
+// same staged epilogue as the untransposed kernel.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_t tbase,
+                                                    int lane, int feat0, int tok0, uint4* blk,
+                                                    const float* vec) {
+  constexpr int NC = BN / 32;
+  float* stage = reinterpret_cast<float*>(blk);
+  RowIn in[2];
+  load_block_in<EPI>(p.epi, tok0, p.tokens - tok0, feat0, lane, in[0]);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    const int row0 = tok0 + c * 32;
+    if (c + 1 < NC)
+      load_block_in<EPI>(p.epi, row0 + 32, p.tokens - row0 - 32, feat0, lane,
+                         in[(c + 1) & 1]);
     tmem_wait_ld(r);
 #pragma unroll
     for (int t = 0; t < 32; ++t) stage[t * 32 + ((lane + t) & 31)] = __uint_as_float(r[t]);
@@ -383,9 +597,7 @@ __device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_
     uint32_t v[32];
 #pragma unroll
     for (int f = 0; f < 32; ++f) v[f] = __float_as_uint(stage[lane * 32 + ((f + lane) & 31)]);
-    __syncwarp();
-    const int tok = tok0 + c * 32 + lane;
-    if (tok < p.tokens) epilogue_chunk<EPI>(p.epi, tok, feat0, v, in[c & 1]);
+    epilogue_block<EPI>(p.epi, row0, p.tokens - row0, feat0, v, in[c & 1], blk, vec, lane);
   }
 }
 
@@ -614,10 +826,10 @@ struct PairCfg {
   static constexpr uint32_t kABytes = 128 * kTileBytesK;       // this CTA's 128 rows of A
   static constexpr uint32_t kBBytes = (BN / 2) * kTileBytesK;  // this CTA's half of B
   static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;  // two accumulators
-  // transposed epilogue: a 32 x 32 fp32 staging block per epilogue warp
-  static constexpr uint32_t kStageOut = TRANS ? 4 * 32 * 32 * 4 : 0;
+  static constexpr uint32_t kStageOut = 4 * kWarpStage;  // the 4 epilogue warps' staging
   static constexpr size_t kSmem =
       1024 + size_t(kStages) * (kABytes + kBBytes) + kStageOut + 256;
+  static_assert(kSmem <= 232448, "pair kernel shared memory above the 227 KB limit");
 };
 
 template <int BN, bool INT8, int EPI, bool TRANS>
@@ -638,7 +850,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * HA;
-  float* sOut = reinterpret_cast<float*>(sB + STAGES * HB);  // transposed epilogue staging
+  uint8_t* sEpi = sB + STAGES * HB;  // epilogue staging, kWarpStage per epilogue warp
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB + Cfg::kStageOut);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -770,6 +982,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int slot_id = pair * 2 + static_cast<int>(rank);
+    uint4* blk = reinterpret_cast<uint4*>(sEpi + quarter * kWarpStage);
+    float* vec = reinterpret_cast<float*>(sEpi + quarter * kWarpStage + 4096);
     int local = 0;
     Sched sc;
     sched_init(p, sc, pair, npairs);
@@ -779,6 +993,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
+      // the tile's column vectors, fetched while the accumulator is being computed
+      if constexpr (TRANS)
+        stage_vectors<EPI, 32>(p.epi, mb * 256 + static_cast<int>(rank) * 128 + quarter * 32,
+                               vec, lane);
+      else
+        stage_vectors<EPI, BN>(p.epi, nb * BN, vec, lane);
       bool ok = wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -820,12 +1040,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           ok = __all_sync(0xffffffffu, seen);
         }
       }
+      __syncwarp();  // staged vectors visible to every lane
       if constexpr (TRANS)
         epilogue_unit_trans<BN, EPI>(p, tbase, lane, mb * 256 + static_cast<int>(rank) * 128 +
-                                     quarter * 32, nb * BN, sOut + quarter * 1024);
+                                     quarter * 32, nb * BN, blk, vec);
       else
-        epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo, pair, 2,
-                                     static_cast<int>(rank));
+        epilogue_unit_pair<BN, INT8, EPI>(p, tbase, row - lane, row_in_tile, nb * BN, c_lo,
+                                          pair, 2, static_cast<int>(rank), blk, vec, lane);
       __syncwarp();
       if (lane == 0)
         for (int src = c_lo; src < pair; ++src)
