@@ -73,6 +73,47 @@ def test_gemm_epilogues(M, N, K, epi, sk):
     assert torch.equal(again, out)
 
 
+def test_gemm_hybrid_stream_k_schedule():
+    # The CTA-pair kernel splits only its last one to two tiles per pair stream-K and runs
+    # the whole waves before them data-parallel; the cost model picks that form only where
+    # it wins, so force it (H3B_GEMM_SCHED is read once per process: run a child) on shapes
+    # with a data-parallel phase, partial tiles and a ragged last row tile.
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, torch\n"
+        "from oracle import oracle as O\n"
+        "from tests.helpers import max_block_rel_l2, np64, rel_l2, rnd\n"
+        "from video_diffusion_transformer_03_b200 import h3b\n"
+        "ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device='cuda')\n"
+        "for (M, N, K, epi) in [(1000, 9728, 512, h3b.EPI_GATE_RESID),\n"
+        "                       (1600, 12288, 3072, h3b.EPI_BIAS_GELU)]:\n"
+        "    A = rnd((M, K), 1.0, seed=11); B = rnd((N, K), K ** -0.5, seed=12)\n"
+        "    bias = rnd((N,), 0.1, seed=13)\n"
+        "    acc = np64(A) @ np64(B).T + np64(bias)\n"
+        "    out = torch.empty((M, N), dtype=torch.bfloat16, device='cuda'); gate = None\n"
+        "    if epi == h3b.EPI_GATE_RESID:\n"
+        "        resid = rnd((M, N), 1.0, seed=14); g = rnd((N,), 0.5, seed=15, dtype=torch.float32)\n"
+        "        out.copy_(resid.to('cuda')); gate = g.to('cuda')\n"
+        "        want = O.gated_residual(np64(resid), np64(g), acc)\n"
+        "    else:\n"
+        "        want = O.gelu_tanh(acc)\n"
+        "    h3b.gemm_bf16(A.cuda(), B.cuda(), epi, bias.cuda(), out, gate=gate, ws=ws)\n"
+        "    h3b.sync_status()\n"
+        "    got = np64(out)\n"
+        "    assert rel_l2(got, want) < 4e-3 and max_block_rel_l2(got, want) < 8e-3, (M, N, K)\n"
+        "print('ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, H3B_GEMM_SCHED="sk", H3B_GEMM_TRANS="0", H3B_TRACE_GEMM="1",
+               PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=600, cwd=root)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+    # the launches took the hybrid form: a data-parallel phase before the split tiles
+    assert "sk_tile0=74" in r.stderr and "sk_tile0=222" in r.stderr, r.stderr
+
+
 @pytest.mark.parametrize("grid,n_audio,heads,hd,split", [
     ((2, 4, 4), 8, 4, 64, (16, 24, 24)),
     ((6, 16, 16), 64, 24, 128, (32, 48, 48)),

@@ -47,15 +47,17 @@ struct GemmCfg {
 struct GemmParams {
   int M, N, k_blocks, m_tiles, n_tiles;
   int tokens;  // transposed pair kernel: output rows (the B operand's rows); else unused
-  // Stream-K: the tiles x k_blocks iterations are cut into one equal contiguous range per
-  // scheduling unit (CTA or CTA pair).  Each unit walks its range backwards, tile by tile
-  // (k-blocks inside a tile still run forwards), so the partial tile at the end of its
-  // range is computed first: the unit stores it in its slot and publishes sk_seq in its
-  // flag.  The unit holding the tile's last k-block reaches that tile last and adds the
-  // slots of the lower-numbered units that computed the rest of it: waits only ever point
-  // at lower-numbered units, which are dispatched first.
+  // Stream-K: the iterations (tile, k-block) of tiles [sk_tile0, tiles) are cut into one
+  // equal contiguous range per scheduling unit (CTA or CTA pair).  Each unit walks its
+  // range backwards, tile by tile (k-blocks inside a tile still run forwards), so the
+  // partial tile at the end of its range is computed first: the unit stores it in its slot
+  // and publishes sk_seq in its flag.  The unit holding the tile's last k-block reaches
+  // that tile last and adds the slots of the lower-numbered units that computed the rest
+  // of it: waits only ever point at lower-numbered units, which are dispatched first.
+  // Tiles [0, sk_tile0), whole waves of one tile per unit, then run data-parallel.
   int sk;
-  long long sk_iters;
+  int sk_tile0;
+  long long sk_iters;  // (tiles - sk_tile0) x k_blocks
   uint32_t* sk_slots;            // [gridDim.x][BN / 4][128] uint4 of raw accumulator words
   unsigned long long* sk_flags;  // [gridDim.x][4]
   unsigned long long sk_seq;
@@ -76,7 +78,7 @@ __device__ __forceinline__ long long sk_begin(const GemmParams& p, int c, int co
   return p.sk_iters * c / count;
 }
 
-// Unit whose range contains iteration i.
+// Unit whose range contains iteration i (counted from the first stream-K tile).
 __device__ __forceinline__ int sk_owner(const GemmParams& p, long long i, int count) {
   int c = static_cast<int>(i * count / p.sk_iters);
   while (c + 1 < count && sk_begin(p, c + 1, count) <= i) ++c;
@@ -86,34 +88,37 @@ __device__ __forceinline__ int sk_owner(const GemmParams& p, long long i, int co
 
 // Work items of this unit: (tile, k-block range).  Every role walks the same sequence.
 struct Sched {
-  long long it, it_end;  // stream-K
-  int tile;              // data-parallel
+  long long it, it_end;  // stream-K phase
+  int tile, dp_end;      // data-parallel phase: tiles me, me + count, ... below dp_end
   int count;
 };
 
 __device__ __forceinline__ void sched_init(const GemmParams& p, Sched& s, int me, int count) {
   s.count = count;
+  s.tile = me;
   if (p.sk) {
     s.it = sk_begin(p, me, count);
     s.it_end = sk_begin(p, me + 1, count);
+    s.dp_end = p.sk_tile0;
   } else {
-    s.tile = me;
+    s.it = s.it_end = 0;
+    s.dp_end = p.m_tiles * p.n_tiles;
   }
 }
 
 __device__ __forceinline__ bool sched_next(const GemmParams& p, Sched& s, int& tile, int& kb0,
                                            int& kb1) {
-  if (p.sk) {  // backwards over the range [it, it_end): it_end moves down
-    if (s.it_end <= s.it) return false;
-    tile = static_cast<int>((s.it_end - 1) / p.k_blocks);
-    const long long t0 = static_cast<long long>(tile) * p.k_blocks;
+  if (s.it_end > s.it) {  // stream-K: backwards over [it, it_end), it_end moves down
+    const int rel = static_cast<int>((s.it_end - 1) / p.k_blocks);
+    const long long t0 = static_cast<long long>(rel) * p.k_blocks;
     const long long start = s.it > t0 ? s.it : t0;
+    tile = p.sk_tile0 + rel;
     kb0 = static_cast<int>(start - t0);
     kb1 = static_cast<int>(s.it_end - t0);
     s.it_end = start;
     return true;
   }
-  if (s.tile >= p.m_tiles * p.n_tiles) return false;
+  if (s.tile >= s.dp_end) return false;
   tile = s.tile;
   kb0 = 0;
   kb1 = p.k_blocks;
@@ -769,7 +774,7 @@ __global__ void __launch_bounds__(192, 1)
       // tile owner: add the partials of the CTAs that computed the rest of this tile
       int c_lo = static_cast<int>(blockIdx.x);
       if (kb0 > 0) {
-        c_lo = sk_owner(p, static_cast<long long>(tile) * p.k_blocks, gridDim.x);
+        c_lo = sk_owner(p, static_cast<long long>(tile - p.sk_tile0) * p.k_blocks, gridDim.x);
         for (int c = c_lo; c < static_cast<int>(blockIdx.x) && ok; ++c) {
           const unsigned long long* f = p.sk_flags + c * 4 + quarter;
           bool seen = ld_acquire_u64(f) == p.sk_seq;
@@ -1022,7 +1027,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       int c_lo = pair;
       if (kb0 > 0) {
-        c_lo = sk_owner(p, static_cast<long long>(tile) * p.k_blocks, npairs);
+        c_lo = sk_owner(p, static_cast<long long>(tile - p.sk_tile0) * p.k_blocks, npairs);
         for (int c = c_lo; c < pair && ok; ++c) {
           const unsigned long long* f = p.sk_flags + (c * 2 + static_cast<int>(rank)) * 4 + quarter;
           bool seen = ld_acquire_u64(f) == p.sk_seq;
@@ -1084,16 +1089,26 @@ unsigned long long next_sk_seq() {
   return salt + (g_sk_seq.fetch_add(1) << 1);
 }
 
-// Schedule choice from a cost model in units of one K slice of one tile on one scheduling
-// unit.  Data-parallel: ceil(tiles / units) waves of k_blocks slices.  Stream-K: the even
-// share tiles * k_blocks / units, times 1.24, plus 23 (partial-tile parking and merging,
-// the exposed epilogue of the merged tile).  The two constants fit the CTA-pair kernel on
-// B200 at M = 832 and 1600, N = 3072, K = 3072 and 12288 (stream-K / data-parallel time
-// 0.94, 1.28, 0.76, 0.94 measured; the model gives 0.94, 1.28, 0.76, 0.92).
-bool want_stream_k(int tiles, int units, int k_blocks) {
-  const double dp = double((tiles + units - 1) / units) * k_blocks;
-  const double sk = 1.24 * double(tiles) * k_blocks / units + 23.0;
-  return sk < dp;
+// First stream-K tile of the pair kernel's hybrid schedule: every whole wave of tiles but
+// the last runs data-parallel, so the split part holds between one and two tiles per unit.
+int hybrid_tile0(int tiles, int units) { return std::max(0, tiles / units - 1) * units; }
+
+// Schedule costs in units of one K slice of one tile on one scheduling unit.
+// Data-parallel: ceil(tiles / units) waves of k_blocks slices.  Stream-K over the tiles
+// from dp_tiles on: the whole waves before it, plus the even share of the split tiles
+// times 1.28, plus 17 (partial-tile parking and merging, the exposed epilogue of the merged
+// tile).  The constants fit the CTA-pair kernel on B200 (CUDA graphs of 20 launches) at
+// M = 832, 1600 and 11344 with the four block GEMM shapes of a 3072-wide model; the choice
+// they make was the faster schedule for all ten shapes measured.
+double dp_cost(int tiles, int units, int k_blocks) {
+  return double((tiles + units - 1) / units) * k_blocks;
+}
+double sk_cost(int tiles, int units, int k_blocks, int dp_tiles) {
+  return double(dp_tiles / units) * k_blocks +
+         1.28 * double(tiles - dp_tiles) * k_blocks / units + 17.0;
+}
+bool want_stream_k(int tiles, int units, int k_blocks, int dp_tiles = 0) {
+  return sk_cost(tiles, units, k_blocks, dp_tiles) < dp_cost(tiles, units, k_blocks);
 }
 
 template <int BN, bool INT8, int EPI>
@@ -1134,7 +1149,7 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
   const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
                      iters >= 4LL * sk_ctas;
-  const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() == 1
+  const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() >= 1
                                                     : want_stream_k(tiles, ctx.num_sms, p.k_blocks));
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm 1cta BN=%d M=%d N=%d K=%d tiles=%d sms=%d -> %s grid=%d\n", BN,
@@ -1218,18 +1233,23 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   p.err = ctx.err_flag;
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
-  const long long iters = static_cast<long long>(tiles) * p.k_blocks;
+  // hybrid: all whole waves but the last run data-parallel, the rest is split stream-K
+  const int sk_tile0 = forced_sched() == 2 ? 0 : hybrid_tile0(tiles, sk_pairs);
+  const long long iters = static_cast<long long>(tiles - sk_tile0) * p.k_blocks;
   const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
                      iters >= 4LL * sk_pairs;
-  const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() == 1
-                                                    : want_stream_k(tiles, cap, p.k_blocks));
+  const bool use_sk =
+      sk_ok && (forced_sched() >= 0 ? forced_sched() >= 1
+                                    : want_stream_k(tiles, sk_pairs, p.k_blocks, sk_tile0));
   if (trace_gemm())
-    std::fprintf(stderr, "h3b gemm pair BN=%d M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d\n",
+    std::fprintf(stderr,
+                 "h3b gemm pair BN=%d M=%d N=%d K=%d tiles=%d cap=%d -> %s pairs=%d sk_tile0=%d\n",
                  BN, M, N, K, tiles, cap, use_sk ? "stream-K" : "data-parallel",
-                 use_sk ? sk_pairs : std::min(tiles, cap));
+                 use_sk ? sk_pairs : std::min(tiles, cap), use_sk ? sk_tile0 : 0);
   if (use_sk) {
     GemmParams q = p;
     q.sk = 1;
+    q.sk_tile0 = sk_tile0;
     q.sk_iters = iters;
     q.sk_slots = static_cast<uint32_t*>(scratch);
     q.sk_flags =
@@ -1293,14 +1313,15 @@ int launch_pair_trans(const DevCtx& ctx, const bf16* X, const bf16* W, int M, in
   return 0;
 }
 
-// H3B_GEMM_SCHED=sk|dp forces the stream-K or the data-parallel schedule where the
+// H3B_GEMM_SCHED=sk|skall|dp forces the hybrid stream-K schedule (the pair kernel's
+// default form), stream-K over every tile, or the data-parallel schedule, where the
 // scratch allows it (diagnostics and measurements only).
 int forced_sched() {
   static const int forced = [] {
     const char* v = std::getenv("H3B_GEMM_SCHED");
     if (!v) return -1;
     const std::string t(v);
-    return t == "sk" ? 1 : t == "dp" ? 0 : -1;
+    return t == "skall" ? 2 : t == "sk" ? 1 : t == "dp" ? 0 : -1;
   }();
   return forced;
 }
@@ -1394,8 +1415,8 @@ int forced_trans() {
 // kernel's best schedule against ceil(tiles / pairs) waves of 160 / 256 of a tile, times
 // kTransCost for the narrower tile's lower efficiency.  Measured on B200 (CUDA graphs of
 // 20 launches): the 160-wide tile does ~1.5x the time per FLOP of the 256-wide one, so the
-// transposed kernel is picked only where it wins: the out-projection at 1,600 tokens
-// (42.1 vs 44.7 us) and 832 tokens (28.0 vs 30.2 us); QKV, FC1 and FC2 stay untransposed.
+// transposed kernel is picked only where it wins: the out-projection at 832 tokens (24.9
+// vs 25.5 us data-parallel); at 1,600 tokens stream-K does it in 36.9 us against 39.5.
 constexpr double kTransCost = 1.5;
 
 bool want_trans(const DevCtx& ctx, int M, int N, int K, bool sk_possible) {
@@ -1404,8 +1425,9 @@ bool want_trans(const DevCtx& ctx, int M, int N, int K, bool sk_possible) {
   const int pairs = std::max(1, ctx.num_sms / 2);
   const double kb = K / 64;
   const int tiles_n = ((M + 255) / 256) * (N / 256);
-  double best_n = double((tiles_n + pairs - 1) / pairs);
-  if (sk_possible) best_n = std::min(best_n, (1.24 * tiles_n * kb / pairs + 23.0) / kb);
+  double best_n = dp_cost(tiles_n, pairs, 1);
+  if (sk_possible)
+    best_n = std::min(best_n, sk_cost(tiles_n, pairs, K / 64, hybrid_tile0(tiles_n, pairs)) / kb);
   const int tiles_t = (N / 256) * ((M + kTransBN - 1) / kTransBN);
   const double t = double((tiles_t + pairs - 1) / pairs) * kTransBN / 256.0 * kTransCost;
   return t < best_n;
