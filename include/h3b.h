@@ -124,6 +124,23 @@ size_t h3b_gemm_workspace_size(void);
  * stream's buffers. */
 size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce);
 
+/* ---------------------------------------------------------------- diagnostics */
+/* The GEMM kernels' work schedule, computed on the host by the same functions the kernels
+ * run (no GPU, no CUDA call): the work items of scheduling unit `unit` (a CTA pair of the
+ * pair kernel, a CTA of the single-SM kernel) out of `units`, for `tiles` output tiles of
+ * `k_blocks` K slices each.  mode: 0 data-parallel; 1 hybrid stream-K (the pair kernel's
+ * form: whole waves but the last data-parallel, the rest split evenly); 2 stream-K over
+ * every tile (the single-SM kernel's form).  Item i goes to items[4 i .. 4 i + 3] (host,
+ * caller-owned) as (tile, first K slice, end K slice, merge), in processing order: merge
+ * is -1 for a partial tile the unit parks for a higher unit, else the first unit whose
+ * parked partial the item's epilogue adds (the unit itself when it adds none).  At most
+ * max_items items are written.  Returns the number of items, or H3B_EINVAL for
+ * non-positive sizes, a unit outside [0, units), a mode outside 0-2, a missing buffer, or
+ * a stream-K mode with fewer than 4 split K slices per unit (the GEMM calls run those
+ * shapes data-parallel). */
+int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, int* items,
+                      int max_items);
+
 /* ---------------------------------------------------------------- hot-path steps */
 /* AdaLN modulation vectors: mod[j] = sum_k w[j, k] c[k] + b[j], j < n_out.
  * w [n_out, c_dim] bf16, b [n_out] bf16, c [c_dim] bf16, mod [n_out] fp32 (all device).

@@ -74,12 +74,12 @@ static_assert(kSkFlagsOffset >= size_t(kMaxSkCtas) * kBM * 256 * 4,
 
 // Scheduling units are CTAs (single-SM kernel) or CTA pairs (pair kernel): `me` is this
 // unit's index and `count` the number of units in the grid.
-__device__ __forceinline__ long long sk_begin(const GemmParams& p, int c, int count) {
+__host__ __device__ __forceinline__ long long sk_begin(const GemmParams& p, int c, int count) {
   return p.sk_iters * c / count;
 }
 
 // Unit whose range contains iteration i (counted from the first stream-K tile).
-__device__ __forceinline__ int sk_owner(const GemmParams& p, long long i, int count) {
+__host__ __device__ __forceinline__ int sk_owner(const GemmParams& p, long long i, int count) {
   int c = static_cast<int>(i * count / p.sk_iters);
   while (c + 1 < count && sk_begin(p, c + 1, count) <= i) ++c;
   while (c > 0 && sk_begin(p, c, count) > i) --c;
@@ -93,7 +93,8 @@ struct Sched {
   int count;
 };
 
-__device__ __forceinline__ void sched_init(const GemmParams& p, Sched& s, int me, int count) {
+__host__ __device__ __forceinline__ void sched_init(const GemmParams& p, Sched& s, int me,
+                                                   int count) {
   s.count = count;
   s.tile = me;
   if (p.sk) {
@@ -106,8 +107,8 @@ __device__ __forceinline__ void sched_init(const GemmParams& p, Sched& s, int me
   }
 }
 
-__device__ __forceinline__ bool sched_next(const GemmParams& p, Sched& s, int& tile, int& kb0,
-                                           int& kb1) {
+__host__ __device__ __forceinline__ bool sched_next(const GemmParams& p, Sched& s, int& tile,
+                                                    int& kb0, int& kb1) {
   if (s.it_end > s.it) {  // stream-K: backwards over [it, it_end), it_end moves down
     const int rel = static_cast<int>((s.it_end - 1) / p.k_blocks);
     const long long t0 = static_cast<long long>(rel) * p.k_blocks;
@@ -1389,6 +1390,43 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
 }  // namespace
 
 size_t gemm_scratch_bytes() { return kScratchBytes; }
+
+// The work items of one scheduling unit, from the functions the kernels run: (tile, first
+// K slice, end K slice, merge) with merge = -1 for a partial tile the unit parks for a
+// higher unit, else the first unit whose parked partial the item's epilogue adds (the unit
+// itself when it adds none).  -1 for a stream-K schedule the launches never run (fewer
+// than 4 split K slices per unit: a unit with an empty range would leave its flag unset).
+int gemm_schedule_items(int tiles, int k_blocks, int units, int mode, int unit, int* items,
+                        int max_items) {
+  GemmParams p{};
+  p.k_blocks = k_blocks;
+  p.m_tiles = tiles;
+  p.n_tiles = 1;
+  if (mode != 0) {
+    p.sk = 1;
+    p.sk_tile0 = mode == 1 ? hybrid_tile0(tiles, units) : 0;
+    p.sk_iters = static_cast<long long>(tiles - p.sk_tile0) * k_blocks;
+    if (p.sk_iters < 4LL * units) return -1;
+  }
+  Sched sc;
+  sched_init(p, sc, unit, units);
+  int n = 0, tile, kb0, kb1;
+  while (sched_next(p, sc, tile, kb0, kb1)) {
+    int merge = unit;
+    if (kb1 < k_blocks)
+      merge = -1;
+    else if (kb0 > 0)
+      merge = sk_owner(p, static_cast<long long>(tile - p.sk_tile0) * k_blocks, units);
+    if (n < max_items) {
+      items[4 * n + 0] = tile;
+      items[4 * n + 1] = kb0;
+      items[4 * n + 2] = kb1;
+      items[4 * n + 3] = merge;
+    }
+    ++n;
+  }
+  return n;
+}
 
 unsigned long long next_scratch_seq() { return next_sk_seq(); }
 

@@ -353,6 +353,20 @@ int h3b_sync_status(void* stream) {
 
 size_t h3b_gemm_workspace_size(void) { return gemm_scratch_bytes(); }
 
+int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, int* items,
+                      int max_items) {
+  if (tiles <= 0 || k_blocks <= 0 || units <= 0 || unit < 0 || unit >= units)
+    return set_error(H3B_EINVAL, "gemm_schedule: tiles=%d k_blocks=%d units=%d unit=%d", tiles,
+                     k_blocks, units, unit);
+  if (mode < 0 || mode > 2) return set_error(H3B_EINVAL, "gemm_schedule: mode %d", mode);
+  if (max_items < 0 || (max_items > 0 && !items))
+    return set_error(H3B_EINVAL, "gemm_schedule: items buffer");
+  const int n = gemm_schedule_items(tiles, k_blocks, units, mode, unit, items, max_items);
+  if (n < 0)
+    return set_error(H3B_EINVAL, "gemm_schedule: fewer than 4 split K slices per unit");
+  return n;
+}
+
 size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens) {
   if (check_dims(dims) || n_tokens < 0) return 0;
   return arena_bytes(dims, n_tokens);

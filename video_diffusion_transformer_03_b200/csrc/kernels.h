@@ -66,6 +66,9 @@ constexpr size_t kScratchBytes = kAttnFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
 size_t gemm_scratch_bytes();
 // A value no flag can hold from an earlier launch of this process.
 unsigned long long next_scratch_seq();
+// Host enumeration of one scheduling unit's GEMM work items (h3b_gemm_schedule).
+int gemm_schedule_items(int tiles, int k_blocks, int units, int mode, int unit, int* items,
+                        int max_items);
 
 // out = A[M, K] * B[N, K]^T with epilogue; bf16 inputs.  K % 64 == 0, N % 128 == 0.
 // scratch (>= gemm_scratch_bytes(), or null) enables the stream-K schedule when the

@@ -56,6 +56,7 @@ _SIGS = {
     "h3b_workspace_size": (_SZ, [ctypes.POINTER(Dims), _I]),
     "h3b_gemm_workspace_size": (_SZ, []),
     "h3b_denoise_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I]),
+    "h3b_gemm_schedule": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int), _I]),
     "h3b_adaln_modulation": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "h3b_rope_table": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I, _P, _P]),
     "h3b_ln_modulate": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
@@ -156,6 +157,23 @@ def make_block_weights(p) -> BlockWeights:
 
 def gemm_workspace_size() -> int:
     return int(lib.h3b_gemm_workspace_size())
+
+
+SCHED_DATA_PARALLEL, SCHED_HYBRID_STREAM_K, SCHED_STREAM_K = 0, 1, 2
+
+
+def gemm_schedule(tiles: int, k_blocks: int, units: int, mode: int, unit: int):
+    """Work items (tile, first K slice, end K slice, merge) of one GEMM scheduling unit, in
+    processing order, as the kernels compute them (host only, no GPU)."""
+    cap = 16
+    while True:
+        buf = (ctypes.c_int * (4 * cap))()
+        n = int(lib.h3b_gemm_schedule(tiles, k_blocks, units, mode, unit, buf, cap))
+        if n < 0:
+            _check(n)
+        if n <= cap:
+            return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
+        cap = n
 
 
 def _wsargs(ws):
