@@ -42,11 +42,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # ncu --set full, one launch of the dit512 shape after 3 warm-ups (profiles/)
     "gemm_fc2_gate": {"bytes": 136698880 + 17368576, "src": "gemm_tc.cu",
-                      "src_sha": "79db5b50ff5f8350"},
+                      "src_sha": "85fffcd9e59c9ba3"},
     "gemm_out_gate": {"bytes": 38648832 + 1331968, "src": "gemm_tc.cu",
-                      "src_sha": "79db5b50ff5f8350"},
+                      "src_sha": "85fffcd9e59c9ba3"},
     "gemm_fc1_gelu": {"bytes": 85517824 + 18561280, "src": "gemm_tc.cu",
-                      "src_sha": "79db5b50ff5f8350"},
+                      "src_sha": "85fffcd9e59c9ba3"},
 }
 
 

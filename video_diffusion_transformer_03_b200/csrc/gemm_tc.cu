@@ -1091,7 +1091,8 @@ unsigned long long next_sk_seq() {
 }
 
 // First stream-K tile of the pair kernel's hybrid schedule: every whole wave of tiles but
-// the last runs data-parallel, so the split part holds between one and two tiles per unit.
+// the last runs data-parallel, so the split part holds between one and two tiles per unit
+// (all tiles, when there are fewer than two waves).
 int hybrid_tile0(int tiles, int units) { return std::max(0, tiles / units - 1) * units; }
 
 // Schedule costs in units of one K slice of one tile on one scheduling unit.
