@@ -143,6 +143,11 @@ def test_rope_positions_layout():
     assert pr[3].tolist() == [0, 1, 2.5]
     ph = O.rope_positions((2, 2, 4), n_audio=0, halved=True)
     assert ph[15].tolist() == [1, 0.5, 1.5]
+    # halved and paired: the merged token's w is the mean of its sources' halved w
+    php = O.rope_positions((2, 2, 4), n_audio=1, halved=True, paired=True)
+    assert php.shape == (9, 3)
+    assert php[0].tolist() == [0, 0, 0.25] and php[7].tolist() == [1, 0.5, 1.25]
+    assert php[8].tolist() == [0, 0, 0]
     # audio tokens are left unrotated
     x = RNG.standard_normal((19, 1, 8))
     out = O.rope_rotate(x, pos, (2, 2, 4), 10.0)
@@ -400,3 +405,182 @@ def test_denoise_update_with_constant_velocity():
     want[:8] -= 0.5
     want[8:] += 2.0
     assert np.allclose(out, want, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- denoise loop
+# The Euler loop with token reduction composed independently of oracle.denoise: torch
+# average pooling for the pairing (positions pooled the same way as the tokens, so the
+# merged token's position is the mean of its sources), repeat_interleave for the bypass
+# restore, torch layer_norm for the final AdaLN, and _torch_block for every block.
+F = torch.nn.functional
+
+
+def _grid_positions(grid, n_audio, halved):
+    t_n, h_n, w_n = grid
+    vid = torch.cartesian_prod(torch.arange(t_n, dtype=torch.float64),
+                               torch.arange(h_n, dtype=torch.float64),
+                               torch.arange(w_n, dtype=torch.float64))
+    if halved:
+        vid[:, 1:] *= 0.5
+    return torch.cat([vid, torch.zeros((n_audio, 3), dtype=torch.float64)])
+
+
+def _pool_w(x, grid):
+    """Width-2 average pool over the w axis of the video rows of x [N, c]."""
+    t_n, h_n, w_n = grid
+    nv = t_n * h_n * w_n
+    vid = x[:nv].reshape(t_n * h_n, w_n, -1).transpose(1, 2)            # [t h, c, w]
+    return F.avg_pool1d(vid, 2).transpose(1, 2).reshape(nv // 2, -1)
+
+
+def _torch_pair(x, grid, n_audio):
+    nv = grid[0] * grid[1] * grid[2]
+    return torch.cat([_pool_w(x, grid), x[nv:nv + n_audio]])
+
+
+def _torch_unpair(x_red, grid, n_audio, saved):
+    nv = grid[0] * grid[1] * grid[2]
+    red = x_red[:nv // 2]
+    if saved is None:
+        vid = red.repeat_interleave(2, dim=0)
+    else:
+        vid = saved[:nv] + (red - _pool_w(saved, grid)).repeat_interleave(2, dim=0)
+    return torch.cat([vid, x_red[nv // 2:nv // 2 + n_audio]])
+
+
+def _torch_denoise(x0, blocks, mods, fm, grid, n_audio, heads, split, theta, eps, steps,
+                   active=None, reduce_after=-1, halved=False, bypass=True):
+    x_state = torch.from_numpy(np.asarray(x0, np.float64))
+    fm = torch.from_numpy(np.asarray(fm, np.float64))
+    nv = grid[0] * grid[1] * grid[2]
+    pos_full = _grid_positions(grid, n_audio, halved)
+    pos_red = torch.cat([_pool_w(pos_full, grid), pos_full[nv:]])
+    order = [b for b in range(len(blocks)) if active is None or active[b]]
+    for i in range(steps):
+        s, s_next = 1.0 - i / steps, 1.0 - (i + 1) / steps
+        x = x_state.to(torch.bfloat16).to(torch.float64)
+        saved, pos = None, pos_full
+        for k, b in enumerate(order):
+            x = torch.from_numpy(_torch_block(x.numpy(), blocks[b], mods[b], pos.numpy(),
+                                              heads, split, theta, eps))
+            if k + 1 == reduce_after and k + 1 < len(order):
+                saved, x, pos = x, _torch_pair(x, grid, n_audio), pos_red
+        if saved is not None:
+            x = _torch_unpair(x, grid, n_audio, saved if bypass else None)
+        xn = F.layer_norm(x, (x.shape[1],), eps=eps)
+        v = torch.cat([xn[:nv] * (1 + fm[0, 1]) + fm[0, 0], xn[nv:] * (1 + fm[1, 1]) + fm[1, 0]])
+        x_state = x_state + (s_next - s) * v
+    return x_state.numpy()
+
+
+def _denoise_case(n_blocks=4, seed=21):
+    blocks, mods = [], []
+    for b in range(n_blocks):
+        w, mod = _tiny_block(seed=seed + b)
+        blocks.append(w)
+        mods.append(mod)
+    r = np.random.default_rng(seed + 100)
+    fm = r.standard_normal((2, 2, 64)) * 0.3
+    grid, na = (2, 2, 4), 3
+    x0 = O.round_to_bf16(r.standard_normal((16 + na, 64))).astype(np.float64)
+    return blocks, np.stack(mods), fm, grid, na, x0
+
+
+_DENOISE_ARGS = dict(heads=2, split=(8, 12, 12), theta=1e4, eps=1e-6)
+
+
+@pytest.mark.parametrize("reduce_after,active,halved,bypass", [
+    (2, None, False, True), (1, [1, 1, 0, 1], False, True), (2, [1, 0, 1, 1], True, True),
+    (3, None, False, False), (-1, [1, 1, 0, 1], True, True)])
+def test_denoise_matches_independent_torch_composition(reduce_after, active, halved, bypass):
+    blocks, mods, fm, grid, na, x0 = _denoise_case()
+    a = _DENOISE_ARGS
+    want = _torch_denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                          a["eps"], 2, active, reduce_after, halved, bypass)
+    got = O.denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                    a["eps"], steps=2, run_steps=2, active=active, reduce_after=reduce_after,
+                    halved=halved, unpair_bypass=bypass)
+    assert np.max(np.abs(got - want)) < 1e-10
+
+
+def _oracle_denoise_2(blocks, mods, fm, grid, na, x0, **kw):
+    a = _DENOISE_ARGS
+    return O.denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                     a["eps"], steps=2, run_steps=2, **kw)
+
+
+def test_denoise_with_identity_reduced_blocks_equals_the_unreduced_prefix():
+    # blocks after the pairing with zero gates are identities, so the bypass restore gets
+    # back exactly the stream saved at the pairing: the trajectory is that of the first
+    # reduce_after blocks alone, without any reduction
+    blocks, mods, fm, grid, na, x0 = _denoise_case()
+    mods = mods.copy()
+    mods[2:, 2] = 0
+    mods[2:, 5] = 0
+    got = _oracle_denoise_2(blocks, mods, fm, grid, na, x0, reduce_after=2)
+    want = _oracle_denoise_2(blocks[:2], mods[:2], fm, grid, na, x0)
+    assert np.max(np.abs(got - want)) < 1e-12
+    # the duplicate restore instead gives each video token its pair's mean
+    got_dup = _oracle_denoise_2(blocks, mods, fm, grid, na, x0, reduce_after=2,
+                                unpair_bypass=False)
+    assert np.max(np.abs(got_dup - want)) > 1e-3
+
+
+def test_denoise_duplicate_restore_closed_form_one_step():
+    # one step, identity blocks after the pairing, duplicate restore: the final AdaLN sees
+    # each video token replaced by the mean of its horizontal pair (audio untouched)
+    blocks, mods, fm, grid, na, x0 = _denoise_case()
+    mods = mods.copy()
+    mods[1:, 2] = 0
+    mods[1:, 5] = 0
+    a = _DENOISE_ARGS
+    got = O.denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                    a["eps"], steps=4, run_steps=1, reduce_after=1, unpair_bypass=False)
+    pos = O.rope_positions(grid, na)
+    x = O.round_to_bf16(x0).astype(np.float64)
+    x1, _ = O.block_forward(x, blocks[0], mods[0], pos, a["heads"], a["split"], a["theta"],
+                            a["eps"])
+    dup = x1.copy()
+    dup[0:16:2] = dup[1:16:2] = 0.5 * (x1[0:16:2] + x1[1:16:2])
+    v = O.final_adaln(dup, fm, 16, a["eps"])
+    assert np.max(np.abs(got - (x0 - 0.25 * v))) < 1e-12
+
+
+@pytest.mark.parametrize("mistake", ["pair_late", "full_positions", "unpair_saved_early",
+                                     "final_on_reduced"])
+def test_denoise_comparison_catches_planted_mistakes(mistake, monkeypatch):
+    # each plausible slip in the orchestration, planted in the oracle, makes the
+    # comparison with the independent composition fail
+    blocks, mods, fm, grid, na, x0 = _denoise_case()
+    a = _DENOISE_ARGS
+    want = _torch_denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                          a["eps"], 2, None, 2)
+    kw = dict(reduce_after=2)
+    if mistake == "pair_late":
+        kw["reduce_after"] = 3
+    elif mistake == "full_positions":
+        real = O.rope_positions
+        monkeypatch.setattr(O, "rope_positions",
+                            lambda g, n, halved=False, paired=False, dt=np.float64:
+                            real(g, n, halved, False, dt)
+                            if not paired else
+                            real(g, n, halved, False, dt)[np.r_[0:16:2, 16:16 + n]])
+    elif mistake == "unpair_saved_early":
+        real_pair = O.token_pair
+        first = {}
+
+        def pair_and_keep(x, g, n, dt=np.float64):
+            first.setdefault("x", x)
+            return real_pair(x, g, n, dt)
+        real_unpair = O.token_unpair
+        monkeypatch.setattr(O, "token_pair", pair_and_keep)
+        monkeypatch.setattr(O, "token_unpair",
+                            lambda xr, g, n, saved=None, dt=np.float64:
+                            real_unpair(xr, g, n, first["x"] * 0.5 + saved * 0.5, dt))
+    elif mistake == "final_on_reduced":
+        real_unpair = O.token_unpair
+        monkeypatch.setattr(O, "token_unpair",
+                            lambda xr, g, n, saved=None, dt=np.float64:
+                            real_unpair(xr, g, n, None, dt))
+    got = _oracle_denoise_2(blocks, mods, fm, grid, na, x0, **kw)
+    assert np.max(np.abs(got - want)) > 1e-4
