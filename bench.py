@@ -11,9 +11,11 @@ weights of the stated architecture).  The metric is DiT block tokens per second:
 processed by each executed block, summed over blocks and Euler steps, per second of
 device time; TFLOPS counts 24 N d^2 + 4 N^2 d per block.
 
-Multi-GPU (torchrun, one process per GPU): every rank denoises its own latent with the
-same weights (independent replicas, no data-path collective); value = all ranks' tokens
-/ the slowest rank's device time.
+Multi-GPU (one process per GPU): every rank denoises its own latent with the same weights
+(independent replicas, no data-path collective); value = all ranks' tokens / the slowest
+rank's device time.  Under torchrun the ranks come from the environment; `--gpus N` with
+N > 1 and no WORLD_SIZE set re-launches this script under torch.distributed.run with N
+processes (127.0.0.1 rendezvous), so N GPUs really run.
 
 --impl reference runs the CPU oracle (the plain float64 definition of the same block) on
 a bounded sample of the workload: one block over the full token count per step.
@@ -50,7 +52,7 @@ NCU_TRAFFIC = {
 }
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -67,7 +69,10 @@ def parse_args():
                     help="skip the secondary measurements of the other workloads")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying a CUDA graph")
-    return ap.parse_args()
+    ap.add_argument("--replica-check", action="store_true",
+                    help="CPU only: run the replica plumbing (gloo barrier, max over ranks, "
+                         "job rate) through the same launcher and print what every rank saw")
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -203,7 +208,9 @@ def run_reference(args):
     except Exception:
         cores = os.cpu_count()
     flops = block_flops(cfg.n_tokens, cfg.d, cfg.d_ff)
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    # one process (rank 0) ran the CPU oracle on the host cores; no GPU was used
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "processes": 1, "ranks_launched": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -687,9 +694,53 @@ def run_gpu(args):
         print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse_args()
-    if args.impl == "reference":
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_command(n: int, argv, port: int):
+    """The torch.distributed.run command that starts this script as n local ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__)] + list(argv)
+
+
+def relaunch_as_ranks(n: int, argv, timeout_s: float = 3600.0) -> int:
+    """Run this script as n ranks (one process per GPU) and return the launcher's status.
+    The ranks' process group has its own short timeout; this bound sits well above it."""
+    cmd = launch_command(n, argv, _free_port())
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1")
+    try:
+        return subprocess.run(cmd, env=env, timeout=timeout_s).returncode
+    except subprocess.TimeoutExpired:
+        return 124
+
+
+def run_replica_check(args):
+    """The N-rank plumbing on CPU (gloo): barrier, max of a per-rank time, job rate."""
+    import torch
+    reps = Replicas("gloo", torch.device("cpu"), timeout_s=60)
+    reps.barrier()
+    ms = reps.max(10.0 + 5.0 * reps.rank)
+    value = reps.throughput(1000, 4, ms)
+    reps.barrier()
+    line = {"replica_check": True, "rank": reps.rank, "world": reps.world, "max_ms": ms,
+            "value": value}
+    reps.close()
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl != "reference":
+        sys.exit(relaunch_as_ranks(args.gpus, argv))
+    if args.replica_check:
+        run_replica_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

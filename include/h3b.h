@@ -33,7 +33,15 @@
  *     nothing.  h3b_last_error() returns a message for the calling thread's last error.
  *   - Device-side waits inside the kernels give up after about two seconds; the kernel
  *     then returns early and records the event in a per-device flag, which the next
- *     h3b_sync_status call reports as H3B_ETIMEOUT.
+ *     h3b_sync_status call reports as H3B_ETIMEOUT.  The outputs of that work are
+ *     invalid, and so are split-schedule flags it left in the caller's workspace: when
+ *     h3b_sync_status reports H3B_ETIMEOUT the library drops its cached denoise graphs
+ *     (the next host call captures fresh ones with new sequence numbers); a CUDA graph
+ *     the caller captured around library calls must be captured again too.
+ *   - Per device, the library caches the device addresses of its module variables, its
+ *     copy streams and its captured graphs for the life of the process; it assumes the
+ *     device's primary context lives as long (cudaDeviceReset while the library is in
+ *     use is not supported).
  */
 #ifndef H3B_H_
 #define H3B_H_
@@ -140,6 +148,20 @@ size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, in
  * shapes data-parallel). */
 int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, int* items,
                       int max_items);
+
+/* Force the GEMM dispatch for every later GEMM launch of this process, for measurements
+ * and tests (the automatic choice is the product path; this call exists so that each
+ * tile configuration and schedule can be exercised and timed on purpose, in place of
+ * environment switches).  -1 restores the automatic choice for that field.
+ *   tile:  0 CTA-pair 256-wide, 1 CTA-pair 128-wide, 2 single-CTA 256, 3 single-CTA 128
+ *          (used where the shape allows it);
+ *   sched: 0 data-parallel, 1 hybrid stream-K, 2 stream-K over every tile (where the
+ *          scratch allows it and each unit gets at least 4 split K slices);
+ *   trans: 0 never, 1 always use the transposed pair kernel where the shape allows it.
+ * Returns H3B_OK, or H3B_EINVAL (nothing changed) for a value out of range.  Applies to
+ * launches issued after the call, on every thread; a CUDA graph keeps the launches it
+ * captured. */
+int h3b_set_gemm_override(int tile, int sched, int trans);
 
 /* ---------------------------------------------------------------- hot-path steps */
 /* AdaLN modulation vectors: mod[j] = sum_k w[j, k] c[k] + b[j], j < n_out.

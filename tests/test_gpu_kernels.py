@@ -76,8 +76,9 @@ def test_gemm_epilogues(M, N, K, epi, sk):
 def test_gemm_hybrid_stream_k_schedule():
     # The CTA-pair kernel splits only its last one to two tiles per pair stream-K and runs
     # the whole waves before them data-parallel; the cost model picks that form only where
-    # it wins, so force it (H3B_GEMM_SCHED is read once per process: run a child) on shapes
-    # with a data-parallel phase, partial tiles and a ragged last row tile.
+    # it wins, so force it (h3b_set_gemm_override) on shapes with a data-parallel phase,
+    # partial tiles and a ragged last row tile.  A child process, so that the schedule
+    # trace (H3B_TRACE_GEMM, read once per process) shows the form each launch took.
     import os
     import subprocess
     import sys
@@ -87,6 +88,7 @@ def test_gemm_hybrid_stream_k_schedule():
         "from tests.helpers import max_block_rel_l2, np64, rel_l2, rnd\n"
         "from video_diffusion_transformer_03_b200 import h3b\n"
         "ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device='cuda')\n"
+        "h3b.set_gemm_override(-1, h3b.SCHED_HYBRID_STREAM_K, 0)\n"
         "for (M, N, K, epi) in [(1000, 9728, 512, h3b.EPI_GATE_RESID),\n"
         "                       (1600, 12288, 3072, h3b.EPI_BIAS_GELU)]:\n"
         "    A = rnd((M, K), 1.0, seed=11); B = rnd((N, K), K ** -0.5, seed=12)\n"
@@ -105,13 +107,90 @@ def test_gemm_hybrid_stream_k_schedule():
         "    assert rel_l2(got, want) < 4e-3 and max_block_rel_l2(got, want) < 8e-3, (M, N, K)\n"
         "print('ok')\n")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, H3B_GEMM_SCHED="sk", H3B_GEMM_TRANS="0", H3B_TRACE_GEMM="1",
-               PYTHONPATH=root)
+    env = dict(os.environ, H3B_TRACE_GEMM="1", PYTHONPATH=root)
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
                        timeout=600, cwd=root)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
     # the launches took the hybrid form: a data-parallel phase before the split tiles
     assert "sk_tile0=74" in r.stderr and "sk_tile0=222" in r.stderr, r.stderr
+
+
+def _rope_want(acc, grid, n_audio, heads, hd, split):
+    d = heads * hd
+    M = acc.shape[0]
+    pos = O.rope_positions(grid, n_audio)
+    want = acc.copy()
+    for part in range(2):
+        blk = acc[:, part * d:(part + 1) * d].reshape(M, heads, hd)
+        want[:, part * d:(part + 1) * d] = O.rope_rotate(blk, pos, split, 1e4).reshape(M, d)
+    return want
+
+
+# (grid, audio tokens) giving M = 832, 1000 and 1600 rows: the transposed kernel's 160-token
+# tiles end ragged at 832 and 1000 (M % 160 = 32 and 40) and exactly at 1600
+TRANS_GRIDS = [((6, 16, 8), 64), ((5, 10, 18), 100), ((6, 16, 16), 64)]
+
+
+@pytest.mark.parametrize("grid,n_audio", TRANS_GRIDS)
+@pytest.mark.parametrize("epi", [h3b.EPI_BIAS, h3b.EPI_BIAS_GELU, h3b.EPI_BIAS_ROPE,
+                                 h3b.EPI_GATE_RESID])
+def test_gemm_transposed_pair_kernel_forced(grid, n_audio, epi):
+    # the weight-rows-by-token-tiles kernel runs where the cost model picks it (the
+    # out-projection at 832 tokens); forced here on every epilogue and on ragged token counts
+    heads, hd, split = 8, 128, (32, 48, 48)
+    d = heads * hd
+    M = grid[0] * grid[1] * grid[2] + n_audio
+    N, K = 3 * d, d
+    A = rnd((M, K), 1.0, seed=71)
+    B = rnd((N, K), K ** -0.5, seed=72)
+    bias = rnd((N,), 0.1, seed=73)
+    acc = np64(A) @ np64(B).T + np64(bias)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    kw = {}
+    if epi == h3b.EPI_BIAS:
+        want = acc
+    elif epi == h3b.EPI_BIAS_GELU:
+        want = O.gelu_tanh(acc)
+    elif epi == h3b.EPI_BIAS_ROPE:
+        dims = h3b.make_dims(d, heads, hd, 4 * d, 256, split)
+        cs = torch.empty((M, hd // 2, 2), dtype=torch.float32, device=DEV)
+        h3b.rope_table(dims, h3b.make_grid(*grid, n_audio), False, cs)
+        kw = dict(rope_cs=cs, rope_cols=2 * d, head_dim=hd)
+        want = _rope_want(acc, grid, n_audio, heads, hd, split)
+    else:
+        resid = rnd((M, N), 1.0, seed=74)
+        g = rnd((N,), 0.5, seed=75, dtype=torch.float32)
+        out.copy_(resid.to(DEV))
+        kw = dict(gate=g.to(DEV))
+        want = O.gated_residual(np64(resid), np64(g), acc)
+    with h3b.gemm_override(trans=1):
+        h3b.gemm_bf16(A.to(DEV), B.to(DEV), epi, bias.to(DEV), out, ws=gemm_scratch(), **kw)
+        _sync()
+    got = np64(out)
+    assert rel_l2(got, want) < 4e-3
+    assert max_block_rel_l2(got, want) < 8e-3
+
+
+@pytest.mark.parametrize("tile", [h3b.TILE_PAIR128, h3b.TILE_SINGLE256, h3b.TILE_SINGLE128])
+@pytest.mark.parametrize("sched", [h3b.SCHED_DATA_PARALLEL, h3b.SCHED_STREAM_K])
+def test_gemm_forced_tile_configurations(tile, sched):
+    # every tile configuration and schedule the dispatch can take, at a shape with a ragged
+    # last row tile and enough K slices for stream-K
+    M, N, K = 1000, 1280, 4096
+    A = rnd((M, K), 1.0, seed=81)
+    B = rnd((N, K), K ** -0.5, seed=82)
+    bias = rnd((N,), 0.1, seed=83)
+    resid = rnd((M, N), 1.0, seed=84)
+    g = rnd((N,), 0.5, seed=85, dtype=torch.float32)
+    want = O.gated_residual(np64(resid), np64(g), np64(A) @ np64(B).T + np64(bias))
+    out = resid.to(DEV)
+    with h3b.gemm_override(tile=tile, sched=sched, trans=0):
+        h3b.gemm_bf16(A.to(DEV), B.to(DEV), h3b.EPI_GATE_RESID, bias.to(DEV), out,
+                      gate=g.to(DEV), ws=gemm_scratch())
+        _sync()
+    got = np64(out)
+    assert rel_l2(got, want) < 4e-3
+    assert max_block_rel_l2(got, want) < 8e-3
 
 
 @pytest.mark.parametrize("grid,n_audio,heads,hd,split", [
@@ -134,11 +213,7 @@ def test_gemm_rope_epilogue(grid, n_audio, heads, hd, split):
                   rope_cols=2 * d, head_dim=hd, ws=gemm_scratch())
     _sync()
     acc = np64(A) @ np64(B).T + np64(bias)
-    pos = O.rope_positions(grid, n_audio)
-    want = acc.copy()
-    for part in range(2):
-        blk = acc[:, part * d:(part + 1) * d].reshape(M, heads, hd)
-        want[:, part * d:(part + 1) * d] = O.rope_rotate(blk, pos, split, 1e4).reshape(M, d)
+    want = _rope_want(acc, grid, n_audio, heads, hd, split)
     got = np64(out)
     assert rel_l2(got, want) < 4e-3
     assert max_block_rel_l2(got, want) < 8e-3
@@ -387,6 +462,7 @@ def test_adaln_modulation():
     ((6, 16, 16), 64, False, False, 128, (32, 48, 48)),
     ((6, 16, 16), 64, False, True, 128, (32, 48, 48)),
     ((6, 8, 8), 64, True, False, 128, (32, 48, 48)),
+    ((6, 8, 8), 64, True, True, 128, (32, 48, 48)),       # halved and paired: w = (2j + 0.5) / 2
     ((2, 4, 4), 8, False, False, 64, (16, 24, 24)),
     ((11, 24, 42), 256, False, False, 128, (32, 48, 48)),
 ])

@@ -70,7 +70,34 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         sys.argv = ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
                     "--warmup", "0"]
         try:
-            bench.run_reference(bench.parse_args())
+            bench.run_reference(bench.parse_args(sys.argv[1:]))
         finally:
             sys.argv = sys_argv
     assert buf.getvalue() == ""              # the other ranks exit without work or output
+
+
+def test_gpus_flag_starts_that_many_ranks_through_the_launcher():
+    # `bench.py --gpus 2` without torchrun re-launches itself as 2 ranks; the replica check
+    # runs the same plumbing the GPU arm uses (gloo on CPU here) and every rank reports
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--replica-check"], env=env, capture_output=True, text=True,
+                       timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert sorted(l["rank"] for l in lines) == [0, 1], r.stdout
+    for l in lines:
+        assert l["world"] == 2 and l["max_ms"] == 15.0
+        assert abs(l["value"] - 1000 * 4 * 2 / 15e-3) < 1e-6 * l["value"]
+
+
+def test_launch_command_is_one_local_node_on_loopback():
+    cmd = bench.launch_command(4, ["--gpus", "4", "--steps", "3"], 29555)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]
+    assert cmd[-5].endswith("bench.py")

@@ -23,7 +23,6 @@
 #include <cstdio>
 #include <cstdlib>
 #include <random>
-#include <string>
 
 namespace h3b {
 
@@ -1315,18 +1314,13 @@ int launch_pair_trans(const DevCtx& ctx, const bf16* X, const bf16* W, int M, in
   return 0;
 }
 
-// H3B_GEMM_SCHED=sk|skall|dp forces the hybrid stream-K schedule (the pair kernel's
-// default form), stream-K over every tile, or the data-parallel schedule, where the
-// scratch allows it (diagnostics and measurements only).
-int forced_sched() {
-  static const int forced = [] {
-    const char* v = std::getenv("H3B_GEMM_SCHED");
-    if (!v) return -1;
-    const std::string t(v);
-    return t == "skall" ? 2 : t == "sk" ? 1 : t == "dp" ? 0 : -1;
-  }();
-  return forced;
-}
+// Process-wide overrides of the GEMM dispatch (h3b_set_gemm_override; diagnostics and
+// measurements only, -1 = automatic).  Set through the C ABI, never from the environment.
+std::atomic<int> g_force_tile{-1}, g_force_sched{-1}, g_force_trans{-1};
+
+// Forced schedule: 2 stream-K over every tile, 1 hybrid stream-K (the pair kernel's
+// default form), 0 data-parallel, -1 the cost model's choice; where the scratch allows it.
+int forced_sched() { return g_force_sched.load(std::memory_order_relaxed); }
 
 // H3B_TRACE_GEMM=1 prints each GEMM's schedule to stderr (diagnostics only).
 bool trace_gemm() {
@@ -1340,21 +1334,8 @@ bool trace_gemm() {
 // Tile configurations of the bf16 / int8 GEMM.
 enum TileCfg { kPair256 = 0, kPair128 = 1, kSingle256 = 2, kSingle128 = 3, kAuto = -1 };
 
-// H3B_GEMM_TILE=pair256|pair128|single256|single128 forces one configuration where the
-// shape allows it (diagnostics and measurements only).
-int forced_tile() {
-  static const int forced = [] {
-    const char* v = std::getenv("H3B_GEMM_TILE");
-    if (!v) return int(kAuto);
-    const std::string t(v);
-    if (t == "pair256") return int(kPair256);
-    if (t == "pair128") return int(kPair128);
-    if (t == "single256") return int(kSingle256);
-    if (t == "single128") return int(kSingle128);
-    return int(kAuto);
-  }();
-  return forced;
-}
+// Forced tile configuration (a TileCfg value), where the shape allows it.
+int forced_tile() { return g_force_tile.load(std::memory_order_relaxed); }
 
 bool tile_allowed(int cfg, int M, int N) {
   switch (cfg) {
@@ -1391,6 +1372,15 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
 }  // namespace
 
 size_t gemm_scratch_bytes() { return kScratchBytes; }
+
+int set_gemm_override(int tile, int sched, int trans) {
+  if (tile < -1 || tile > kSingle128 || sched < -1 || sched > 2 || trans < -1 || trans > 1)
+    return -1;
+  g_force_tile.store(tile);
+  g_force_sched.store(sched);
+  g_force_trans.store(trans);
+  return 0;
+}
 
 // The work items of one scheduling unit, from the functions the kernels run: (tile, first
 // K slice, end K slice, merge) with merge = -1 for a partial tile the unit parks for a
@@ -1438,16 +1428,8 @@ bool try_pair_bf16(int bn, const DevCtx& ctx, const bf16* A, const bf16* B, int 
   return launch_pair<128, false, EPI>(ctx, A, B, M, N, K, epi, ws, wsb, s, rc) == 0;
 }
 
-// H3B_GEMM_TRANS=0|1 forbids or forces the transposed pair kernel where the shape allows
-// it (diagnostics and measurements only).
-int forced_trans() {
-  static const int forced = [] {
-    const char* v = std::getenv("H3B_GEMM_TRANS");
-    if (!v || !v[0]) return -1;
-    return v[0] == '1' ? 1 : 0;
-  }();
-  return forced;
-}
+// Forced use (1) or exclusion (0) of the transposed pair kernel where the shape allows it.
+int forced_trans() { return g_force_trans.load(std::memory_order_relaxed); }
 
 // Transposed (tokens on the 160-wide side) or not, from the same cost reasoning as the
 // stream-K choice, in units of one 256 x 256 tile on one CTA pair: the untransposed

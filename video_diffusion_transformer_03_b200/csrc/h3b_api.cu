@@ -38,6 +38,23 @@ bool debug_mode() {
 
 constexpr int kMaxDevices = 64;
 
+// Captured whole denoises of the host entry points (see denoise_graph), per device.
+struct DenoiseGraph {
+  std::vector<uint8_t> key;
+  cudaGraphExec_t exec = nullptr;
+};
+std::mutex g_graph_mu;
+std::vector<DenoiseGraph> g_graphs[kMaxDevices];
+
+// Forget a device's captured denoises: after a wait timed out, the split schedules'
+// flags in the workspace may hold a sequence number a replay would reuse.
+void drop_graphs(int device) {
+  if (device < 0 || device >= kMaxDevices) return;
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  for (DenoiseGraph& g : g_graphs[device]) cudaGraphExecDestroy(g.exec);
+  g_graphs[device].clear();
+}
+
 }  // namespace
 
 int set_error(int code, const char* fmt, ...) {
@@ -346,6 +363,8 @@ int h3b_sync_status(void* stream) {
   if (flag) {
     const uint32_t zero = 0;
     cudaMemcpyToSymbol(g_h3b_wait_error, &zero, sizeof(zero));
+    int dev = -1;
+    if (cudaGetDevice(&dev) == cudaSuccess) drop_graphs(dev);
     return set_error(H3B_ETIMEOUT, "a device-side wait gave up (code %u)", flag);
   }
   return H3B_OK;
@@ -365,6 +384,13 @@ int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, in
   if (n < 0)
     return set_error(H3B_EINVAL, "gemm_schedule: fewer than 4 split K slices per unit");
   return n;
+}
+
+int h3b_set_gemm_override(int tile, int sched, int trans) {
+  if (set_gemm_override(tile, sched, trans))
+    return set_error(H3B_EINVAL, "set_gemm_override: tile=%d sched=%d trans=%d", tile, sched,
+                     trans);
+  return H3B_OK;
 }
 
 size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens) {
@@ -509,13 +535,8 @@ namespace {
 // Captured whole denoises (the Euler steps of one request on one state buffer), kept per
 // device and keyed by every argument that shapes the launches: a replay relaunches the
 // same kernels with the same arguments (the split schedules' flags are handed back at zero
-// by their readers, so replays stay correct).  Captured on a stream of the library's and
-// launched on the caller's.
-struct DenoiseGraph {
-  std::vector<uint8_t> key;
-  cudaGraphExec_t exec = nullptr;
-};
-
+// by their readers, so replays stay correct; after a timed-out wait h3b_sync_status drops
+// them all).  Captured on a stream of the library's and launched on the caller's.
 constexpr size_t kGraphCacheSize = 4;
 
 void key_bytes(std::vector<uint8_t>& k, const void* v, size_t n) {
@@ -529,8 +550,6 @@ int denoise_graph(const DevCtx& ctx, const h3b_dims* dims, const h3b_grid* grid,
                   const float* mods, const float* final_mod, int reduce_after,
                   int unpair_bypass, int n_steps, int first_step, int n_run, float* state,
                   const StepBufs& b, void* ws, size_t ws_bytes, cudaGraphExec_t* out) {
-  static std::mutex mu;
-  static std::vector<DenoiseGraph> cache[kMaxDevices];
   static cudaStream_t capture_stream[kMaxDevices] = {};
   std::vector<uint8_t> key;
   H3B_KEY_PUT(key, *dims);
@@ -551,8 +570,8 @@ int denoise_graph(const DevCtx& ctx, const h3b_dims* dims, const h3b_grid* grid,
   H3B_KEY_PUT(key, state);
   H3B_KEY_PUT(key, ws);
   H3B_KEY_PUT(key, ws_bytes);
-  std::lock_guard<std::mutex> lock(mu);
-  auto& c = cache[ctx.device];
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  auto& c = g_graphs[ctx.device];
   for (const DenoiseGraph& gph : c)
     if (gph.key == key) {
       *out = gph.exec;

@@ -69,6 +69,8 @@ unsigned long long next_scratch_seq();
 // Host enumeration of one scheduling unit's GEMM work items (h3b_gemm_schedule).
 int gemm_schedule_items(int tiles, int k_blocks, int units, int mode, int unit, int* items,
                         int max_items);
+// Process-wide GEMM dispatch overrides (h3b_set_gemm_override); -1 on bad values.
+int set_gemm_override(int tile, int sched, int trans);
 
 // out = A[M, K] * B[N, K]^T with epilogue; bf16 inputs.  K % 64 == 0, N % 128 == 0.
 // scratch (>= gemm_scratch_bytes(), or null) enables the stream-K schedule when the

@@ -57,6 +57,7 @@ _SIGS = {
     "h3b_gemm_workspace_size": (_SZ, []),
     "h3b_denoise_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I]),
     "h3b_gemm_schedule": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int), _I]),
+    "h3b_set_gemm_override": (_I, [_I, _I, _I]),
     "h3b_adaln_modulation": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "h3b_rope_table": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I, _P, _P]),
     "h3b_ln_modulate": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
@@ -174,6 +175,30 @@ def gemm_schedule(tiles: int, k_blocks: int, units: int, mode: int, unit: int):
         if n <= cap:
             return [tuple(buf[4 * i:4 * i + 4]) for i in range(n)]
         cap = n
+
+
+TILE_PAIR256, TILE_PAIR128, TILE_SINGLE256, TILE_SINGLE128 = 0, 1, 2, 3
+
+
+def set_gemm_override(tile: int = -1, sched: int = -1, trans: int = -1) -> None:
+    """Force the GEMM tile configuration / schedule / transposed kernel for later launches
+    of this process (tests and measurements); -1 restores the automatic choice."""
+    _check(lib.h3b_set_gemm_override(tile, sched, trans))
+
+
+class gemm_override:
+    """Context manager around set_gemm_override that restores the automatic choice."""
+
+    def __init__(self, tile: int = -1, sched: int = -1, trans: int = -1):
+        self.args = (tile, sched, trans)
+
+    def __enter__(self):
+        set_gemm_override(*self.args)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemm_override(-1, -1, -1)
+        return False
 
 
 def _wsargs(ws):
