@@ -720,17 +720,22 @@ def relaunch_as_ranks(n: int, argv, timeout_s: float = 3600.0) -> int:
 
 
 def run_replica_check(args):
-    """The N-rank plumbing on CPU (gloo): barrier, max of a per-rank time, job rate."""
+    """The N-rank plumbing on CPU (gloo): barrier, max of a per-rank time, job rate; rank 0
+    prints one line with what every rank saw."""
     import torch
     reps = Replicas("gloo", torch.device("cpu"), timeout_s=60)
     reps.barrier()
     ms = reps.max(10.0 + 5.0 * reps.rank)
     value = reps.throughput(1000, 4, ms)
+    seen = {"rank": reps.rank, "world": reps.world, "max_ms": ms, "value": value}
+    views = [seen]
+    if reps.world > 1:
+        views = [None] * reps.world
+        reps.dist.all_gather_object(views, seen)
     reps.barrier()
-    line = {"replica_check": True, "rank": reps.rank, "world": reps.world, "max_ms": ms,
-            "value": value}
     reps.close()
-    print(json.dumps(line), flush=True)
+    if reps.rank == 0:
+        print(json.dumps({"replica_check": True, "ranks": views}), flush=True)
 
 
 def main(argv=None):

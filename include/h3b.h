@@ -91,7 +91,15 @@ typedef struct h3b_grid {
 
 /* Parameters of one block (device, bf16).  Weights are [out, in]: w_qkv [3d, d] (q rows,
  * then k, then v; head j at rows j*head_dim), w_o [d, d], w_fc1 [d_ff, d], w_fc2 [d, d_ff];
- * biases b_qkv [3d], b_o [d], b_fc1 [d_ff], b_fc2 [d]. */
+ * biases b_qkv [3d], b_o [d], b_fc1 [d_ff], b_fc2 [d].
+ *
+ * The last six fields are optional (all NULL = absent): the block's two AdaLN
+ * modulations folded into the projections that consume them, as h3b_fold_adaln writes
+ * them -- w_qkv_fold [3d, d] bf16 with c_qkv, d_qkv [3d] fp32 from (shift_msa,
+ * scale_msa); w_fc1_fold [d_ff, d] bf16 with c_fc1, d_fc1 [d_ff] fp32 from (shift_mlp,
+ * scale_mlp).  With them the block reads the raw residual and no LayerNorm pass runs
+ * (h3b_block_forward_folded; h3b_denoise_step uses them when every active block has
+ * them).  h3b_block_forward ignores them. */
 typedef struct h3b_block_weights {
   const h3b_bf16* w_qkv;
   const h3b_bf16* b_qkv;
@@ -101,6 +109,12 @@ typedef struct h3b_block_weights {
   const h3b_bf16* b_fc1;
   const h3b_bf16* w_fc2;
   const h3b_bf16* b_fc2;
+  const h3b_bf16* w_qkv_fold;
+  const float* c_qkv;
+  const float* d_qkv;
+  const h3b_bf16* w_fc1_fold;
+  const float* c_fc1;
+  const float* d_fc1;
 } h3b_block_weights;
 
 /* ---------------------------------------------------------------- library information */
@@ -204,6 +218,43 @@ int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const fl
                       int compute_h, h3b_bf16* x, h3b_bf16* h, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* AdaLN folded into the projection that consumes it (dothoosh.com, "DiT fusions and
+ * memory management": the attention gate fused with the MLP AdaLN, the MLP gate producing
+ * the next block's attention AdaLN).  For h = LN(x)(1 + scale) + shift (LN without affine,
+ * biased variance) feeding y = h W^T + b:
+ *   y[r, j] = rstd_r (sum_k x[r, k] W'[j, k] - mean_r c_j) + dv_j,  with
+ *   W'[j, k] = bf16(W[j, k] (1 + scale_k)),  c_j = sum_k W'[j, k] (over the stored W'),
+ *   dv_j = sum_k shift_k W[j, k] + b_j.
+ * Exact in real arithmetic whenever the modulation vectors are fixed for the run (they are
+ * here: the conditioning vector is constant over the steps).  w [n_out, d] bf16, b [n_out]
+ * bf16, shift, scale [d] fp32; outputs w_out [n_out, d] bf16 (must not overlap w), c_out,
+ * dv_out [n_out] fp32; all device, d % 8 == 0.  Run once per block per conditioning:
+ * (shift_msa, scale_msa) with w_qkv, (shift_mlp, scale_mlp) with w_fc1. */
+int h3b_fold_adaln(const h3b_bf16* w, const h3b_bf16* b, const float* shift, const float* scale,
+                   int n_out, int d, h3b_bf16* w_out, float* c_out, float* dv_out,
+                   void* stream);
+
+/* Row statistics of the residual in the form the folded block consumes and produces:
+ * stats [n_tokens, d / 256] float2, per row and 256-column group (mean, M2) of the bf16
+ * values (M2 = sum of squared deviations from the group mean).  x [n_tokens, d] bf16
+ * device, d % 256 == 0.  (The denoise step computes these itself.) */
+int h3b_row_stats(const h3b_bf16* x, int n_tokens, int d, float* stats, void* stream);
+
+/* One DiT block with both AdaLN LayerNorms folded into the projections (the folded fields
+ * of w, from h3b_fold_adaln with this block's mod):
+ *   qkv = the folded QKV of x (reads x and its row statistics `stats`), RoPE in the epilogue
+ *   o   = attention; x = x + gate_msa (o W_o^T + b_o), the epilogue writing x's new
+ *         row statistics into stats
+ *   g   = GELU of the folded FC1 of x (reads x and stats)
+ *   x   = x + gate_mlp (g W_fc2^T + b_fc2), the epilogue writing the new statistics
+ * The result equals h3b_block_forward's x up to rounding; no h is produced: the next
+ * block (folded) reads x and stats.  mod [6, d] fp32 (the gates); x [n_tokens, d] bf16
+ * in/out; stats [n_tokens, d / 256] float2 in/out (see h3b_row_stats); ws as
+ * h3b_block_forward.  All device. */
+int h3b_block_forward_folded(const h3b_dims* dims, const h3b_block_weights* w, const float* mod,
+                             const float* rope_cs, int n_tokens, h3b_bf16* x, float* stats,
+                             void* ws, size_t ws_bytes, void* stream);
+
 /* h3b_block_forward without a caller-supplied workspace, for callers that cannot allocate
  * device memory: plug-in hosts that hand a module only its input and output buffers,
  * deployments whose memory plan is fixed before launch, and latency-critical loops that
@@ -237,7 +288,8 @@ int h3b_final_euler(const h3b_bf16* x_l, int n_tokens, int n_video, int d, float
                     void* stream);
 
 /* One Euler step of the denoising loop over all active blocks:
- *   x = bf16(x_state); for each active block b: h3b_block_forward; after `reduce_after`
+ *   x = bf16(x_state); for each active block b: h3b_block_forward (or, when every active
+ *   block carries its folded weights, h3b_block_forward_folded); after `reduce_after`
  *   executed blocks (if > 0 and blocks remain) pair horizontal video tokens; restore
  *   before the final AdaLN (bypass restore if unpair_bypass, else duplicate);
  *   x_state += (sigma_next - sigma) final_adaln(x).

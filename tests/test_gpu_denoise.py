@@ -26,9 +26,10 @@ def f64(t):
     return t.float().numpy().astype(np.float64)
 
 
-def test_tiny_denoise_vs_oracle():
+@pytest.mark.parametrize("fold", [True, False], ids=["folded", "layernorm-pass"])
+def test_tiny_denoise_vs_oracle(fold):
     cfg = synth.CONFIGS["tiny"]
-    m = DiTDenoiser(cfg, keep_host_params=True)
+    m = DiTDenoiser(cfg, keep_host_params=True, fold=fold)
     x0 = synth.latent_noise(cfg)
     x = x0.to(DEV)
     m.run(x)
@@ -41,11 +42,12 @@ def test_tiny_denoise_vs_oracle():
     assert rel_l2(got - f64(x0), want - f64(x0)) < TOL_STEPS
 
 
+@pytest.mark.parametrize("fold", [True, False], ids=["folded", "layernorm-pass"])
 @pytest.mark.parametrize("name", ["dit512", "dit512_tokred", "dit256_halved"])
-def test_denoise_vs_golden(name):
+def test_denoise_vs_golden(name, fold):
     ref = np.load(os.path.join(GOLDEN, f"{name}_oracle.npz"))
     cfg = synth.CONFIGS[name]
-    m = DiTDenoiser(cfg)
+    m = DiTDenoiser(cfg, fold=fold)
     active = np.ones(cfg.n_blocks, bool) if m.active is None else np.array(m.active)
     assert np.array_equal(active, ref["active"]), "layer-thinning mask differs from the oracle's"
     rows = ref["rows"]

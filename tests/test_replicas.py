@@ -88,8 +88,10 @@ def test_gpus_flag_starts_that_many_ranks_through_the_launcher():
                        timeout=300, cwd=ROOT)
     assert r.returncode == 0, r.stdout + r.stderr
     lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
-    assert sorted(l["rank"] for l in lines) == [0, 1], r.stdout
-    for l in lines:
+    assert len(lines) == 1, r.stdout                  # rank 0 alone prints
+    views = lines[0]["ranks"]
+    assert sorted(v["rank"] for v in views) == [0, 1], r.stdout
+    for l in views:
         assert l["world"] == 2 and l["max_ms"] == 15.0
         assert abs(l["value"] - 1000 * 4 * 2 / 15e-3) < 1e-6 * l["value"]
 

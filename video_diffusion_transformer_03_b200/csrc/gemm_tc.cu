@@ -185,6 +185,56 @@ __device__ __forceinline__ void load_f32x32(const float* src, float (&v)[32]) {
   }
 }
 
+// Row statistics an LN-folded epilogue applies to its row: mean and 1 / sqrt(var + eps).
+struct LnRow {
+  float mu, rstd;
+};
+
+// Merge a row's group statistics (mean, M2 of each 256-column group, in group order) into
+// the row's mean and reciprocal standard deviation (biased variance over all columns).
+__device__ __forceinline__ LnRow ln_row(const GemmEpilogue& e, int row) {
+  const float2* s = e.stats_in + size_t(row) * e.stats_parts;
+  float mu = 0.f;
+  for (int g = 0; g < e.stats_parts; ++g) mu += __ldg(s + g).x;
+  mu /= static_cast<float>(e.stats_parts);
+  float m2 = 0.f;
+  for (int g = 0; g < e.stats_parts; ++g) {
+    const float2 v = __ldg(s + g);
+    const float t = v.x - mu;
+    m2 += fmaf(256.0f * t, t, v.y);
+  }
+  const float var = fmaxf(m2 / (256.0f * static_cast<float>(e.stats_parts)), 0.0f);
+  return LnRow{mu, rsqrtf(var + e.ln_eps)};
+}
+
+// Shifted sums of one output row over a 256-column tile, about the row's first stored
+// value k: s1 = sum (x - k), s2 = sum (x - k)^2 of the bf16 values written.
+struct StatAcc {
+  float k, s1, s2;
+};
+
+// Add 32 stored values (16 packed bf16 pairs) of this lane's row; `first` marks the
+// tile's first chunk, whose first value becomes the shift.
+__device__ __forceinline__ void stat_add(StatAcc& a, const uint32_t (&pk)[16], bool first) {
+  if (first) {
+    a.k = __uint_as_float(pk[0] << 16);
+    a.s1 = 0.f;
+    a.s2 = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float lo = __uint_as_float(pk[i] << 16) - a.k;
+    const float hi = __uint_as_float(pk[i] & 0xFFFF0000u) - a.k;
+    a.s1 += lo + hi;
+    a.s2 = fmaf(lo, lo, fmaf(hi, hi, a.s2));
+  }
+}
+
+// The tile row's group statistics (mean, M2) over its 256 columns.
+__device__ __forceinline__ float2 stat_final(const StatAcc& a) {
+  return make_float2(a.k + a.s1 * (1.0f / 256.0f), a.s2 - a.s1 * a.s1 * (1.0f / 256.0f));
+}
+
 // Row operands of one 32-column chunk that come from global memory, loaded one chunk
 // ahead of their use so that their latency overlaps the previous chunk's work.
 struct RowIn {
@@ -199,7 +249,7 @@ __device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int 
 #pragma unroll
     for (int i = 0; i < 4; ++i) in.res[i] = s[i];  // coherent: this kernel rewrites it
   }
-  if constexpr (EPI == kEpiRope) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
       const int half = e.head_dim >> 1;
       const float4* cs = reinterpret_cast<const float4*>(
@@ -210,10 +260,12 @@ __device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int 
   }
 }
 
-// Epilogue of one 32-column chunk of one row.
+// Epilogue of one 32-column chunk of one row.  ln: the row's statistics (LN-folded
+// kinds); sa: the row's running statistics of the stored output, or null.
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, int col,
-                                               const uint32_t (&r)[32], const RowIn& in) {
+                                               const uint32_t (&r)[32], const RowIn& in,
+                                               const LnRow& ln, StatAcc* sa, bool first) {
   float v[32];
   if constexpr (EPI == kEpiInt8Deq) {
     const float rs = __ldg(e.row_scale + row);
@@ -235,6 +287,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += b[j];
     }
+  } else if constexpr (epi_ln_fold(EPI)) {
+    float c[32], dv[32];
+    load_f32x32(e.fold_c + col, c);
+    load_f32x32(e.bias_f32 + col, dv);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = fmaf(ln.rstd, fmaf(-ln.mu, c[j], __uint_as_float(r[j])), dv[j]);
   } else {
     float b[32];
     load_bf16x32(e.bias + col, b);
@@ -242,11 +301,11 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + b[j];
   }
 
-  if constexpr (EPI == kEpiGelu) {
+  if constexpr (epi_base(EPI) == kEpiGelu) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
   }
-  if constexpr (EPI == kEpiRope) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {  // 2 pairs per float4 (cos0, sin0, cos1, sin1)
@@ -274,7 +333,15 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
       }
     }
   }
-  store_bf16x32(dst, v);
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  if constexpr (EPI == kEpiGateResid) {
+    if (sa != nullptr) stat_add(*sa, pk, first);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
 // Stream-K slot of a unit: BN / 4 column groups of 128 rows, so that the 32 rows of a warp
@@ -328,6 +395,12 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
   const bool valid = row < p.M;
   const bool has_part = src_lo < src_hi;
   const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
+  LnRow ln{0.f, 1.f};
+  if constexpr (epi_ln_fold(EPI)) {
+    if (valid) ln = ln_row(p.epi, row);
+  }
+  StatAcc sa{0.f, 0.f, 0.f};
+  const bool want_stats = EPI == kEpiGateResid && BN == 256 && p.epi.stats_out != nullptr;
   RowIn in[2];
   uint4 part[2][8];
   if (valid) load_row_in<EPI>(p.epi, row, col0, in[0]);
@@ -358,8 +431,12 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
         add_part<INT8>(r, more);
       }
     }
-    if (valid) epilogue_chunk<EPI>(p.epi, row, col0 + c * 32, r, in[c & 1]);
+    if (valid)
+      epilogue_chunk<EPI>(p.epi, row, col0 + c * 32, r, in[c & 1], ln,
+                          want_stats ? &sa : nullptr, c == 0);
   }
+  if (want_stats && valid)
+    p.epi.stats_out[size_t(row) * (p.epi.ld_out / 256) + col0 / 256] = stat_final(sa);
 }
 
 // ---------------------------------------------------------------- staged pair epilogue
@@ -392,6 +469,9 @@ __device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, f
     if constexpr (EPI == kEpiInt8Deq) {
       vec[kVecBias + i] = e.bias_f32 ? __ldg(e.bias_f32 + col) : 0.0f;
       vec[kVecScale + i] = __ldg(e.col_scale + col);
+    } else if constexpr (epi_ln_fold(EPI)) {
+      vec[kVecBias + i] = __ldg(e.bias_f32 + col);   // dv
+      vec[kVecScale + i] = __ldg(e.fold_c + col);    // c
     } else {
       const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(e.bias) + col);
       vec[kVecBias + i] = __uint_as_float(b << 16);
@@ -416,7 +496,7 @@ __device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, i
                             : make_uint4(0u, 0u, 0u, 0u);  // coherent: this kernel rewrites it
     }
   }
-  if constexpr (EPI == kEpiRope) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
       const int half = e.head_dim >> 1;
       const int pair0 = (col % e.head_dim) >> 1;
@@ -433,12 +513,14 @@ __device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, i
 }
 
 // Epilogue of one 32 x 32 chunk held one row per lane (lane L: row row0 + L, columns col +
-// [0, 32)); vec points at the chunk's first column in the staged vectors.
+// [0, 32)); vec points at the chunk's first column in the staged vectors.  ln: this lane's
+// row statistics (LN-folded kinds); sa: its running output statistics, or null.
 template <int EPI>
 __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, int nrows,
                                                int col, const uint32_t (&r)[32],
                                                const RowIn& in, uint4* blk, const float* vec,
-                                               int lane) {
+                                               int lane, const LnRow& ln, StatAcc* sa,
+                                               bool first) {
   const bool valid = lane < nrows;
   float v[32];
   if constexpr (EPI == kEpiInt8Deq) {
@@ -458,15 +540,20 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += vec[kVecBias + j];
     }
+  } else if constexpr (epi_ln_fold(EPI)) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = fmaf(ln.rstd, fmaf(-ln.mu, vec[kVecScale + j], __uint_as_float(r[j])),
+                  vec[kVecBias + j]);
   } else {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + vec[kVecBias + j];
   }
-  if constexpr (EPI == kEpiGelu) {
+  if constexpr (epi_base(EPI) == kEpiGelu) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
   }
-  if constexpr (EPI == kEpiRope) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
       __syncwarp();
 #pragma unroll
@@ -508,12 +595,16 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
       }
     }
   }
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  if constexpr (EPI == kEpiGateResid) {
+    if (sa != nullptr) stat_add(*sa, pk, first);
+  }
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    blk[blk16(lane, i)] =
-        make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                   pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+    blk[blk16(lane, i)] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
   __syncwarp();
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -539,6 +630,12 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
   const int nrows = p.M - row0;
   const bool has_part = src_lo < src_hi;
   const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
+  LnRow ln{0.f, 1.f};
+  if constexpr (epi_ln_fold(EPI)) {
+    if (lane < nrows) ln = ln_row(p.epi, row0 + lane);
+  }
+  StatAcc sa{0.f, 0.f, 0.f};
+  const bool want_stats = EPI == kEpiGateResid && BN == 256 && p.epi.stats_out != nullptr;
   RowIn in[2];
   uint4 part[2][8];
   load_block_in<EPI>(p.epi, row0, nrows, col0, lane, in[0]);
@@ -570,8 +667,10 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
       }
     }
     epilogue_block<EPI>(p.epi, row0, nrows, col0 + c * 32, r, in[c & 1], blk, vec + c * 32,
-                        lane);
+                        lane, ln, want_stats ? &sa : nullptr, c == 0);
   }
+  if (want_stats && lane < nrows)
+    p.epi.stats_out[size_t(row0 + lane) * (p.epi.ld_out / 256) + col0 / 256] = stat_final(sa);
 }
 
 // Epilogue of the transposed pair kernel (A = weights, B = activations, so the TMEM lane
@@ -602,7 +701,8 @@ __device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_
     uint32_t v[32];
 #pragma unroll
     for (int f = 0; f < 32; ++f) v[f] = __float_as_uint(stage[lane * 32 + ((f + lane) & 31)]);
-    epilogue_block<EPI>(p.epi, row0, p.tokens - row0, feat0, v, in[c & 1], blk, vec, lane);
+    epilogue_block<EPI>(p.epi, row0, p.tokens - row0, feat0, v, in[c & 1], blk, vec, lane,
+                        LnRow{0.f, 1.f}, nullptr, false);
   }
 }
 
@@ -1365,6 +1465,10 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
     case kEpiRope: return launch_impl<BN, false, kEpiRope>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     case kEpiGateResid:
       return launch_impl<BN, false, kEpiGateResid>(ctx, A, B, M, N, K, epi, ws, wsb, s);
+    case kEpiRopeLN:
+      return launch_impl<BN, false, kEpiRopeLN>(ctx, A, B, M, N, K, epi, ws, wsb, s);
+    case kEpiGeluLN:
+      return launch_impl<BN, false, kEpiGeluLN>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
   }
 }
@@ -1458,8 +1562,13 @@ int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int
                      const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream) {
   if (M <= 0) return 0;
-  const int tile = choose_tile(M, N);
-  if (tile == kPair256 &&
+  int tile = choose_tile(M, N);
+  // Row statistics of the output need a tile that covers a whole 256-column group, and the
+  // transposed kernel spreads a token's columns over several warps: 256-wide untransposed
+  // tiles for them, and for the LN-folded kinds (row statistics read per row).
+  const bool row_stats = epi.stats_out != nullptr || epi_ln_fold(epi.kind);
+  if (epi.stats_out != nullptr) tile = M >= 256 ? kPair256 : kSingle256;
+  if (tile == kPair256 && !row_stats &&
       want_trans(ctx, M, N, K, scratch != nullptr && scratch_bytes >= kScratchBytes)) {
     int rc = 0, r = 1;
     switch (epi.kind) {
@@ -1493,6 +1602,14 @@ int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int
       case kEpiGateResid:
         done = try_pair_bf16<kEpiGateResid>(bn, ctx, A, B, M, N, K, epi, scratch,
                                             scratch_bytes, stream, &rc);
+        break;
+      case kEpiRopeLN:
+        done = try_pair_bf16<kEpiRopeLN>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                         stream, &rc);
+        break;
+      case kEpiGeluLN:
+        done = try_pair_bf16<kEpiGeluLN>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                         stream, &rc);
         break;
       default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
     }

@@ -153,6 +153,18 @@ int check_weights(const h3b_block_weights* w) {
   return H3B_OK;
 }
 
+bool has_fold(const h3b_block_weights* w) {
+  return w->w_qkv_fold && w->c_qkv && w->d_qkv && w->w_fc1_fold && w->c_fc1 && w->d_fc1;
+}
+
+int check_fold(const h3b_block_weights* w) {
+  if (!has_fold(w)) return set_error(H3B_EINVAL, "folded block weights missing");
+  const void* p[6] = {w->w_qkv_fold, w->c_qkv, w->d_qkv, w->w_fc1_fold, w->c_fc1, w->d_fc1};
+  for (const void* q : p)
+    if (!al16(q)) return set_error(H3B_EINVAL, "folded weight pointer not 16-byte aligned");
+  return H3B_OK;
+}
+
 size_t activations_bytes(const h3b_dims* d, int n) {
   return a256(size_t(n) * std::max(4 * d->d, d->d_ff) * 2);
 }
@@ -230,6 +242,69 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   return H3B_OK;
 }
 
+// The block with both AdaLN LayerNorms folded into the QKV and FC1 projections: the
+// gated-residual epilogues of the out-projection and FC2 write the residual's row
+// statistics, which the next folded projection's epilogue applies (no LayerNorm pass).
+int block_forward_folded_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_weights* w,
+                              const float* mod, const float* rope_cs, int n, bf16* x,
+                              float2* stats, void* arena, cudaStream_t s) {
+  const int D = d->d;
+  const BlockBufs b = carve_block(d, n, arena);
+  int rc;
+  GemmEpilogue e;
+  e.kind = kEpiRopeLN;
+  e.bias_f32 = w->d_qkv;
+  e.fold_c = w->c_qkv;
+  e.stats_in = stats;
+  e.stats_parts = D / 256;
+  e.ln_eps = d->ln_eps;
+  e.rope_cs = rope_cs;
+  e.rope_cols = 2 * D;
+  e.head_dim = d->head_dim;
+  e.out = b.qkv;
+  e.ld_out = 3 * D;
+  if ((rc = launch_gemm_bf16(ctx, x, reinterpret_cast<const bf16*>(w->w_qkv_fold), n, 3 * D, D, e,
+                             b.gemm_scratch, gemm_scratch_bytes(), s)))
+    return rc;
+  if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, b.gemm_scratch,
+                             gemm_scratch_bytes(), s)))
+    return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGateResid;
+  e.bias = reinterpret_cast<const bf16*>(w->b_o);
+  e.gate = mod + 2 * D;
+  e.out = x;
+  e.ld_out = D;
+  e.stats_out = stats;
+  if ((rc = launch_gemm_bf16(ctx, b.attn, reinterpret_cast<const bf16*>(w->w_o), n, D, D, e,
+                             b.gemm_scratch, gemm_scratch_bytes(), s)))
+    return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGeluLN;
+  e.bias_f32 = w->d_fc1;
+  e.fold_c = w->c_fc1;
+  e.stats_in = stats;
+  e.stats_parts = D / 256;
+  e.ln_eps = d->ln_eps;
+  e.out = b.g;
+  e.ld_out = d->d_ff;
+  if ((rc = launch_gemm_bf16(ctx, x, reinterpret_cast<const bf16*>(w->w_fc1_fold), n, d->d_ff, D,
+                             e, b.gemm_scratch, gemm_scratch_bytes(), s)))
+    return rc;
+
+  e = GemmEpilogue();
+  e.kind = kEpiGateResid;
+  e.bias = reinterpret_cast<const bf16*>(w->b_fc2);
+  e.gate = mod + 5 * D;
+  e.out = x;
+  e.ld_out = D;
+  e.stats_out = stats;
+  return launch_gemm_bf16(ctx, b.g, reinterpret_cast<const bf16*>(w->w_fc2), n, D, d->d_ff, e,
+                          b.gemm_scratch, gemm_scratch_bytes(), s);
+}
+
 // Workspace of one denoise step.
 struct StepBufs {
   bf16* x_res;      // [N, d] residual stream (bf16)
@@ -237,6 +312,8 @@ struct StepBufs {
   float* rope;      // [N, hd/2, 2]
   float* rope_red;  // [N_red, hd/2, 2]
   bf16* x_red;      // [N_red, d]
+  float2* stats;    // [N, d / 256] row statistics of the residual (folded blocks)
+  float2* stats_red;  // [N_red, d / 256]
   void* arena;      // block arena sized for N tokens
   size_t total;
 };
@@ -255,9 +332,11 @@ StepBufs carve_step(const h3b_dims* d, const h3b_grid* g, bool reduce, void* ws)
   b.x_res = reinterpret_cast<bf16*>(take(n * d->d * 2));
   b.h = reinterpret_cast<bf16*>(take(n * d->d * 2));
   b.rope = reinterpret_cast<float*>(take(n * d->head_dim * 4));
+  b.stats = reinterpret_cast<float2*>(take(n * (d->d / 256) * sizeof(float2)));
   if (reduce) {
     b.rope_red = reinterpret_cast<float*>(take(nr * d->head_dim * 4));
     b.x_red = reinterpret_cast<bf16*>(take(nr * d->d * 2));
+    b.stats_red = reinterpret_cast<float2*>(take(nr * (d->d / 256) * sizeof(float2)));
   }
   b.arena = take(arena_bytes(d, static_cast<int>(n)));
   b.total = off;
@@ -284,8 +363,41 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
     return rc;
 
   std::vector<int> order;
+  bool folded = true;
   for (int i = 0; i < n_blocks; ++i)
-    if (!active || active[i]) order.push_back(i);
+    if (!active || active[i]) {
+      order.push_back(i);
+      folded = folded && has_fold(&blocks[i]);
+    }
+  if (folded && !order.empty()) {
+    // every block reads the raw residual and its row statistics (no LayerNorm pass)
+    if ((rc = launch_state_to_residual(x_state, n, D, b.x_res, b.stats, s))) return rc;
+    bf16* cur = b.x_res;
+    float2* cur_stats = b.stats;
+    int cur_n = n;
+    const float* rope = b.rope;
+    for (size_t k = 0; k < order.size(); ++k) {
+      const int blk = order[k];
+      if ((rc = block_forward_folded_impl(ctx, d, &blocks[blk], mods + size_t(blk) * 6 * D, rope,
+                                          cur_n, cur, cur_stats, b.arena, s)))
+        return rc;
+      if (may_reduce && int(k + 1) == reduce_after && k + 1 < order.size()) {
+        if ((rc = launch_token_pair(b.x_res, b.x_red, g->t, g->h, g->w, g->n_audio, D, s)))
+          return rc;
+        cur = b.x_red;
+        cur_n = n_red;
+        cur_stats = b.stats_red;
+        rope = b.rope_red;
+        if ((rc = launch_row_stats(cur, cur_n, D, cur_stats, s))) return rc;
+      }
+    }
+    if (cur == b.x_red &&
+        (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
+                                  g->w, g->n_audio, D, s)))
+      return rc;
+    return launch_final_euler(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
+                              x_state, s);
+  }
   const float* first_mod = order.empty() ? final_mod : mods + size_t(order[0]) * 6 * D;
   if ((rc = launch_ln_modulate_from_state(x_state, n, D, d->ln_eps, first_mod, first_mod + D,
                                           b.x_res, b.h, s)))
@@ -329,7 +441,9 @@ int check_step_args(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
   if ((rc = check_grid(grid, reduce_after > 0))) return rc;
   if (n_blocks < 0 || (n_blocks > 0 && !blocks)) return set_error(H3B_EINVAL, "bad block list");
   for (int i = 0; i < n_blocks; ++i)
-    if ((!active || active[i]) && (rc = check_weights(&blocks[i]))) return rc;
+    if ((!active || active[i]) &&
+        ((rc = check_weights(&blocks[i])) || (has_fold(&blocks[i]) && (rc = check_fold(&blocks[i])))))
+      return rc;
   if (!mods && n_blocks > 0) return set_error(H3B_EINVAL, "mods is NULL");
   if (!final_mod || !x_state || !al16(mods) || !al16(final_mod) || !al16(x_state))
     return set_error(H3B_EINVAL, "final_mod / x_state NULL or not 16-byte aligned");
@@ -458,6 +572,54 @@ int h3b_block_forward(const h3b_dims* dims, const h3b_block_weights* w, const fl
   return block_forward_impl(ctx, dims, w, mod, mod_next, rope_cs, n_tokens, compute_h != 0,
                             reinterpret_cast<bf16*>(x), reinterpret_cast<bf16*>(h), ws,
                             static_cast<cudaStream_t>(stream));
+}
+
+int h3b_fold_adaln(const h3b_bf16* w, const h3b_bf16* b, const float* shift, const float* scale,
+                   int n_out, int d, h3b_bf16* w_out, float* c_out, float* dv_out,
+                   void* stream) {
+  if (n_out < 0 || d <= 0 || d % 8)
+    return set_error(H3B_EINVAL, "fold_adaln: d=%d must be a positive multiple of 8", d);
+  const void* ptrs[7] = {w, b, shift, scale, w_out, c_out, dv_out};
+  for (const void* q : ptrs)
+    if (!q || !al16(q)) return set_error(H3B_EINVAL, "fold_adaln: NULL or misaligned pointer");
+  const uintptr_t w0 = reinterpret_cast<uintptr_t>(w), o0 = reinterpret_cast<uintptr_t>(w_out);
+  const uintptr_t bytes = uintptr_t(n_out) * d * 2;
+  if (w0 < o0 + bytes && o0 < w0 + bytes)
+    return set_error(H3B_EINVAL, "fold_adaln: w_out overlaps w");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_fold_adaln(reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+                           shift, scale, n_out, d, reinterpret_cast<bf16*>(w_out), c_out, dv_out,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int h3b_row_stats(const h3b_bf16* x, int n_tokens, int d, float* stats, void* stream) {
+  if (n_tokens < 0 || d <= 0 || d % 256 || d > 4096)
+    return set_error(H3B_EINVAL, "row_stats: d=%d must be a multiple of 256 <= 4096", d);
+  if (!x || !stats || !al16(x) || !al16(stats))
+    return set_error(H3B_EINVAL, "row_stats: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_row_stats(reinterpret_cast<const bf16*>(x), n_tokens, d,
+                          reinterpret_cast<float2*>(stats), static_cast<cudaStream_t>(stream));
+}
+
+int h3b_block_forward_folded(const h3b_dims* dims, const h3b_block_weights* w, const float* mod,
+                             const float* rope_cs, int n_tokens, h3b_bf16* x, float* stats,
+                             void* ws, size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_weights(w)) || (rc = check_fold(w))) return rc;
+  if (n_tokens < 0 || n_tokens > (1 << 24)) return set_error(H3B_EINVAL, "n_tokens=%d", n_tokens);
+  if (!mod || !rope_cs || !x || !stats || !al16(mod) || !al16(rope_cs) || !al16(x) || !al16(stats))
+    return set_error(H3B_EINVAL, "block_forward_folded: NULL or misaligned pointer");
+  if (!ws || !al16(ws) || ws_bytes < arena_bytes(dims, n_tokens))
+    return set_error(H3B_EWORKSPACE, "block_forward_folded: workspace of %zu bytes needed, %zu given",
+                     arena_bytes(dims, n_tokens), ws_bytes);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return block_forward_folded_impl(ctx, dims, w, mod, rope_cs, n_tokens, reinterpret_cast<bf16*>(x),
+                                   reinterpret_cast<float2*>(stats), ws,
+                                   static_cast<cudaStream_t>(stream));
 }
 
 int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,

@@ -31,7 +31,18 @@ enum GemmEpi : int {
   kEpiRope = 2,       // out = bf16(rope(acc + bias)) on columns < rope_cols
   kEpiGateResid = 3,  // out = bf16(out + gate * (acc + bias))
   kEpiInt8Deq = 4,    // int8 path: out = bf16(out + gate * (acc * row_scale * col_scale + bias))
+  // LN-folded forms: A is the raw bf16 residual x and B the AdaLN-folded weights W'
+  // (launch_fold_adaln); pre = rstd_r (acc - mean_r c_j) + dv_j with the row statistics
+  // merged from stats_in, then the base epilogue
+  kEpiRopeLN = 5,     // out = bf16(rope(pre)) on columns < rope_cols
+  kEpiGeluLN = 6,     // out = bf16(gelu_tanh(pre))
 };
+
+// The base epilogue of a kind (the LN-folded kinds share their base's arithmetic).
+__host__ __device__ constexpr int epi_base(int k) {
+  return k == kEpiRopeLN ? kEpiRope : k == kEpiGeluLN ? kEpiGelu : k;
+}
+__host__ __device__ constexpr bool epi_ln_fold(int k) { return k == kEpiRopeLN || k == kEpiGeluLN; }
 
 struct GemmEpilogue {
   int kind = kEpiBias;
@@ -46,6 +57,15 @@ struct GemmEpilogue {
   const float* row_scale = nullptr;  // int8 path, [M]
   const float* col_scale = nullptr;  // int8 path, [N]
   int32_t* acc_out = nullptr;        // int8 path, [M, N] or null
+  // kEpiGateResid: per row, (mean, M2) of each 256-column group of the stored bf16 output,
+  // [M, ld_out / 256]; or null
+  float2* stats_out = nullptr;
+  // LN-folded kinds: the A rows' group statistics [M, stats_parts], the folded weights'
+  // row sums c [N] (dv [N] comes in bias_f32) and the LayerNorm epsilon
+  const float2* stats_in = nullptr;
+  const float* fold_c = nullptr;
+  int stats_parts = 0;
+  float ln_eps = 1e-6f;
 };
 
 // Kernel scratch: one caller buffer per stream, used by one kernel at a time.  Layout:
@@ -97,6 +117,16 @@ int launch_ln_modulate(const bf16* x, int n, int d, float eps, const float* shif
 int launch_ln_modulate_from_state(const float* x_state, int n, int d, float eps,
                                   const float* shift, const float* scale, bf16* x_res,
                                   bf16* h, cudaStream_t stream);
+// x_res = bf16(x_state) and the (mean, M2) of each 256-column group of its rows,
+// stats [n, d / 256] (the row statistics the LN-folded GEMM epilogues consume)
+int launch_state_to_residual(const float* x_state, int n, int d, bf16* x_res, float2* stats,
+                             cudaStream_t stream);
+// (mean, M2) of each 256-column group of the rows of x, stats [n, d / 256]
+int launch_row_stats(const bf16* x, int n, int d, float2* stats, cudaStream_t stream);
+// W' = bf16(W diag(1 + scale)), c = row sums of W', dv = W shift + b (see k_fold_adaln)
+int launch_fold_adaln(const bf16* w, const bf16* b, const float* shift, const float* scale,
+                      int n_out, int d, bf16* w_out, float* c_out, float* d_out,
+                      cudaStream_t stream);
 int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,
                        const float* final_mod, float dt_sigma, float* x_state,
                        cudaStream_t stream);

@@ -149,6 +149,107 @@ __global__ void __launch_bounds__(128) k_final_euler(const bf16* __restrict__ xl
   }
 }
 
+// Statistics of one 256-column group of a row, held as 8 values per lane: the group's
+// mean and M2 (sum of squared deviations from it), accumulated about the group's first
+// value so that a large common offset does not cancel.  The GEMM epilogues write the
+// same (mean, M2) per group for the rows they produce; a consumer merges a row's groups.
+__device__ __forceinline__ float2 group_stats(const float (&v)[8]) {
+  const float k = __shfl_sync(0xffffffffu, v[0], 0);
+  float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float t = v[i] - k;
+    s1 += t;
+    s2 = fmaf(t, t, s2);
+  }
+  s1 = warp_sum(s1);
+  s2 = warp_sum(s2);
+  return make_float2(k + s1 * (1.0f / 256.0f), s2 - s1 * s1 * (1.0f / 256.0f));
+}
+
+// x_res = bf16(x_state) (the block input) and the (mean, M2) of each 256-column group of
+// the stored bf16 row: stats [n, D / 256].
+template <int NV>
+__global__ void __launch_bounds__(128) k_state_to_residual(const float* __restrict__ xs, int n,
+                                                           bf16* __restrict__ x_res,
+                                                           float2* __restrict__ stats) {
+  constexpr int D = NV * 256;
+  const int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int col = (i * 32 + lane) * 8;
+    float f[8], v[8];
+    load8f(xs + size_t(row) * D + col, f);
+    const uint4 u = pack8(f);
+    reinterpret_cast<uint4*>(x_res + size_t(row) * D + col)[0] = u;
+    unpack8(u, v);
+    const float2 g = group_stats(v);
+    if (lane == 0) stats[size_t(row) * NV + i] = g;
+  }
+}
+
+// (mean, M2) of each 256-column group of the bf16 rows of x: stats [n, D / 256].
+template <int NV>
+__global__ void __launch_bounds__(128) k_row_stats(const bf16* __restrict__ x, int n,
+                                                   float2* __restrict__ stats) {
+  constexpr int D = NV * 256;
+  const int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float v[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(x + size_t(row) * D + (i * 32 + lane) * 8)), v);
+    const float2 g = group_stats(v);
+    if (lane == 0) stats[size_t(row) * NV + i] = g;
+  }
+}
+
+// AdaLN folded into the projection that consumes the modulated LayerNorm output: for
+// h = LN(x)(1 + scale) + shift and y = h W^T + b,
+//   y[r, j] = rstd_r (sum_k x[r, k] W'[j, k] - mean_r c_j) + d_j,
+//   W'[j, k] = bf16(W[j, k] (1 + scale_k)),  c_j = sum_k W'[j, k],  d_j = sum_k shift_k W[j, k] + b_j.
+// One warp per output row j; c is summed over the stored (rounded) W' so that the mean
+// term cancels exactly what the tensor cores accumulate.
+__global__ void __launch_bounds__(256) k_fold_adaln(const bf16* __restrict__ w,
+                                                    const bf16* __restrict__ b,
+                                                    const float* __restrict__ shift,
+                                                    const float* __restrict__ scale, int n_out,
+                                                    int d, bf16* __restrict__ w_out,
+                                                    float* __restrict__ c_out,
+                                                    float* __restrict__ d_out) {
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (j >= n_out) return;
+  const int lane = threadIdx.x & 31;
+  const uint4* wr = reinterpret_cast<const uint4*>(w + size_t(j) * d);
+  uint4* wo = reinterpret_cast<uint4*>(w_out + size_t(j) * d);
+  float cs = 0.f, ds = 0.f;
+  for (int v = lane; v < (d >> 3); v += 32) {
+    float a[8], sh[8], sc[8], f[8], r[8];
+    unpack8(__ldg(wr + v), a);
+    load8f(shift + v * 8, sh);
+    load8f(scale + v * 8, sc);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) f[k] = fmaf(a[k], sc[k], a[k]);
+    const uint4 u = pack8(f);
+    wo[v] = u;
+    unpack8(u, r);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      cs += r[k];
+      ds = fmaf(sh[k], a[k], ds);
+    }
+  }
+  cs = warp_sum(cs);
+  ds = warp_sum(ds);
+  if (lane == 0) {
+    c_out[j] = cs;
+    d_out[j] = ds + __bfloat162float(b[j]);
+  }
+}
+
 // Pairing: reduced video token r averages full tokens 2r and 2r + 1 (w is even, so the
 // horizontal neighbours (t, h, 2j), (t, h, 2j+1) are consecutive rows).
 __global__ void k_token_pair(const bf16* __restrict__ src, bf16* __restrict__ dst, int nv_red,
@@ -363,6 +464,31 @@ int launch_ln_modulate_from_state(const float* x_state, int n, int d, float eps,
   H3B_NV_SWITCH(d / 256, (k_ln_modulate<NV, true><<<grid, 32 * kRowWarps, 0, stream>>>(
                              x_state, n, eps, shift, scale, x_res, h)));
   return check_launch("ln_modulate_from_state");
+}
+
+int launch_state_to_residual(const float* x_state, int n, int d, bf16* x_res, float2* stats,
+                             cudaStream_t stream) {
+  if (n <= 0) return 0;
+  const int grid = (n + kRowWarps - 1) / kRowWarps;
+  H3B_NV_SWITCH(d / 256, (k_state_to_residual<NV><<<grid, 32 * kRowWarps, 0, stream>>>(
+                             x_state, n, x_res, stats)));
+  return check_launch("state_to_residual");
+}
+
+int launch_row_stats(const bf16* x, int n, int d, float2* stats, cudaStream_t stream) {
+  if (n <= 0) return 0;
+  const int grid = (n + kRowWarps - 1) / kRowWarps;
+  H3B_NV_SWITCH(d / 256, (k_row_stats<NV><<<grid, 32 * kRowWarps, 0, stream>>>(x, n, stats)));
+  return check_launch("row_stats");
+}
+
+int launch_fold_adaln(const bf16* w, const bf16* b, const float* shift, const float* scale,
+                      int n_out, int d, bf16* w_out, float* c_out, float* d_out,
+                      cudaStream_t stream) {
+  if (n_out <= 0) return 0;
+  const int grid = (n_out + 7) / 8;
+  k_fold_adaln<<<grid, 256, 0, stream>>>(w, b, shift, scale, n_out, d, w_out, c_out, d_out);
+  return check_launch("fold_adaln");
 }
 
 int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,

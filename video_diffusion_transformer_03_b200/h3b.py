@@ -38,9 +38,12 @@ class Grid(ctypes.Structure):
                 ("n_audio", ctypes.c_int), ("rope_halved", ctypes.c_int)]
 
 
+WEIGHT_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")
+FOLD_FIELDS = ("w_qkv_fold", "c_qkv", "d_qkv", "w_fc1_fold", "c_fc1", "d_fc1")
+
+
 class BlockWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in
-                ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS + FOLD_FIELDS]
 
 
 _P = ctypes.c_void_p
@@ -65,6 +68,10 @@ _SIGS = {
                                _I, _I, _P, _P, _P, _SZ, _P]),
     "h3b_block_forward_noalloc": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _P,
                                        _P, _P, _I, _I, _P, _P, _P]),
+    "h3b_fold_adaln": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
+    "h3b_row_stats": (_I, [_P, _I, _I, _P, _P]),
+    "h3b_block_forward_folded": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights), _P, _P,
+                                      _I, _P, _P, _P, _SZ, _P]),
     "h3b_final_euler": (_I, [_P, _I, _I, _I, _F, _P, _F, _F, _P, _P]),
     "h3b_denoise_step": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                               ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P, _P,
@@ -149,11 +156,16 @@ def make_grid(t, h, w, n_audio, rope_halved=False) -> Grid:
 
 def make_block_weights(p) -> BlockWeights:
     """p: mapping with the eight bf16 CUDA tensors w_qkv, b_qkv, w_o, b_o, w_fc1, b_fc1,
-    w_fc2, b_fc2."""
-    for k in ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2"):
+    w_fc2, b_fc2, and optionally the six folded ones (fold_block): w_qkv_fold, w_fc1_fold
+    (bf16) and c_qkv, d_qkv, c_fc1, d_fc1 (fp32)."""
+    for k in WEIGHT_FIELDS:
         _dev(p[k], torch.bfloat16, k)
-    return BlockWeights(*[_ptr(p[k]) for k in
-                          ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")])
+    folded = all(k in p for k in FOLD_FIELDS)
+    if folded:
+        for k in FOLD_FIELDS:
+            _dev(p[k], torch.bfloat16 if k.startswith("w_") else torch.float32, k)
+    return BlockWeights(*[_ptr(p[k]) for k in WEIGHT_FIELDS],
+                        *[_ptr(p[k]) if folded else None for k in FOLD_FIELDS])
 
 
 def gemm_workspace_size() -> int:
@@ -248,6 +260,44 @@ def block_forward(dims: Dims, weights: BlockWeights, mod, mod_next, rope_cs, x, 
                                  _ptr(mod_next), _ptr(rope_cs), x.shape[0], int(bool(compute_h)),
                                  _ptr(x), _ptr(h), _ptr(ws), ws.numel() * ws.element_size(),
                                  _stream(stream)))
+
+
+def fold_adaln(w, b, shift, scale, w_out, c_out, d_out, stream=None) -> None:
+    """W' = bf16(W diag(1 + scale)), c = row sums of W', d = W shift + b (h3b_fold_adaln)."""
+    _dev(w, torch.bfloat16, "w"); _dev(b, torch.bfloat16, "b"); _dev(w_out, torch.bfloat16, "w_out")
+    _dev(shift, torch.float32, "shift"); _dev(scale, torch.float32, "scale")
+    _dev(c_out, torch.float32, "c_out"); _dev(d_out, torch.float32, "d_out")
+    n_out, d = w.shape
+    _check(lib.h3b_fold_adaln(_ptr(w), _ptr(b), _ptr(shift), _ptr(scale), n_out, d, _ptr(w_out),
+                              _ptr(c_out), _ptr(d_out), _stream(stream)))
+
+
+def fold_block(p, mod, stream=None):
+    """The folded fields of one block (device tensors) from its weights p and its AdaLN
+    vectors mod [6, d]: (shift_msa, scale_msa) into w_qkv, (shift_mlp, scale_mlp) into w_fc1."""
+    out = {}
+    for name, sh, sc in (("qkv", 0, 1), ("fc1", 3, 4)):
+        w, b = p["w_" + name], p["b_" + name]
+        out["w_%s_fold" % name] = torch.empty_like(w)
+        out["c_" + name] = torch.empty(w.shape[0], dtype=torch.float32, device=w.device)
+        out["d_" + name] = torch.empty(w.shape[0], dtype=torch.float32, device=w.device)
+        fold_adaln(w, b, mod[sh].contiguous(), mod[sc].contiguous(), out["w_%s_fold" % name],
+                   out["c_" + name], out["d_" + name], stream)
+    return out
+
+
+def row_stats(x, stats, stream=None) -> None:
+    """stats [n, d / 256, 2] fp32: per row and 256-column group, (mean, M2) of x."""
+    _dev(x, torch.bfloat16, "x"); _dev(stats, torch.float32, "stats")
+    _check(lib.h3b_row_stats(_ptr(x), x.shape[0], x.shape[1], _ptr(stats), _stream(stream)))
+
+
+def block_forward_folded(dims: Dims, weights: BlockWeights, mod, rope_cs, x, stats, ws,
+                         stream=None) -> None:
+    _dev(x, torch.bfloat16, "x"); _dev(stats, torch.float32, "stats"); _dev(mod, torch.float32, "mod")
+    _check(lib.h3b_block_forward_folded(ctypes.byref(dims), ctypes.byref(weights), _ptr(mod),
+                                        _ptr(rope_cs), x.shape[0], _ptr(x), _ptr(stats), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)))
 
 
 NOALLOC_WORKSPACE_BYTES = 64 << 20

@@ -26,9 +26,14 @@ def grid_of(cfg: DiTConfig) -> h3b.Grid:
 
 
 class DiTDenoiser:
+    """fold=True (default) folds each block's two AdaLN modulations into its QKV and FC1
+    weights once (h3b_fold_adaln), so the step runs without LayerNorm passes; fold=False
+    keeps the LayerNorm + AdaLN kernel between the projections."""
+
     def __init__(self, cfg: DiTConfig, device: str = "cuda", gen_device: str = "cpu",
-                 keep_host_params: bool = False):
+                 keep_host_params: bool = False, fold: bool = True):
         self.cfg = cfg
+        self.fold = fold
         self.device = torch.device(device)
         self.dims = dims_of(cfg)
         self.grid = grid_of(cfg)
@@ -43,6 +48,8 @@ class DiTDenoiser:
             pd = {k: v.to(self.device) for k, v in p.items()}
             del p
             h3b.adaln_modulation(pd.pop("w_ada"), pd.pop("b_ada"), self.c, self.mods[b])
+            if fold:
+                pd.update(h3b.fold_block(pd, self.mods[b]))
             self.params.append(pd)
         self.weights = [h3b.make_block_weights(p) for p in self.params]
         fin = synth.final_params(cfg, gen_device)
