@@ -419,3 +419,87 @@ def fc2_int8_row(act, w_q, w_scale, gate, resid, bias=None, rows=None):
         y = y + np.asarray(bias, F64)[None, :]
     out = np.asarray(resid, F64) + np.asarray(gate, F64)[None, :] * y
     return q, s_r, acc, out
+
+
+# --------------------------------------------------------------------------------------
+# reuse policies: whole-velocity reuse and core-residual reuse
+# --------------------------------------------------------------------------------------
+def reuse_schedule(steps: int, every: int) -> np.ndarray:
+    """Which Euler steps evaluate the model when only every `every`-th one does.
+
+    [aihot] section 4 and [dothoosh] "Aggressive optimisation levers": at 20 steps,
+    reuse 1, 2 and 3 evaluate the denoiser 20, 11 and 8 times.  Reading that fits those
+    counts: step i is fresh when i % every == 0, and the last step is always fresh."""
+    i = np.arange(steps)
+    return (i % every == 0) | (i == steps - 1)
+
+
+def denoise_velocity_reuse(x0, blocks, mods, final_mod, grid, n_audio: int, n_heads: int,
+                           split, theta: float, eps: float, steps: int, reuse: int,
+                           active=None, reduce_after: int = -1, halved: bool = False,
+                           unpair_bypass: bool = True, dt=F64) -> np.ndarray:
+    """Euler loop with whole-velocity reuse ([dothoosh] "Aggressive optimisation levers":
+    the skipped transitions are extrapolated).  Reading: a fresh step runs the model and
+    keeps its velocity; a skipped step takes the Euler transition with the velocity of the
+    last fresh step."""
+    fresh = reuse_schedule(steps, reuse)
+    sig = sigma_grid(steps, dt)
+    x_state = np.asarray(x0, dt)
+    v = None
+    for i in range(steps):
+        if fresh[i]:
+            x_l = _core(x_state, blocks, mods, grid, n_audio, n_heads, split, theta, eps,
+                        active, reduce_after, halved, unpair_bypass, dt)
+            v = final_adaln(x_l, final_mod, grid[0] * grid[1] * grid[2], eps, dt)
+        x_state = euler_update(x_state, v, sig[i], sig[i + 1], dt)
+    return x_state
+
+
+def denoise_core_reuse(x0, blocks, mods, final_mod, grid, n_audio: int, n_heads: int,
+                       split, theta: float, eps: float, steps: int, reuse: int,
+                       active=None, reduce_after: int = -1, halved: bool = False,
+                       unpair_bypass: bool = True, dt=F64) -> np.ndarray:
+    """Euler loop with core-residual reuse ([aihot] section 4, [dothoosh] "Aggressive
+    optimisation levers": the work around the core is refreshed every step, the expensive
+    core runs less often).  Reading: the core is the stack of DiT blocks, with residual
+    r = x_L - x_in; a fresh step (same schedule as reuse_schedule) runs the core and keeps
+    r; a skipped step takes x_L = bf16(x_in + r) with its own x_in = bf16(x_state), and
+    the final AdaLN and the Euler update run every step."""
+    fresh = reuse_schedule(steps, reuse)
+    sig = sigma_grid(steps, dt)
+    x_state = np.asarray(x0, dt)
+    nv = grid[0] * grid[1] * grid[2]
+    r = None
+    for i in range(steps):
+        x_in = round_to_bf16(x_state).astype(dt)
+        if fresh[i]:
+            x_l = _core(x_state, blocks, mods, grid, n_audio, n_heads, split, theta, eps,
+                        active, reduce_after, halved, unpair_bypass, dt)
+            r = x_l - x_in
+        else:
+            x_l = round_to_bf16(x_in + r).astype(dt)
+        v = final_adaln(x_l, final_mod, nv, eps, dt)
+        x_state = euler_update(x_state, v, sig[i], sig[i + 1], dt)
+    return x_state
+
+
+def _core(x_state, blocks, mods, grid, n_audio, n_heads, split, theta, eps, active,
+          reduce_after, halved, unpair_bypass, dt):
+    """The block stack of one Euler step on bf16(x_state): the same sequence as one step
+    of denoise() up to (not including) the final AdaLN."""
+    nb = len(blocks)
+    act = np.ones(nb, bool) if active is None else np.asarray(active, bool)
+    order = [b for b in range(nb) if act[b]]
+    pos = rope_positions(grid, n_audio, halved=halved, dt=dt)
+    pos_red = rope_positions(grid, n_audio, halved=halved, paired=True, dt=dt)
+    x = round_to_bf16(x_state).astype(dt)
+    saved = None
+    for n_exec, b in enumerate(order, start=1):
+        x, _ = block_forward(x, blocks[b], mods[b], pos, n_heads, split, theta, eps, dt=dt)
+        if n_exec == reduce_after and n_exec < len(order):
+            saved = x
+            x = token_pair(x, grid, n_audio, dt)
+            pos = pos_red
+    if saved is not None:
+        x = token_unpair(x, grid, n_audio, saved if unpair_bypass else None, dt)
+    return x

@@ -1,6 +1,7 @@
 """Pins of the CPU oracle against things other than itself: closed forms, brute force on
 tiny inputs, library routines, invariants and exact identities.  No GPU needed."""
 import math
+import os
 
 import numpy as np
 import pytest
@@ -584,3 +585,97 @@ def test_denoise_comparison_catches_planted_mistakes(mistake, monkeypatch):
                             real_unpair(xr, g, n, None, dt))
     got = _oracle_denoise_2(blocks, mods, fm, grid, na, x0, **kw)
     assert np.max(np.abs(got - want)) > 1e-4
+
+
+# ----------------------------------------------------------------------------- reuse policies
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def test_reuse_schedule_matches_the_pages_counts():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "reuse_counts.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 3
+    for steps, reuse, fresh in rows:
+        assert int(O.reuse_schedule(int(steps), int(reuse)).sum()) == int(fresh)
+    s = O.reuse_schedule(7, 3)
+    assert s.tolist() == [True, False, False, True, False, False, True]
+    assert O.reuse_schedule(5, 1).all()
+
+
+def _torch_denoise_reuse(x0, blocks, mods, fm, grid, n_audio, steps, reuse, mode):
+    """Independent composition of the two reuse loops from _torch_block and torch ops."""
+    a = _DENOISE_ARGS
+    nv = grid[0] * grid[1] * grid[2]
+    pos = _grid_positions(grid, n_audio, False).numpy()
+    fmt = torch.from_numpy(np.asarray(fm, np.float64))
+    x_state = torch.from_numpy(np.asarray(x0, np.float64))
+    held = None
+    for i in range(steps):
+        fresh = i % reuse == 0 or i == steps - 1
+        x_in = x_state.to(torch.bfloat16).to(torch.float64)
+        if fresh:
+            x = x_in
+            for b in range(len(blocks)):
+                x = torch.from_numpy(_torch_block(x.numpy(), blocks[b], mods[b], pos,
+                                                  a["heads"], a["split"], a["theta"], a["eps"]))
+            x_l = x
+            if mode == "core":
+                held = x_l - x_in
+        elif mode == "core":
+            x_l = (x_in + held).to(torch.bfloat16).to(torch.float64)
+        if fresh or mode == "core":
+            xn = F.layer_norm(x_l, (x_l.shape[1],), eps=a["eps"])
+            v = torch.cat([xn[:nv] * (1 + fmt[0, 1]) + fmt[0, 0],
+                           xn[nv:] * (1 + fmt[1, 1]) + fmt[1, 0]])
+            if mode == "velocity":
+                held = v
+        else:
+            v = held
+        x_state = x_state + ((1.0 - (i + 1) / steps) - (1.0 - i / steps)) * v
+    return x_state.numpy()
+
+
+@pytest.mark.parametrize("mode", ["velocity", "core"])
+@pytest.mark.parametrize("steps,reuse", [(5, 2), (7, 3), (4, 1)])
+def test_reuse_loops_match_independent_composition(mode, steps, reuse):
+    blocks, mods, fm, grid, na, x0 = _denoise_case(n_blocks=2)
+    a = _DENOISE_ARGS
+    fn = O.denoise_velocity_reuse if mode == "velocity" else O.denoise_core_reuse
+    got = fn(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"], a["eps"],
+             steps, reuse)
+    want = _torch_denoise_reuse(x0, blocks, mods, fm, grid, na, steps, reuse, mode)
+    assert np.max(np.abs(got - want)) < 1e-10
+
+
+@pytest.mark.parametrize("mode", ["velocity", "core"])
+def test_reuse_one_is_the_plain_loop(mode):
+    blocks, mods, fm, grid, na, x0 = _denoise_case(n_blocks=3)
+    a = _DENOISE_ARGS
+    fn = O.denoise_velocity_reuse if mode == "velocity" else O.denoise_core_reuse
+    kw = dict(active=[1, 0, 1], reduce_after=1)
+    got = fn(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"], a["eps"],
+             4, 1, **kw)
+    want = O.denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                     a["eps"], steps=4, run_steps=4, **kw)
+    assert np.array_equal(got, want)
+
+
+def test_reuse_closed_forms():
+    blocks, mods, fm, grid, na, x0 = _denoise_case(n_blocks=2)
+    a = _DENOISE_ARGS
+    args = (grid, na, a["heads"], a["split"], a["theta"], a["eps"])
+    # constant velocity (final scale -1): every policy follows the same trajectory
+    fc = np.zeros_like(fm)
+    fc[:, 1] = -1
+    fc[0, 0], fc[1, 0] = 0.7, -0.4
+    base = O.denoise(x0, blocks, mods, fc, *args, steps=6, run_steps=6)
+    for fn in (O.denoise_velocity_reuse, O.denoise_core_reuse):
+        assert np.allclose(fn(x0, blocks, mods, fc, *args, 6, 3), base, atol=1e-12)
+    # identity core (zero gates): the core residual is zero, so core reuse is exact
+    mz = mods.copy()
+    mz[:, 2] = 0
+    mz[:, 5] = 0
+    full = O.denoise(x0, blocks, mz, fm, *args, steps=6, run_steps=6)
+    assert np.array_equal(O.denoise_core_reuse(x0, blocks, mz, fm, *args, 6, 4), full)
+    # ... while velocity reuse holds a stale velocity and departs from it
+    assert np.max(np.abs(O.denoise_velocity_reuse(x0, blocks, mz, fm, *args, 6, 4) - full)) > 1e-3
