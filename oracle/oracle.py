@@ -149,6 +149,21 @@ def rope_rotate(x, pos, split: Sequence[int], theta: float, dt=F64) -> np.ndarra
 
 
 # --------------------------------------------------------------------------------------
+# f2: Q/K RMSNorm (before RoPE)
+# --------------------------------------------------------------------------------------
+def rms_norm(x, gain, eps: float, dt=F64) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gain.
+
+    Applied to each head of q and k inside the QKV projection's tile, before the rotation
+    ([dothoosh] "The powerful int8 path": RMS normalisation and RoPE for Q/K in the QKV
+    tile).  Reading: per head over the head dimension, one learned gain vector [hd] for q
+    and one for k, shared by the heads; eps as the LayerNorm's."""
+    x = np.asarray(x, dt)
+    ms = (x * x).mean(axis=-1, keepdims=True)
+    return x / np.sqrt(ms + dt(eps)) * np.asarray(gain, dt)
+
+
+# --------------------------------------------------------------------------------------
 # a5: joint self-attention
 # --------------------------------------------------------------------------------------
 def attention(q, k, v, q_rows: Optional[np.ndarray] = None, dt=F64) -> np.ndarray:
@@ -191,7 +206,8 @@ def block_forward(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int,
 
     Steps in the pages' order ([dothoosh] "DiT fusions and memory management"):
       h  = LN(x) (1 + scale_msa) + shift_msa
-      q, k, v = split(h W_qkv^T + b_qkv); q, k rotated by 3D RoPE
+      q, k, v = split(h W_qkv^T + b_qkv); q, k rotated by 3D RoPE (after a per-head
+                RMSNorm with gains w["q_norm"], w["k_norm"] when the block has them)
       o  = attention(q, k, v)
       x1 = x + gate_msa (o W_o^T + b_o)           (attention gate -> MLP AdaLN)
       h2 = LN(x1) (1 + scale_mlp) + shift_mlp
@@ -212,10 +228,14 @@ def block_forward(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int,
     b_qkv = np.asarray(w["b_qkv"], dt)
     # keys and values for every token, queries for the selected ones
     kv = h @ w_qkv[d:].T + b_qkv[d:]
-    k = rope_rotate(kv[:, :d].reshape(n, n_heads, hd), pos, split, theta, dt)
+    k = kv[:, :d].reshape(n, n_heads, hd)
     v = kv[:, d:].reshape(n, n_heads, hd)
-    q = h[sel] @ w_qkv[:d].T + b_qkv[:d]
-    q = rope_rotate(q.reshape(len(sel), n_heads, hd), np.asarray(pos)[sel], split, theta, dt)
+    q = (h[sel] @ w_qkv[:d].T + b_qkv[:d]).reshape(len(sel), n_heads, hd)
+    if w.get("q_norm") is not None:
+        q = rms_norm(q, w["q_norm"], eps, dt)
+        k = rms_norm(k, w["k_norm"], eps, dt)
+    k = rope_rotate(k, pos, split, theta, dt)
+    q = rope_rotate(q, np.asarray(pos)[sel], split, theta, dt)
     o = attention(q, k, v, dt=dt).reshape(len(sel), d)
 
     x1 = gated_residual(x[sel], mod[2], o @ np.asarray(w["w_o"], dt).T + np.asarray(w["b_o"], dt), dt)

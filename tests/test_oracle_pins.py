@@ -679,3 +679,66 @@ def test_reuse_closed_forms():
     assert np.array_equal(O.denoise_core_reuse(x0, blocks, mz, fm, *args, 6, 4), full)
     # ... while velocity reuse holds a stale velocity and departs from it
     assert np.max(np.abs(O.denoise_velocity_reuse(x0, blocks, mz, fm, *args, 6, 4) - full)) > 1e-3
+
+
+# ----------------------------------------------------------------------------- Q/K RMSNorm
+def test_rms_norm_closed_form_and_torch():
+    out = O.rms_norm(np.array([[3.0, 4.0]]), np.ones(2), 0.0)
+    r = math.sqrt(12.5)
+    assert np.allclose(out, [[3 / r, 4 / r]], atol=1e-15)
+    x = RNG.standard_normal((7, 3, 128)) * 2.5
+    g = 1 + RNG.standard_normal(128) * 0.1
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (128,), torch.from_numpy(g),
+                                       eps=1e-6).numpy()
+    assert np.max(np.abs(O.rms_norm(x, g, 1e-6) - ref)) < 1e-13
+    # scale invariance and unit mean square with unit gains
+    assert np.allclose(O.rms_norm(5.0 * x, g, 0.0), O.rms_norm(x, g, 0.0), atol=1e-13)
+    y = O.rms_norm(x, np.ones(128), 0.0)
+    assert np.allclose((y * y).mean(axis=-1), 1.0, atol=1e-13)
+
+
+def _torch_block_qk(x, w, mod, pos, heads, split, theta, eps):
+    """_torch_block with torch's rms_norm on each head of q and k before the rotation."""
+    F_ = torch.nn.functional
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    xt, m = t(x), t(mod)
+    n, d = xt.shape
+    hd = d // heads
+    h = F_.layer_norm(xt, (d,), eps=eps) * (1 + m[1]) + m[0]
+    qkv = F_.linear(h, t(w["w_qkv"]), t(w["b_qkv"]))
+    q, k, v = (qkv[:, i * d:(i + 1) * d].reshape(n, heads, hd) for i in range(3))
+    q = F_.rms_norm(q, (hd,), t(w["q_norm"]), eps=eps)
+    k = F_.rms_norm(k, (hd,), t(w["k_norm"]), eps=eps)
+    ang = []
+    for axis, width in enumerate(split):
+        kk = torch.arange(width // 2, dtype=torch.float64)
+        ang.append(t(pos)[:, axis:axis + 1] * theta ** (-2.0 * kk / width))
+    rot = torch.polar(torch.ones(n, hd // 2, dtype=torch.float64), torch.cat(ang, 1))[:, None]
+
+    def rope(a):
+        z = torch.view_as_complex(a.reshape(n, heads, hd // 2, 2).contiguous())
+        return torch.view_as_real(z * rot).reshape(n, heads, hd)
+
+    o = F_.scaled_dot_product_attention(rope(q).transpose(0, 1), rope(k).transpose(0, 1),
+                                        v.transpose(0, 1)).transpose(0, 1).reshape(n, d)
+    x1 = xt + m[2] * F_.linear(o, t(w["w_o"]), t(w["b_o"]))
+    h2 = F_.layer_norm(x1, (d,), eps=eps) * (1 + m[4]) + m[3]
+    g = F_.gelu(F_.linear(h2, t(w["w_fc1"]), t(w["b_fc1"])), approximate="tanh")
+    return (x1 + m[5] * F_.linear(g, t(w["w_fc2"]), t(w["b_fc2"]))).numpy()
+
+
+def test_block_with_qk_norm_vs_torch_composition():
+    w, mod = _tiny_block(seed=31)
+    r = np.random.default_rng(32)
+    w["q_norm"] = 1 + r.standard_normal(32) * 0.1
+    w["k_norm"] = 1 + r.standard_normal(32) * 0.1
+    grid = (2, 3, 4)
+    x = RNG.standard_normal((24 + 5, 64))
+    pos = O.rope_positions(grid, 5)
+    out, _ = O.block_forward(x, w, mod, pos, 2, (8, 12, 12), 1e4, 1e-6)
+    ref = _torch_block_qk(x, w, mod, pos, 2, (8, 12, 12), 1e4, 1e-6)
+    assert np.max(np.abs(out - ref)) < 1e-12
+    # the norm matters: without it the block differs
+    w0 = {k: v for k, v in w.items() if k not in ("q_norm", "k_norm")}
+    plain, _ = O.block_forward(x, w0, mod, pos, 2, (8, 12, 12), 1e4, 1e-6)
+    assert np.max(np.abs(plain - out)) > 1e-3
