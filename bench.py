@@ -258,26 +258,55 @@ def time_kernels(model, cfg, peaks, counts_per_step, reps=20, only=None, warm=3)
     P = model.params
     nb = len(P)
     ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
+    st = torch.empty((n, d // 256, 2), dtype=torch.float32, device=dev)
+    h3b.row_stats(x, st)
+    if model.fold:
+        # the kernels of the folded block: projections that read the raw residual and its
+        # row statistics, gated-residual epilogues that write the statistics
+        gemms = {
+            "gemm_qkv_rope": (lambda i: h3b.gemm_bf16_ln(
+                x, P[i % nb]["w_qkv_fold"], h3b.EPI_LN_ROPE, qkv, fold_c=P[i % nb]["c_qkv"],
+                fold_dv=P[i % nb]["d_qkv"], stats_in=st, ln_eps=cfg.ln_eps, rope_cs=cs,
+                rope_cols=2 * d, head_dim=hd, ws=ws), "tensor", 2 * n * d * 3 * d),
+            "gemm_out_gate": (lambda i: h3b.gemm_bf16_ln(
+                attn, P[i % nb]["w_o"], h3b.EPI_GATE_RESID, x, bias=P[i % nb]["b_o"],
+                gate=mod[2], stats_out=st, ws=ws), "tensor", 2 * n * d * d),
+            "gemm_fc1_gelu": (lambda i: h3b.gemm_bf16_ln(
+                x, P[i % nb]["w_fc1_fold"], h3b.EPI_LN_GELU, gbuf, fold_c=P[i % nb]["c_fc1"],
+                fold_dv=P[i % nb]["d_fc1"], stats_in=st, ln_eps=cfg.ln_eps, ws=ws),
+                "tensor", 2 * n * d * f),
+            "gemm_fc2_gate": (lambda i: h3b.gemm_bf16_ln(
+                gbuf, P[i % nb]["w_fc2"], h3b.EPI_GATE_RESID, x, bias=P[i % nb]["b_fc2"],
+                gate=mod[5], stats_out=st, ws=ws), "tensor", 2 * n * f * d),
+        }
+    else:
+        gemms = {
+            "gemm_qkv_rope": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_qkv"], h3b.EPI_BIAS_ROPE,
+                                                      P[i % nb]["b_qkv"], qkv, rope_cs=cs,
+                                                      rope_cols=2 * d, head_dim=hd, ws=ws),
+                              "tensor", 2 * n * d * 3 * d),
+            "gemm_out_gate": (lambda i: h3b.gemm_bf16(attn, P[i % nb]["w_o"], h3b.EPI_GATE_RESID,
+                                                      P[i % nb]["b_o"], x, gate=mod[2], ws=ws),
+                              "tensor", 2 * n * d * d),
+            "gemm_fc1_gelu": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_fc1"], h3b.EPI_BIAS_GELU,
+                                                      P[i % nb]["b_fc1"], gbuf, ws=ws),
+                              "tensor", 2 * n * d * f),
+            "gemm_fc2_gate": (lambda i: h3b.gemm_bf16(gbuf, P[i % nb]["w_fc2"], h3b.EPI_GATE_RESID,
+                                                      P[i % nb]["b_fc2"], x, gate=mod[5], ws=ws),
+                              "tensor", 2 * n * f * d),
+        }
     kinds = {
-        "gemm_qkv_rope": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_qkv"], h3b.EPI_BIAS_ROPE,
-                                                  P[i % nb]["b_qkv"], qkv, rope_cs=cs,
-                                                  rope_cols=2 * d, head_dim=hd, ws=ws),
-                          "tensor", 2 * n * d * 3 * d),
+        "gemm_qkv_rope": gemms["gemm_qkv_rope"],
         "attention": (lambda i: h3b.attention(qkv, H, hd, attn, ws=ws), "tensor", 4 * n * n * d),
-        "gemm_out_gate": (lambda i: h3b.gemm_bf16(attn, P[i % nb]["w_o"], h3b.EPI_GATE_RESID,
-                                                  P[i % nb]["b_o"], x, gate=mod[2], ws=ws),
-                          "tensor", 2 * n * d * d),
-        "gemm_fc1_gelu": (lambda i: h3b.gemm_bf16(h, P[i % nb]["w_fc1"], h3b.EPI_BIAS_GELU,
-                                                  P[i % nb]["b_fc1"], gbuf, ws=ws),
-                          "tensor", 2 * n * d * f),
-        "gemm_fc2_gate": (lambda i: h3b.gemm_bf16(gbuf, P[i % nb]["w_fc2"], h3b.EPI_GATE_RESID,
-                                                  P[i % nb]["b_fc2"], x, gate=mod[5], ws=ws),
-                          "tensor", 2 * n * f * d),
-        "ln_modulate": (lambda i: h3b.ln_modulate(x, cfg.ln_eps, mod[0], mod[1], h), "hbm",
-                        4 * n * d),
+        "gemm_out_gate": gemms["gemm_out_gate"],
+        "gemm_fc1_gelu": gemms["gemm_fc1_gelu"],
+        "gemm_fc2_gate": gemms["gemm_fc2_gate"],
         "final_euler": (lambda i: h3b.final_euler(x, cfg.n_video, cfg.ln_eps, model.final_mod,
                                                   1.0, 0.75, xs), "hbm", 10 * n * d),
     }
+    if not model.fold:
+        kinds["ln_modulate"] = (lambda i: h3b.ln_modulate(x, cfg.ln_eps, mod[0], mod[1], h),
+                                "hbm", 4 * n * d)
     blocks = counts_per_step["blocks"]
     launches = {"gemm_qkv_rope": blocks, "attention": blocks, "gemm_out_gate": blocks,
                 "gemm_fc1_gelu": blocks, "gemm_fc2_gate": blocks, "ln_modulate": 2 * blocks,

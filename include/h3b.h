@@ -305,6 +305,39 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                      int unpair_bypass, float sigma, float sigma_next, float* x_state,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- reuse policies */
+/* Whole-velocity reuse and core-residual reuse (dothoosh.com, "Aggressive optimisation
+ * levers"; aihot.vn section 4 "Speed/quality presets": --reuse and --core-reuse; the two
+ * are mutually exclusive).  The schedule: step i of `steps` runs the model when
+ * i % every == 0, and the last step always does (20 steps: every = 1, 2, 3 give 20, 11,
+ * 8 fresh evaluations, the counts the pages print).  fresh_out: host [steps], 1 = run
+ * the model.  Returns the number of fresh steps, or H3B_EINVAL. */
+int h3b_reuse_schedule(int steps, int every, unsigned char* fresh_out);
+
+/* h3b_denoise_step that also keeps what a skipped step needs: v_out [n_tokens, d] fp32,
+ * the velocity the step applied (whole-velocity reuse); core_res_out [n_tokens, d] fp32,
+ * the block stack's residual r = x_L - bf16(x_state) with x_state the step's input
+ * (core-residual reuse).  Either may be NULL; device. */
+int h3b_denoise_step_keep(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                          const h3b_block_weights* blocks, const unsigned char* active,
+                          const float* mods, const float* final_mod, int reduce_after,
+                          int unpair_bypass, float sigma, float sigma_next, float* x_state,
+                          float* v_out, float* core_res_out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* A skipped step of whole-velocity reuse: x_state += (sigma_next - sigma) v, with v the
+ * last fresh step's velocity.  v, x_state [n_tokens, d] fp32 device; d % 4 == 0. */
+int h3b_euler_velocity(const float* v, int n_tokens, int d, float sigma, float sigma_next,
+                       float* x_state, void* stream);
+
+/* A skipped step of core-residual reuse: the block stack is replaced by the residual of the
+ * last fresh step, x_L = bf16(bf16(x_state) + core_res); the final AdaLN and the Euler
+ * update run as in h3b_final_euler.  core_res, x_state [n_tokens, d] fp32; final_mod
+ * [2, 2, d] fp32; all device. */
+int h3b_euler_core_reuse(const float* core_res, int n_tokens, int n_video, int d, float eps,
+                         const float* final_mod, float sigma, float sigma_next, float* x_state,
+                         void* stream);
+
 /* Whole denoise from a HOST latent: copies x_host_in [n_tokens, d] fp32 to the device,
  * runs Euler steps first_step .. first_step + n_run - 1 of the linear grid with n_steps
  * intervals (sigma_i = 1 - i / n_steps), copies the state back into x_host_out and
@@ -388,6 +421,22 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
                   const h3b_bf16* bias, const float* gate, const float* rope_cs,
                   int rope_cols, int head_dim, h3b_bf16* out, void* ws, size_t ws_bytes,
                   void* stream);
+
+/* The projection GEMM in the forms of the folded block path (h3b_block_forward_folded):
+ *   H3B_EPI_LN_ROPE, H3B_EPI_LN_GELU: A [M, K] is the raw bf16 residual and B the folded
+ *     weights (h3b_fold_adaln); pre[r, j] = rstd_r (acc - mean_r fold_c[j]) + fold_dv[j],
+ *     with mean_r and rstd_r = 1 / sqrt(var_r + ln_eps) merged from stats_in
+ *     [M, K / 256] (h3b_row_stats form), then RoPE on columns < rope_cols (as
+ *     H3B_EPI_BIAS_ROPE) or GELU_tanh; K % 256 == 0.  bias and gate are unused.
+ *   H3B_EPI_GATE_RESID: as in h3b_gemm_bf16, and the output rows' group statistics go to
+ *     stats_out [M, N / 256] (h3b_row_stats form) when it is not NULL; N % 256 == 0.
+ * fold_c, fold_dv [N] fp32; other arguments as h3b_gemm_bf16.  All device. */
+enum { H3B_EPI_LN_ROPE = 4, H3B_EPI_LN_GELU = 5 };
+int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
+                     const h3b_bf16* bias, const float* gate, const float* fold_c,
+                     const float* fold_dv, const float* stats_in, float* stats_out,
+                     float ln_eps, const float* rope_cs, int rope_cols, int head_dim,
+                     h3b_bf16* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Joint self-attention over one packed QKV buffer: qkv [n_tokens, 3 n_heads head_dim]
  * bf16 (q, then k, then v; head j at column j*head_dim of each), out [n_tokens,

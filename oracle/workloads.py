@@ -49,3 +49,15 @@ def block(cfg, params, c, x, next_params=None, rows=None, dt=np.float64):
     pos = O.rope_positions(cfg.grid, cfg.n_audio, halved=cfg.rope_halved)
     return O.block_forward(x, params, mod, pos, cfg.n_heads, cfg.rope_split, cfg.rope_theta,
                            cfg.ln_eps, mod_next=mod_next, rows=rows, dt=dt)
+
+
+def denoise_reuse(cfg, blocks, final, c, x0, every: int, mode: str, dt=np.float64) -> np.ndarray:
+    """A whole denoise of cfg.steps Euler steps under whole-velocity ("velocity") or
+    core-residual ("core") reuse with the given period."""
+    mods = modulation_vectors(cfg, blocks, c)
+    fm = final_vectors(cfg, final, c)
+    fn = O.denoise_velocity_reuse if mode == "velocity" else O.denoise_core_reuse
+    return fn(x0, blocks, mods, fm, cfg.grid, cfg.n_audio, cfg.n_heads, cfg.rope_split,
+              cfg.rope_theta, cfg.ln_eps, cfg.steps, every, active=active_mask(cfg, mods),
+              reduce_after=cfg.reduce_after, halved=cfg.rope_halved,
+              unpair_bypass=cfg.unpair_bypass, dt=dt)

@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import oracle as O
 from oracle import workloads
 from tests.helpers import rel_l2
 
@@ -169,3 +170,56 @@ def test_cuda_graph_replay_matches_direct_run(name):
         torch.cuda.synchronize()
         assert torch.equal(xg, ref)
     del graph
+
+
+# ------------------------------------------------------------------------------ reuse policies
+@pytest.mark.parametrize("mode,every", [("velocity", 2), ("core", 2), ("core", 3),
+                                        ("velocity", 1)])
+def test_tiny_reuse_policies_vs_oracle(mode, every):
+    # a whole 4-step denoise of the tiny workload under a reuse policy
+    # (dothoosh.com "Aggressive optimisation levers"; aihot.vn section 4)
+    cfg = synth.CONFIGS["tiny"]
+    m = DiTDenoiser(cfg, keep_host_params=True)
+    x0 = synth.latent_noise(cfg)
+    x = x0.to(DEV)
+    fresh = m.run_reuse(x, every, mode)
+    h3b.sync_status()
+    assert fresh == int(O.reuse_schedule(cfg.steps, every).sum())
+    blocks = [{k: f64(v) for k, v in p.items()} for p in m.host_params]
+    final = {k: f64(v) for k, v in m.host_final.items()}
+    want = workloads.denoise_reuse(cfg, blocks, final, f64(synth.conditioning(cfg)), f64(x0),
+                                   every, mode)
+    got = x.cpu().numpy().astype(np.float64)
+    assert rel_l2(got, want) < TOL_STEPS
+    assert rel_l2(got - f64(x0), want - f64(x0)) < TOL_STEPS
+
+
+@pytest.mark.parametrize("name", ["dit512_reuse_velocity2", "dit512_reuse_core3"])
+def test_512_reuse_policies_vs_golden(name):
+    ref = np.load(os.path.join(GOLDEN, f"{name}_oracle.npz"))
+    mode = "velocity" if "velocity" in name else "core"
+    every = int(name[-1])
+    cfg = synth.CONFIGS["dit512"]
+    m = DiTDenoiser(cfg)
+    x0 = synth.latent_noise(cfg)
+    x = x0.to(DEV)
+    m.run_reuse(x, every, mode)
+    h3b.sync_status()
+    rows = ref["rows"]
+    got = x.cpu().numpy()[rows].astype(np.float64)
+    base = f64(x0)[rows]
+    want = ref["final"].astype(np.float64)
+    assert rel_l2(got, want) < TOL_STEPS
+    assert rel_l2(got - base, want - base) < TOL_STEPS
+
+
+def test_reuse_every_one_matches_the_plain_run_bit_for_bit():
+    cfg = synth.CONFIGS["dit512"]
+    m = DiTDenoiser(cfg)
+    x0 = synth.latent_noise(cfg).to(DEV)
+    a, b, c = x0.clone(), x0.clone(), x0.clone()
+    m.run(a)
+    m.run_reuse(b, 1, "velocity")
+    m.run_reuse(c, 1, "core")
+    h3b.sync_status()
+    assert torch.equal(a, b) and torch.equal(a, c)

@@ -156,3 +156,108 @@ def test_folded_block_zero_gates_bit_exact():
     x = synth.latent_noise(cfg).to(torch.bfloat16)
     xg, st, st_ref, _ = _folded_block(cfg, params, c, x)
     assert np.array_equal(bf16_bits(xg), bf16_bits(x))
+
+
+# (M, d, N): the QKV shape of the 512x512 workload, a ragged tiny one, and an FC1 shape
+LN_GEMM_SHAPES = [(1600, 3072, 9216), (40, 256, 768), (1000, 1024, 4096)]
+
+
+def _ln_gemm_inputs(M, d, N, seed, offset=0.0):
+    x = (rnd((M, d), 1.0, seed=seed).float() + offset).to(torch.bfloat16)
+    w = rnd((N, d), 0.02, seed=seed + 1)
+    b = rnd((N,), 0.02, seed=seed + 2)
+    shift = rnd((d,), 0.3, seed=seed + 3, dtype=torch.float32)
+    scale = rnd((d,), 0.3, seed=seed + 4, dtype=torch.float32)
+    return x, w, b, shift, scale
+
+
+def _fold_on_gpu(w, b, shift, scale):
+    N, d = w.shape
+    wo = torch.empty((N, d), dtype=torch.bfloat16, device=DEV)
+    c = torch.empty((N,), dtype=torch.float32, device=DEV)
+    dv = torch.empty((N,), dtype=torch.float32, device=DEV)
+    h3b.fold_adaln(w.to(DEV), b.to(DEV), shift.to(DEV), scale.to(DEV), wo, c, dv)
+    return wo, c, dv
+
+
+@pytest.mark.parametrize("M,d,N", LN_GEMM_SHAPES)
+@pytest.mark.parametrize("epi", [h3b.EPI_LN_GELU, h3b.EPI_LN_ROPE])
+def test_ln_folded_gemm_vs_oracle(M, d, N, epi):
+    x, w, b, shift, scale = _ln_gemm_inputs(M, d, N, seed=M + N)
+    wo, c, dv = _fold_on_gpu(w, b, shift, scale)
+    xd = x.to(DEV)
+    st = torch.empty((M, d // 256, 2), dtype=torch.float32, device=DEV)
+    h3b.row_stats(xd, st)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    h_o = O.modulate(O.layer_norm(np64(x), 1e-6), np64(shift), np64(scale))
+    pre = h_o @ np64(w).T + np64(b)
+    kw = {}
+    if epi == h3b.EPI_LN_GELU:
+        want = O.gelu_tanh(pre)
+    else:
+        hd = 128 if d % 128 == 0 and d >= 256 else 64
+        heads = d // hd
+        split = (32, 48, 48) if hd == 128 else (16, 24, 24)
+        # a token grid of M tokens (one row of video tokens, the rest audio)
+        grid, n_audio = (1, 1, min(M, 8)), M - min(M, 8)
+        dims = h3b.make_dims(d, heads, hd, 4 * d, 256, split)
+        cs = torch.empty((M, hd // 2, 2), dtype=torch.float32, device=DEV)
+        h3b.rope_table(dims, h3b.make_grid(*grid, n_audio), False, cs)
+        rope_cols = min(2 * d, N)
+        kw = dict(rope_cs=cs, rope_cols=rope_cols, head_dim=hd)
+        pos = O.rope_positions(grid, n_audio)
+        want = pre.copy()
+        for part in range(rope_cols // d):
+            blk = pre[:, part * d:(part + 1) * d].reshape(M, heads, hd)
+            want[:, part * d:(part + 1) * d] = O.rope_rotate(blk, pos, split, 1e4).reshape(M, d)
+    h3b.gemm_bf16_ln(xd, wo, epi, out, fold_c=c, fold_dv=dv, stats_in=st,
+                     ws=torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV),
+                     **kw)
+    h3b.sync_status()
+    got = np64(out)
+    from tests.helpers import max_block_rel_l2
+    assert rel_l2(got, want) < 6e-3
+    assert max_block_rel_l2(got, want) < 1.2e-2
+
+
+@pytest.mark.parametrize("M,N,K", [(1600, 3072, 3072), (40, 256, 1024), (1600, 3072, 12288)])
+def test_gate_resid_gemm_writes_row_statistics(M, N, K):
+    A = rnd((M, K), 1.0, seed=91)
+    B = rnd((N, K), K ** -0.5, seed=92)
+    bias = rnd((N,), 0.1, seed=93)
+    resid = rnd((M, N), 1.0, seed=94)
+    g = rnd((N,), 0.5, seed=95, dtype=torch.float32)
+    out = resid.to(DEV)
+    st = torch.empty((M, N // 256, 2), dtype=torch.float32, device=DEV)
+    plain = resid.to(DEV)
+    ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV)
+    h3b.gemm_bf16_ln(A.to(DEV), B.to(DEV), h3b.EPI_GATE_RESID, out, bias=bias.to(DEV),
+                     gate=g.to(DEV), stats_out=st, ws=ws)
+    h3b.gemm_bf16(A.to(DEV), B.to(DEV), h3b.EPI_GATE_RESID, bias.to(DEV), plain, gate=g.to(DEV),
+                  ws=ws)
+    ref = torch.empty_like(st)
+    h3b.row_stats(out, ref)
+    h3b.sync_status()
+    # the output is that of the plain gated-residual epilogue, bit for bit
+    assert torch.equal(out, plain)
+    s, r = st.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(s[..., 0] - r[..., 0])) < 1e-5 * (1 + np.max(np.abs(r[..., 0])))
+    assert rel_l2(s[..., 1], r[..., 1]) < 1e-5
+
+
+def test_ln_folded_gemm_large_row_offset():
+    # rows far from zero mean: the statistics are taken about each group's first value
+    M, d, N = 300, 1024, 1024
+    x, w, b, shift, scale = _ln_gemm_inputs(M, d, N, seed=7, offset=50.0)
+    wo, c, dv = _fold_on_gpu(w, b, shift, scale)
+    xd = x.to(DEV)
+    st = torch.empty((M, d // 256, 2), dtype=torch.float32, device=DEV)
+    h3b.row_stats(xd, st)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    h3b.gemm_bf16_ln(xd, wo, h3b.EPI_LN_GELU, out, fold_c=c, fold_dv=dv, stats_in=st)
+    h3b.sync_status()
+    want = O.gelu_tanh(O.modulate(O.layer_norm(np64(x), 1e-6), np64(shift), np64(scale))
+                       @ np64(w).T + np64(b))
+    # the bf16 residual itself carries 50 * 2^-9 of rounding per element at this offset,
+    # which LN amplifies by 1 / std: the bound scales with it
+    assert rel_l2(np64(out), want) < 2e-2

@@ -347,7 +347,8 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
                       const h3b_block_weights* blocks, const unsigned char* active,
                       const float* mods, const float* final_mod, int reduce_after,
                       int unpair_bypass, float sigma, float sigma_next, float* x_state,
-                      const StepBufs& b, cudaStream_t s) {
+                      const StepBufs& b, cudaStream_t s, float* v_out = nullptr,
+                      float* r_out = nullptr) {
   const int D = d->d;
   const int nv = g->t * g->h * g->w;
   const int n = nv + g->n_audio;
@@ -395,6 +396,9 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
         (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
                                   g->w, g->n_audio, D, s)))
       return rc;
+    if (v_out || r_out)
+      return launch_final_euler_keep(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
+                                     x_state, v_out, r_out, s);
     return launch_final_euler(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
                               x_state, s);
   }
@@ -429,6 +433,9 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
       (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
                                 g->w, g->n_audio, D, s)))
     return rc;
+  if (v_out || r_out)
+    return launch_final_euler_keep(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
+                                   x_state, v_out, r_out, s);
   return launch_final_euler(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma, x_state, s);
 }
 
@@ -690,6 +697,63 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
   return denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
                            reduce_after, unpair_bypass, sigma, sigma_next, x_state, b,
                            static_cast<cudaStream_t>(stream));
+}
+
+int h3b_denoise_step_keep(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                          const h3b_block_weights* blocks, const unsigned char* active,
+                          const float* mods, const float* final_mod, int reduce_after,
+                          int unpair_bypass, float sigma, float sigma_next, float* x_state,
+                          float* v_out, float* core_res_out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  StepBufs b;
+  int rc = check_step_args(dims, grid, n_blocks, blocks, active, mods, final_mod, reduce_after,
+                           x_state, ws, ws_bytes, &b);
+  if (rc) return rc;
+  if ((v_out && !al16(v_out)) || (core_res_out && !al16(core_res_out)))
+    return set_error(H3B_EINVAL, "denoise_step_keep: misaligned v_out / core_res_out");
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
+                           reduce_after, unpair_bypass, sigma, sigma_next, x_state, b,
+                           static_cast<cudaStream_t>(stream), v_out, core_res_out);
+}
+
+int h3b_euler_velocity(const float* v, int n_tokens, int d, float sigma, float sigma_next,
+                       float* x_state, void* stream) {
+  if (n_tokens < 0 || d <= 0 || d % 4)
+    return set_error(H3B_EINVAL, "euler_velocity: bad sizes (n=%d d=%d)", n_tokens, d);
+  if (!v || !x_state || !al16(v) || !al16(x_state))
+    return set_error(H3B_EINVAL, "euler_velocity: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_euler_axpy(v, static_cast<long long>(n_tokens) * d, sigma_next - sigma, x_state,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int h3b_euler_core_reuse(const float* core_res, int n_tokens, int n_video, int d, float eps,
+                         const float* final_mod, float sigma, float sigma_next, float* x_state,
+                         void* stream) {
+  if (n_tokens < 0 || n_video < 0 || n_video > n_tokens || d <= 0 || d % 256 || d > 4096)
+    return set_error(H3B_EINVAL, "euler_core_reuse: bad sizes (n=%d n_video=%d d=%d)", n_tokens,
+                     n_video, d);
+  if (!core_res || !final_mod || !x_state || !al16(core_res) || !al16(final_mod) ||
+      !al16(x_state))
+    return set_error(H3B_EINVAL, "euler_core_reuse: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_core_reuse_final(core_res, n_tokens, n_video, d, eps, final_mod,
+                                 sigma_next - sigma, x_state, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_reuse_schedule(int steps, int every, unsigned char* fresh_out) {
+  if (steps <= 0 || every <= 0 || !fresh_out)
+    return set_error(H3B_EINVAL, "reuse_schedule: steps=%d every=%d", steps, every);
+  int n = 0;
+  for (int i = 0; i < steps; ++i) {
+    fresh_out[i] = (i % every == 0 || i == steps - 1) ? 1 : 0;
+    n += fresh_out[i];
+  }
+  return n;
 }
 
 namespace {
@@ -1016,6 +1080,51 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
   e.out = reinterpret_cast<bf16*>(out);
   e.ld_out = N;
   if (ws && !al16(ws)) return set_error(H3B_EINVAL, "gemm_bf16: misaligned workspace");
+  return launch_gemm_bf16(ctx, reinterpret_cast<const bf16*>(A), reinterpret_cast<const bf16*>(B),
+                          M, N, K, e, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
+                     const h3b_bf16* bias, const float* gate, const float* fold_c,
+                     const float* fold_dv, const float* stats_in, float* stats_out,
+                     float ln_eps, const float* rope_cs, int rope_cols, int head_dim,
+                     h3b_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+  if (M < 0 || K <= 0 || K % 64 || N <= 0 || N % 128)
+    return set_error(H3B_EINVAL, "gemm_bf16_ln: K=%d must be a multiple of 64, N=%d of 128", K, N);
+  if (!A || !B || !out || !al16(A) || !al16(B) || !al16(out) || (ws && !al16(ws)))
+    return set_error(H3B_EINVAL, "gemm_bf16_ln: NULL or misaligned pointer");
+  GemmEpilogue e;
+  e.out = reinterpret_cast<bf16*>(out);
+  e.ld_out = N;
+  if (epilogue == H3B_EPI_LN_ROPE || epilogue == H3B_EPI_LN_GELU) {
+    if (K % 256 || K > 4096 || !fold_c || !fold_dv || !stats_in || !al16(fold_c) ||
+        !al16(fold_dv) || !al16(stats_in) || !(ln_eps > 0.f))
+      return set_error(H3B_EINVAL, "gemm_bf16_ln: LN-folded form needs K %% 256 == 0, c, dv, stats_in, eps > 0");
+    if (epilogue == H3B_EPI_LN_ROPE &&
+        (!rope_cs || !al16(rope_cs) || (head_dim != 64 && head_dim != 128) || rope_cols < 0 ||
+         rope_cols % head_dim || rope_cols > N))
+      return set_error(H3B_EINVAL, "gemm_bf16_ln: bad RoPE arguments");
+    e.kind = epilogue == H3B_EPI_LN_ROPE ? kEpiRopeLN : kEpiGeluLN;
+    e.fold_c = fold_c;
+    e.bias_f32 = fold_dv;
+    e.stats_in = reinterpret_cast<const float2*>(stats_in);
+    e.stats_parts = K / 256;
+    e.ln_eps = ln_eps;
+    e.rope_cs = rope_cs;
+    e.rope_cols = rope_cols;
+    e.head_dim = head_dim;
+  } else if (epilogue == H3B_EPI_GATE_RESID) {
+    if (!bias || !gate || !al16(bias) || !al16(gate) || (stats_out && (N % 256 || !al16(stats_out))))
+      return set_error(H3B_EINVAL, "gemm_bf16_ln: gated residual needs bias, gate (and N %% 256 == 0 for stats)");
+    e.kind = kEpiGateResid;
+    e.bias = reinterpret_cast<const bf16*>(bias);
+    e.gate = gate;
+    e.stats_out = reinterpret_cast<float2*>(stats_out);
+  } else {
+    return set_error(H3B_EINVAL, "gemm_bf16_ln: epilogue %d", epilogue);
+  }
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
   return launch_gemm_bf16(ctx, reinterpret_cast<const bf16*>(A), reinterpret_cast<const bf16*>(B),
                           M, N, K, e, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }

@@ -130,6 +130,18 @@ int launch_fold_adaln(const bf16* w, const bf16* b, const float* shift, const fl
 int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,
                        const float* final_mod, float dt_sigma, float* x_state,
                        cudaStream_t stream);
+// final_euler that also stores the velocity and / or the core residual
+// r = x_l - bf16(x_state) (either may be null)
+int launch_final_euler_keep(const bf16* x_l, int n, int n_video, int d, float eps,
+                            const float* final_mod, float dt_sigma, float* x_state, float* v_out,
+                            float* r_out, cudaStream_t stream);
+// skipped core: x_l = bf16(bf16(x_state) + r_in), then final AdaLN + Euler
+int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float eps,
+                            const float* final_mod, float dt_sigma, float* x_state,
+                            cudaStream_t stream);
+// x_state += dt * v (n elements, n % 4 == 0)
+int launch_euler_axpy(const float* v, long long n, float dt_sigma, float* x_state,
+                      cudaStream_t stream);
 int launch_token_pair(const bf16* src, bf16* dst, int t, int h, int w, int n_audio, int d,
                       cudaStream_t stream);
 int launch_token_unpair(const bf16* src, bf16* dst, const bf16* saved, int t, int h, int w,

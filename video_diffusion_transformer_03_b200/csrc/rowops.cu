@@ -6,6 +6,7 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
+#include <algorithm>
 #include <cmath>
 
 namespace h3b {
@@ -146,6 +147,88 @@ __global__ void __launch_bounds__(128) k_final_euler(const bf16* __restrict__ xl
     }
     st[0] = make_float4(x8[0], x8[1], x8[2], x8[3]);
     st[1] = make_float4(x8[4], x8[5], x8[6], x8[7]);
+  }
+}
+
+// The final AdaLN + Euler step of the reuse policies.  !CORE_IN: as k_final_euler on
+// x_l, also storing the velocity (v_out) and the core residual r = x_l - bf16(x_state)
+// (r_out) when those are not null.  CORE_IN: a skipped core, x_l = bf16(bf16(x_state) +
+// r_in) built in registers.
+template <int NV, bool CORE_IN>
+__global__ void __launch_bounds__(128) k_final_euler_ex(const bf16* __restrict__ xl,
+                                                        const float* __restrict__ r_in, int n,
+                                                        int n_video, float eps,
+                                                        const float* __restrict__ fmod,
+                                                        float dt, float* __restrict__ xs,
+                                                        float* __restrict__ v_out,
+                                                        float* __restrict__ r_out) {
+  constexpr int D = NV * 256;
+  const int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const int lane = threadIdx.x & 31;
+  float v[NV][8];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const size_t off = size_t(row) * D + (i * 32 + lane) * 8;
+    if constexpr (CORE_IN) {
+      float f[8], x_in[8], r[8];
+      load8f(xs + off, f);
+      unpack8(pack8(f), x_in);
+      load8f(r_in + off, r);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = x_in[k] + r[k];
+      unpack8(pack8(f), v[i]);
+    } else {
+      unpack8(__ldg(reinterpret_cast<const uint4*>(xl + off)), v[i]);
+      if (r_out) {
+        float f[8], x_in[8];
+        load8f(xs + off, f);
+        unpack8(pack8(f), x_in);
+        float4* ro = reinterpret_cast<float4*>(r_out + off);
+        ro[0] = make_float4(v[i][0] - x_in[0], v[i][1] - x_in[1], v[i][2] - x_in[2], v[i][3] - x_in[3]);
+        ro[1] = make_float4(v[i][4] - x_in[4], v[i][5] - x_in[5], v[i][6] - x_in[6], v[i][7] - x_in[7]);
+      }
+    }
+  }
+  float mean, rstd;
+  row_stats<NV>(v, D, eps, mean, rstd);
+  const float* shift = fmod + (row < n_video ? 0 : 2 * D);
+  const float* scale = shift + D;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int col = (i * 32 + lane) * 8;
+    const size_t off = size_t(row) * D + col;
+    float sh[8], sc[8], vel[8];
+    load8f(shift + col, sh);
+    load8f(scale + col, sc);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) vel[k] = fmaf((v[i][k] - mean) * rstd, 1.0f + sc[k], sh[k]);
+    if (!CORE_IN && v_out) {
+      float4* vo = reinterpret_cast<float4*>(v_out + off);
+      vo[0] = make_float4(vel[0], vel[1], vel[2], vel[3]);
+      vo[1] = make_float4(vel[4], vel[5], vel[6], vel[7]);
+    }
+    float4* st = reinterpret_cast<float4*>(xs + off);
+    float4 a = st[0], b = st[1];
+    st[0] = make_float4(fmaf(dt, vel[0], a.x), fmaf(dt, vel[1], a.y), fmaf(dt, vel[2], a.z),
+                        fmaf(dt, vel[3], a.w));
+    st[1] = make_float4(fmaf(dt, vel[4], b.x), fmaf(dt, vel[5], b.y), fmaf(dt, vel[6], b.z),
+                        fmaf(dt, vel[7], b.w));
+  }
+}
+
+// x_state += dt * v over n4 float4 elements (a skipped step of whole-velocity reuse).
+__global__ void __launch_bounds__(256) k_euler_axpy(const float4* __restrict__ v, long long n4,
+                                                    float dt, float4* __restrict__ xs) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldg(v + i);
+    float4 x = xs[i];
+    x.x = fmaf(dt, a.x, x.x);
+    x.y = fmaf(dt, a.y, x.y);
+    x.z = fmaf(dt, a.z, x.z);
+    x.w = fmaf(dt, a.w, x.w);
+    xs[i] = x;
   }
 }
 
@@ -499,6 +582,38 @@ int launch_final_euler(const bf16* x_l, int n, int n_video, int d, float eps,
   H3B_NV_SWITCH(d / 256, (k_final_euler<NV><<<grid, 32 * kRowWarps, 0, stream>>>(
                              x_l, n, n_video, eps, final_mod, dt_sigma, x_state)));
   return check_launch("final_euler");
+}
+
+int launch_final_euler_keep(const bf16* x_l, int n, int n_video, int d, float eps,
+                            const float* final_mod, float dt_sigma, float* x_state, float* v_out,
+                            float* r_out, cudaStream_t stream) {
+  if (n <= 0) return 0;
+  const int grid = (n + kRowWarps - 1) / kRowWarps;
+  H3B_NV_SWITCH(d / 256, (k_final_euler_ex<NV, false><<<grid, 32 * kRowWarps, 0, stream>>>(
+                             x_l, nullptr, n, n_video, eps, final_mod, dt_sigma, x_state, v_out,
+                             r_out)));
+  return check_launch("final_euler_keep");
+}
+
+int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float eps,
+                            const float* final_mod, float dt_sigma, float* x_state,
+                            cudaStream_t stream) {
+  if (n <= 0) return 0;
+  const int grid = (n + kRowWarps - 1) / kRowWarps;
+  H3B_NV_SWITCH(d / 256, (k_final_euler_ex<NV, true><<<grid, 32 * kRowWarps, 0, stream>>>(
+                             nullptr, r_in, n, n_video, eps, final_mod, dt_sigma, x_state,
+                             nullptr, nullptr)));
+  return check_launch("core_reuse_final");
+}
+
+int launch_euler_axpy(const float* v, long long n, float dt_sigma, float* x_state,
+                      cudaStream_t stream) {
+  const long long n4 = n / 4;
+  if (n4 <= 0) return 0;
+  const int grid = static_cast<int>(std::min<long long>((n4 + 255) / 256, 148 * 8));
+  k_euler_axpy<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(v), n4, dt_sigma,
+                                         reinterpret_cast<float4*>(x_state));
+  return check_launch("euler_axpy");
 }
 
 int launch_token_pair(const bf16* src, bf16* dst, int t, int h, int w, int n_audio, int d,

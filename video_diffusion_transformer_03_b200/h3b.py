@@ -19,6 +19,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libh3b.so"
 H3B_OK, H3B_EINVAL, H3B_EWORKSPACE, H3B_ECUDA, H3B_ETIMEOUT, H3B_EUNSUPPORTED = 0, -1, -2, -3, -4, -5
 PAIR, UNPAIR = 0, 1
 EPI_BIAS, EPI_BIAS_GELU, EPI_BIAS_ROPE, EPI_GATE_RESID = 0, 1, 2, 3
+EPI_LN_ROPE, EPI_LN_GELU = 4, 5
 
 
 class H3BError(RuntimeError):
@@ -82,10 +83,18 @@ _SIGS = {
     "h3b_denoise_host_pipelined": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                                         ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _I,
                                         _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "h3b_reuse_schedule": (_I, [_I, _I, _P]),
+    "h3b_denoise_step_keep": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                                   ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P,
+                                   _P, _P, _P, _SZ, _P]),
+    "h3b_euler_velocity": (_I, [_P, _I, _I, _F, _F, _P, _P]),
+    "h3b_euler_core_reuse": (_I, [_P, _I, _I, _I, _F, _P, _F, _F, _P, _P]),
     "h3b_token_reduce": (_I, [_I, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "h3b_quantize_rows": (_I, [_P, _I, _I, _P, _P, _P]),
     "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P]),
+    "h3b_gemm_bf16_ln": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _P, _I, _I,
+                              _P, _P, _SZ, _P]),
     "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P, _SZ, _P]),
     "h3b_layer_mask": (_I, [_P, _I, _I, _I, _P]),
 }
@@ -348,6 +357,43 @@ def denoise_step(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active,
     del keep
 
 
+def reuse_schedule(steps: int, every: int) -> np.ndarray:
+    """Host policy: which of `steps` Euler steps run the model (h3b_reuse_schedule)."""
+    out = (ctypes.c_ubyte * max(steps, 1))()
+    n = int(lib.h3b_reuse_schedule(steps, every, ctypes.cast(out, ctypes.c_void_p)))
+    if n < 0:
+        _check(n)
+    return np.array(list(out)[:steps], dtype=bool)
+
+
+def denoise_step_keep(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods,
+                      final_mod, reduce_after: int, unpair_bypass: bool, sigma: float,
+                      sigma_next: float, x_state, v_out, core_res_out, ws, stream=None) -> None:
+    _dev(x_state, torch.float32, "x_state")
+    arr = _blocks_array(blocks)
+    keep, mask = _mask_array(active, len(blocks))
+    _check(lib.h3b_denoise_step_keep(ctypes.byref(dims), ctypes.byref(grid), len(blocks), arr,
+                                     mask, _ptr(mods), _ptr(final_mod), reduce_after,
+                                     int(bool(unpair_bypass)), sigma, sigma_next, _ptr(x_state),
+                                     _ptr(v_out), _ptr(core_res_out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
+def euler_velocity(v, sigma, sigma_next, x_state, stream=None) -> None:
+    _dev(v, torch.float32, "v"); _dev(x_state, torch.float32, "x_state")
+    _check(lib.h3b_euler_velocity(_ptr(v), x_state.shape[0], x_state.shape[1], sigma, sigma_next,
+                                  _ptr(x_state), _stream(stream)))
+
+
+def euler_core_reuse(core_res, n_video, eps, final_mod, sigma, sigma_next, x_state,
+                     stream=None) -> None:
+    _dev(core_res, torch.float32, "core_res"); _dev(x_state, torch.float32, "x_state")
+    _check(lib.h3b_euler_core_reuse(_ptr(core_res), x_state.shape[0], n_video, x_state.shape[1],
+                                    eps, _ptr(final_mod), sigma, sigma_next, _ptr(x_state),
+                                    _stream(stream)))
+
+
 def denoise_host(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods, final_mod,
                  reduce_after: int, unpair_bypass: bool, n_steps: int, first_step: int, n_run: int,
                  x_host_in, x_host_out, x_state_dev, ws, stream=None) -> None:
@@ -415,6 +461,21 @@ def gemm_bf16(A, B, epilogue, bias, out, gate=None, rope_cs=None, rope_cols=0, h
     _check(lib.h3b_gemm_bf16(_ptr(A), _ptr(B), M, N, K, epilogue, _ptr(bias), _ptr(gate),
                              _ptr(rope_cs), rope_cols, head_dim, _ptr(out), wp, wb,
                              _stream(stream)))
+
+
+def gemm_bf16_ln(A, B, epilogue, out, bias=None, gate=None, fold_c=None, fold_dv=None,
+                 stats_in=None, stats_out=None, ln_eps=1e-6, rope_cs=None, rope_cols=0,
+                 head_dim=128, ws=None, stream=None) -> None:
+    """The folded block's GEMM forms (h3b_gemm_bf16_ln): EPI_LN_ROPE / EPI_LN_GELU read the
+    raw residual A with its row statistics stats_in; EPI_GATE_RESID may write stats_out."""
+    _dev(A, torch.bfloat16, "A"); _dev(B, torch.bfloat16, "B"); _dev(out, torch.bfloat16, "out")
+    M, K = A.shape
+    N = B.shape[0]
+    wp, wb = _wsargs(ws)
+    _check(lib.h3b_gemm_bf16_ln(_ptr(A), _ptr(B), M, N, K, epilogue, _ptr(bias), _ptr(gate),
+                                _ptr(fold_c), _ptr(fold_dv), _ptr(stats_in), _ptr(stats_out),
+                                ln_eps, _ptr(rope_cs), rope_cols, head_dim, _ptr(out), wp, wb,
+                                _stream(stream)))
 
 
 def attention(qkv, n_heads, head_dim, out, ws=None, stream=None) -> None:

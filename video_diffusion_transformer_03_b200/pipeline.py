@@ -85,6 +85,33 @@ class DiTDenoiser:
         for i in range(self.cfg.run_steps if n_run is None else n_run):
             self.step(x_state, i, stream)
 
+    def run_reuse(self, x_state: torch.Tensor, every: int, mode: str = "velocity",
+                  stream=None) -> int:
+        """A whole denoise under a reuse policy (host policy over the C ABI): the steps
+        h3b_reuse_schedule marks fresh run the model and keep its velocity ("velocity") or
+        its core residual ("core"); the others reuse it.  Returns the fresh step count."""
+        if mode not in ("velocity", "core"):
+            raise ValueError(mode)
+        steps = self.cfg.steps
+        fresh = h3b.reuse_schedule(steps, every)
+        held = getattr(self, "_reuse_buf", None)
+        if held is None or held.shape != x_state.shape:
+            held = self._reuse_buf = torch.empty_like(x_state)
+        for i in range(steps):
+            sg, sn = self.sigmas(i)
+            if fresh[i]:
+                h3b.denoise_step_keep(self.dims, self.grid, self.weights, self.active, self.mods,
+                                      self.final_mod, self.cfg.reduce_after,
+                                      self.cfg.unpair_bypass, sg, sn, x_state,
+                                      held if mode == "velocity" else None,
+                                      held if mode == "core" else None, self.ws, stream)
+            elif mode == "velocity":
+                h3b.euler_velocity(held, sg, sn, x_state, stream)
+            else:
+                h3b.euler_core_reuse(held, self.cfg.n_video, self.cfg.ln_eps, self.final_mod,
+                                     sg, sn, x_state, stream)
+        return int(fresh.sum())
+
     def capture(self, x_state: torch.Tensor, n_run: Optional[int] = None) -> torch.cuda.CUDAGraph:
         """Record a whole denoise of x_state (in place) as one CUDA graph; replaying it
         relaunches every kernel of every Euler step without host work.  Call run() once
