@@ -523,3 +523,56 @@ def _core(x_state, blocks, mods, grid, n_audio, n_heads, split, theta, eps, acti
     if saved is not None:
         x = token_unpair(x, grid, n_audio, saved if unpair_bypass else None, dt)
     return x
+
+
+# --------------------------------------------------------------------------------------
+# f1: patch embedding and final heads (the steps on either side of the block stack)
+# --------------------------------------------------------------------------------------
+def patch_embed(latent, n_video: int, w_patch, b_patch, dt=F64) -> np.ndarray:
+    """Model-space input of the block stack from the per-token latent [N, C]: one linear
+    projection per stream (video rows [0, n_video), audio rows after), x = latent W^T + b.
+    w_patch [2 streams, d, C], b_patch [2, d].  The latent enters as bf16 (the GPU's
+    operand precision; the state itself stays fp32).  Reading: the pages name patch and
+    head work around the core ([aihot] section 4: core-residual reuse refreshes patch/head
+    every step) but give no dimensions; C is a parameter of the workload."""
+    lat = round_to_bf16(latent).astype(dt)
+    w = np.asarray(w_patch, dt)
+    b = np.asarray(b_patch, dt)
+    out = np.empty((lat.shape[0], w.shape[1]), dt)
+    out[:n_video] = lat[:n_video] @ w[0].T + b[0]
+    out[n_video:] = lat[n_video:] @ w[1].T + b[1]
+    return out
+
+
+def final_head(x_l, final_mod, n_video: int, eps: float, w_head, b_head, dt=F64) -> np.ndarray:
+    """Latent velocity: the per-stream final AdaLN of x_L followed by that stream's linear
+    head, v = (LN(x_L)(1 + scale_s) + shift_s) W_s^T + b_s ([dothoosh] "DiT fusions and
+    memory management": the final BF16 heads apply the AdaLN as they load their tiles).
+    w_head [2, C, d], b_head [2, C]."""
+    h = final_adaln(x_l, final_mod, n_video, eps, dt)
+    w = np.asarray(w_head, dt)
+    b = np.asarray(b_head, dt)
+    v = np.empty((h.shape[0], w.shape[1]), dt)
+    v[:n_video] = h[:n_video] @ w[0].T + b[0]
+    v[n_video:] = h[n_video:] @ w[1].T + b[1]
+    return v
+
+
+def denoise_latent(lat0, blocks, mods, final_mod, heads, grid, n_audio: int, n_heads: int,
+                   split, theta: float, eps: float, steps: int, run_steps: int, active=None,
+                   reduce_after: int = -1, halved: bool = False, unpair_bypass: bool = True,
+                   dt=F64) -> np.ndarray:
+    """The Euler loop on the latent: each step x = bf16(patch_embed(latent)) (the residual
+    stream is stored in bf16), the block stack as in denoise(), then
+    latent += (s' - s) final_head(x_L).  heads: dict with w_patch, b_patch, w_head,
+    b_head."""
+    sig = sigma_grid(steps, dt)
+    lat = np.asarray(lat0, dt)
+    nv = grid[0] * grid[1] * grid[2]
+    for i in range(run_steps):
+        x = patch_embed(lat, nv, heads["w_patch"], heads["b_patch"], dt)
+        x_l = _core(x, blocks, mods, grid, n_audio, n_heads, split, theta, eps, active,
+                    reduce_after, halved, unpair_bypass, dt)
+        v = final_head(x_l, final_mod, nv, eps, heads["w_head"], heads["b_head"], dt)
+        lat = euler_update(lat, v, sig[i], sig[i + 1], dt)
+    return lat

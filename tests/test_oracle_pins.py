@@ -742,3 +742,62 @@ def test_block_with_qk_norm_vs_torch_composition():
     w0 = {k: v for k, v in w.items() if k not in ("q_norm", "k_norm")}
     plain, _ = O.block_forward(x, w0, mod, pos, 2, (8, 12, 12), 1e4, 1e-6)
     assert np.max(np.abs(plain - out)) > 1e-3
+
+
+# ----------------------------------------------------------------------------- patch / heads
+def test_patch_embed_and_head_per_stream_vs_torch():
+    r = np.random.default_rng(41)
+    n, nv, C, d = 11, 7, 16, 24
+    lat = O.round_to_bf16(r.standard_normal((n, C))).astype(np.float64)
+    wp, bp = r.standard_normal((2, d, C)), r.standard_normal((2, d))
+    x = O.patch_embed(lat, nv, wp, bp)
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    want = torch.cat([F.linear(t(lat[:nv]), t(wp[0]), t(bp[0])),
+                      F.linear(t(lat[nv:]), t(wp[1]), t(bp[1]))]).numpy()
+    assert np.max(np.abs(x - want)) < 1e-12
+    fm = r.standard_normal((2, 2, d)) * 0.3
+    wh, bh = r.standard_normal((2, C, d)), r.standard_normal((2, C))
+    v = O.final_head(x, fm, nv, 1e-6, wh, bh)
+    xn = F.layer_norm(t(x), (d,), eps=1e-6)
+    hv = xn[:nv] * (1 + t(fm[0, 1])) + t(fm[0, 0])
+    ha = xn[nv:] * (1 + t(fm[1, 1])) + t(fm[1, 0])
+    want = torch.cat([F.linear(hv, t(wh[0]), t(bh[0])), F.linear(ha, t(wh[1]), t(bh[1]))])
+    assert np.max(np.abs(v - want.numpy())) < 1e-12
+
+
+def test_latent_loop_with_identity_patch_and_head_is_the_model_space_loop():
+    blocks, mods, fm, grid, na, x0 = _denoise_case(n_blocks=3)
+    a = _DENOISE_ARGS
+    d = x0.shape[1]
+    eye = np.stack([np.eye(d)] * 2)
+    heads = {"w_patch": eye, "b_patch": np.zeros((2, d)), "w_head": eye,
+             "b_head": np.zeros((2, d))}
+    kw = dict(active=[1, 0, 1], reduce_after=1)
+    got = O.denoise_latent(x0, blocks, mods, fm, heads, grid, na, a["heads"], a["split"],
+                           a["theta"], a["eps"], 4, 4, **kw)
+    want = O.denoise(x0, blocks, mods, fm, grid, na, a["heads"], a["split"], a["theta"],
+                     a["eps"], steps=4, run_steps=4, **kw)
+    assert np.array_equal(got, want)
+
+
+def test_latent_loop_constant_head_closed_form():
+    # final scale -1: the head sees shift_s on every row, so each step adds
+    # (s' - s)(W_s shift_s + b_s) to the latent whatever the blocks do
+    blocks, mods, fm, grid, na, x0 = _denoise_case(n_blocks=2)
+    a = _DENOISE_ARGS
+    r = np.random.default_rng(43)
+    d, C, n, nv = 64, 8, x0.shape[0], 16
+    fc = np.zeros((2, 2, d))
+    fc[:, 1] = -1
+    fc[:, 0] = r.standard_normal((2, d))
+    heads = {"w_patch": r.standard_normal((2, d, C)) * 0.1, "b_patch": r.standard_normal((2, d)),
+             "w_head": r.standard_normal((2, C, d)) * 0.1, "b_head": r.standard_normal((2, C))}
+    lat0 = r.standard_normal((n, C))
+    got = O.denoise_latent(lat0, blocks, mods, fc, heads, grid, na, a["heads"], a["split"],
+                           a["theta"], a["eps"], 4, 3)
+    vv = heads["w_head"][0] @ fc[0, 0] + heads["b_head"][0]
+    va = heads["w_head"][1] @ fc[1, 0] + heads["b_head"][1]
+    want = lat0.copy()
+    want[:nv] += -0.75 * vv
+    want[nv:] += -0.75 * va
+    assert np.allclose(got, want, atol=1e-12)
