@@ -99,7 +99,13 @@ typedef struct h3b_grid {
  * scale_msa); w_fc1_fold [d_ff, d] bf16 with c_fc1, d_fc1 [d_ff] fp32 from (shift_mlp,
  * scale_mlp).  With them the block reads the raw residual and no LayerNorm pass runs
  * (h3b_block_forward_folded; h3b_denoise_step uses them when every active block has
- * them).  h3b_block_forward ignores them. */
+ * them).  h3b_block_forward ignores them.
+ *
+ * q_norm, k_norm (optional, both or neither): per-head RMSNorm gains [head_dim] fp32 for
+ * q and k.  When present, every head of q and k is normalised inside the QKV
+ * projection's epilogue, before the rotation: q_h <- q_h / sqrt(mean(q_h^2) + ln_eps) *
+ * q_norm (dothoosh.com, "The powerful int8 path": RMS normalisation and RoPE for Q/K in
+ * the QKV tile). */
 typedef struct h3b_block_weights {
   const h3b_bf16* w_qkv;
   const h3b_bf16* b_qkv;
@@ -115,6 +121,8 @@ typedef struct h3b_block_weights {
   const h3b_bf16* w_fc1_fold;
   const float* c_fc1;
   const float* d_fc1;
+  const float* q_norm;
+  const float* k_norm;
 } h3b_block_weights;
 
 /* ---------------------------------------------------------------- library information */
@@ -305,6 +313,42 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
                      int unpair_bypass, float sigma, float sigma_next, float* x_state,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- latent steps */
+/* The steps on either side of the block stack (dothoosh.com, "DiT fusions and memory
+ * management": the final BF16 heads apply the AdaLN as they load their tiles; aihot.vn
+ * section 4: the patch and head work around the core).  The state is a per-token latent
+ * [n_tokens, c_lat] fp32; each stream (video rows, then audio rows) has its own patch
+ * embedding and head.  w_head_fold[s], c_head[s], dv_head[s] are the stream's head with
+ * its final AdaLN folded in (h3b_fold_adaln with the stream's final (shift, scale)). */
+typedef struct h3b_latent_heads {
+  int c_lat;                          /* latent channels per token, multiple of 128 */
+  const h3b_bf16* w_patch[2];         /* [d, c_lat] bf16, per stream (video, audio) */
+  const h3b_bf16* b_patch[2];         /* [d] bf16 */
+  const h3b_bf16* w_head_fold[2];     /* [c_lat, d] bf16 */
+  const float* c_head[2];             /* [c_lat] fp32 */
+  const float* dv_head[2];            /* [c_lat] fp32 */
+} h3b_latent_heads;
+
+/* Bytes of workspace h3b_denoise_step_latent needs (0 on bad arguments). */
+size_t h3b_denoise_latent_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce,
+                                         int c_lat);
+
+/* One Euler step on the latent:
+ *   x = bf16(bf16(latent) W_patch,s^T + b_patch,s)   (GEMM per stream; its epilogue also
+ *       writes x's row statistics)
+ *   every active block in its folded form (each must carry its folded weights), with the
+ *   token pairing / restore of h3b_denoise_step
+ *   latent += (sigma_next - sigma) ((LN(x_L)(1 + scale_s) + shift_s) W_head,s^T + b_head,s)
+ *       (the head GEMM per stream applies the folded final AdaLN and the Euler update in
+ *       its epilogue; no normalised activation is stored).
+ * latent: device [n_tokens, c_lat] fp32 in/out; mods: device [n_blocks, 6, d];
+ * ws: h3b_denoise_latent_workspace_size bytes. */
+int h3b_denoise_step_latent(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                            const h3b_block_weights* blocks, const unsigned char* active,
+                            const float* mods, const h3b_latent_heads* heads, int reduce_after,
+                            int unpair_bypass, float sigma, float sigma_next, float* latent,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- reuse policies */
 /* Whole-velocity reuse and core-residual reuse (dothoosh.com, "Aggressive optimisation
  * levers"; aihot.vn section 4 "Speed/quality presets": --reuse and --core-reuse; the two
@@ -422,21 +466,28 @@ int h3b_gemm_bf16(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int
                   int rope_cols, int head_dim, h3b_bf16* out, void* ws, size_t ws_bytes,
                   void* stream);
 
-/* The projection GEMM in the forms of the folded block path (h3b_block_forward_folded):
+/* The projection GEMM in the forms of the folded block path (h3b_block_forward_folded) and
+ * with the Q/K RMSNorm:
  *   H3B_EPI_LN_ROPE, H3B_EPI_LN_GELU: A [M, K] is the raw bf16 residual and B the folded
  *     weights (h3b_fold_adaln); pre[r, j] = rstd_r (acc - mean_r fold_c[j]) + fold_dv[j],
  *     with mean_r and rstd_r = 1 / sqrt(var_r + ln_eps) merged from stats_in
  *     [M, K / 256] (h3b_row_stats form), then RoPE on columns < rope_cols (as
  *     H3B_EPI_BIAS_ROPE) or GELU_tanh; K % 256 == 0.  bias and gate are unused.
+ *   H3B_EPI_BIAS_ROPE: as in h3b_gemm_bf16.
  *   H3B_EPI_GATE_RESID: as in h3b_gemm_bf16, and the output rows' group statistics go to
  *     stats_out [M, N / 256] (h3b_row_stats form) when it is not NULL; N % 256 == 0.
+ * q_gain, k_gain (RoPE forms only; both or neither): each head_dim slice of columns
+ * [0, rope_cols / 2) (q) and [rope_cols / 2, rope_cols) (k) is RMS-normalised with
+ * eps = ln_eps and multiplied by the gains [head_dim] before the rotation (as the block
+ * does with q_norm, k_norm).
  * fold_c, fold_dv [N] fp32; other arguments as h3b_gemm_bf16.  All device. */
 enum { H3B_EPI_LN_ROPE = 4, H3B_EPI_LN_GELU = 5 };
 int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, int epilogue,
                      const h3b_bf16* bias, const float* gate, const float* fold_c,
                      const float* fold_dv, const float* stats_in, float* stats_out,
                      float ln_eps, const float* rope_cs, int rope_cols, int head_dim,
-                     h3b_bf16* out, void* ws, size_t ws_bytes, void* stream);
+                     const float* q_gain, const float* k_gain, h3b_bf16* out, void* ws,
+                     size_t ws_bytes, void* stream);
 
 /* Joint self-attention over one packed QKV buffer: qkv [n_tokens, 3 n_heads head_dim]
  * bf16 (q, then k, then v; head j at column j*head_dim of each), out [n_tokens,

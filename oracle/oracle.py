@@ -561,15 +561,15 @@ def final_head(x_l, final_mod, n_video: int, eps: float, w_head, b_head, dt=F64)
 def denoise_latent(lat0, blocks, mods, final_mod, heads, grid, n_audio: int, n_heads: int,
                    split, theta: float, eps: float, steps: int, run_steps: int, active=None,
                    reduce_after: int = -1, halved: bool = False, unpair_bypass: bool = True,
-                   dt=F64) -> np.ndarray:
+                   dt=F64, first_step: int = 0) -> np.ndarray:
     """The Euler loop on the latent: each step x = bf16(patch_embed(latent)) (the residual
     stream is stored in bf16), the block stack as in denoise(), then
     latent += (s' - s) final_head(x_L).  heads: dict with w_patch, b_patch, w_head,
-    b_head."""
+    b_head.  Runs steps first_step .. first_step + run_steps - 1 of the sigma grid."""
     sig = sigma_grid(steps, dt)
     lat = np.asarray(lat0, dt)
     nv = grid[0] * grid[1] * grid[2]
-    for i in range(run_steps):
+    for i in range(first_step, first_step + run_steps):
         x = patch_embed(lat, nv, heads["w_patch"], heads["b_patch"], dt)
         x_l = _core(x, blocks, mods, grid, n_audio, n_heads, split, theta, eps, active,
                     reduce_after, halved, unpair_bypass, dt)

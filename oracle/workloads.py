@@ -61,3 +61,21 @@ def denoise_reuse(cfg, blocks, final, c, x0, every: int, mode: str, dt=np.float6
               cfg.rope_theta, cfg.ln_eps, cfg.steps, every, active=active_mask(cfg, mods),
               reduce_after=cfg.reduce_after, halved=cfg.rope_halved,
               unpair_bypass=cfg.unpair_bypass, dt=dt)
+
+
+def denoise_latent(cfg, blocks, final, heads, c, lat0, run_steps: Optional[int] = None,
+                   dt=np.float64, trace: Optional[list] = None) -> np.ndarray:
+    """The Euler loop on the per-token latent (patch embedding, blocks, final heads)."""
+    mods = modulation_vectors(cfg, blocks, c)
+    fm = final_vectors(cfg, final, c)
+    steps = cfg.run_steps if run_steps is None else run_steps
+    lat = lat0
+    for i in range(steps):
+        lat = O.denoise_latent(lat, blocks, mods, fm, heads, cfg.grid, cfg.n_audio,
+                               cfg.n_heads, cfg.rope_split, cfg.rope_theta, cfg.ln_eps,
+                               cfg.steps, 1, active=active_mask(cfg, mods),
+                               reduce_after=cfg.reduce_after, halved=cfg.rope_halved,
+                               unpair_bypass=cfg.unpair_bypass, dt=dt, first_step=i)
+        if trace is not None:
+            trace.append(lat.copy())
+    return lat

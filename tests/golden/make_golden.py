@@ -22,7 +22,7 @@ from oracle import workloads  # noqa: E402
 from video_diffusion_transformer_03_b200 import synth  # noqa: E402
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-NAMES = ("dit512", "dit512_tokred", "dit256_halved")
+NAMES = ("dit512", "dit512_tokred", "dit256_halved", "dit512_qknorm", "dit512_latent")
 REUSE = {"dit512_reuse_velocity2": ("dit512", "velocity", 2),
          "dit512_reuse_core3": ("dit512", "core", 3)}
 
@@ -48,7 +48,12 @@ def make(name: str) -> None:
     x0 = f32(synth.latent_noise(cfg)).astype(np.float64)
     t0 = time.time()
     trace = []
-    workloads.denoise(cfg, blocks, final, c, x0, trace=trace)
+    if cfg.latent_channels:
+        heads = {k: f32(v).astype(np.float64) for k, v in synth.head_params(cfg).items()}
+        x0 = f32(synth.latent_state(cfg)).astype(np.float64)
+        workloads.denoise_latent(cfg, blocks, final, heads, c, x0, trace=trace)
+    else:
+        workloads.denoise(cfg, blocks, final, c, x0, trace=trace)
     mods = workloads.modulation_vectors(cfg, blocks, c)
     mask = workloads.active_mask(cfg, mods)
     rows = sample_rows(cfg)

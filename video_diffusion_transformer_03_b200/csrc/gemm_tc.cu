@@ -260,12 +260,62 @@ __device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int 
   }
 }
 
+// a[i] for i in 0..3 without indexing a register array by a runtime value.
+__device__ __forceinline__ float pick4(const float (&a)[4], int i) {
+  float v = a[0];
+#pragma unroll
+  for (int k = 1; k < 4; ++k) v = (i == k) ? a[k] : v;
+  return v;
+}
+
+// Q/K RMSNorm first pass of the single-CTA kernel (vectors read from global memory): the
+// reciprocal RMS of each head of this lane's row over a BN-column tile at col0.
+template <int BN, int EPI>
+__device__ __forceinline__ void qk_rms_pass_global(const GemmEpilogue& e, uint32_t tbase,
+                                                   int col0, const LnRow& ln,
+                                                   float (&qks)[4]) {
+  float ss[4] = {0.f, 0.f, 0.f, 0.f};
+  const int cpd = e.head_dim >> 5;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    tmem_wait_ld(r);
+    float v[32];
+    const int col = col0 + c * 32;
+    if constexpr (epi_ln_fold(EPI)) {
+      float cv[32], dv[32];
+      load_f32x32(e.fold_c + col, cv);
+      load_f32x32(e.bias_f32 + col, dv);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = fmaf(ln.rstd, fmaf(-ln.mu, cv[j], __uint_as_float(r[j])), dv[j]);
+    } else {
+      float b[32];
+      load_bf16x32(e.bias + col, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + b[j];
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) s = fmaf(v[j], v[j], s);
+    const int h = c / cpd;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ss[k] += (h == k) ? s : 0.f;
+  }
+  const float inv_hd = 1.0f / static_cast<float>(e.head_dim);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) qks[k] = rsqrtf(fmaf(ss[k], inv_hd, e.ln_eps));
+}
+
 // Epilogue of one 32-column chunk of one row.  ln: the row's statistics (LN-folded
-// kinds); sa: the row's running statistics of the stored output, or null.
+// kinds); sa: the row's running statistics of the stored output, or null; qk_s: the Q/K
+// RMSNorm scale of the chunk's head (RoPE kinds with gains).
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, int col,
                                                const uint32_t (&r)[32], const RowIn& in,
-                                               const LnRow& ln, StatAcc* sa, bool first) {
+                                               const LnRow& ln, StatAcc* sa, bool first,
+                                               float qk_s = 1.0f) {
   float v[32];
   if constexpr (EPI == kEpiInt8Deq) {
     const float rs = __ldg(e.row_scale + row);
@@ -301,12 +351,31 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + b[j];
   }
 
+  if constexpr (EPI == kEpiHeadEuler) {
+    float4* st = reinterpret_cast<float4*>(e.out_f32 + size_t(row) * e.ld_out + col);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 x = st[i];
+      x.x = fmaf(e.euler_dt, v[4 * i + 0], x.x);
+      x.y = fmaf(e.euler_dt, v[4 * i + 1], x.y);
+      x.z = fmaf(e.euler_dt, v[4 * i + 2], x.z);
+      x.w = fmaf(e.euler_dt, v[4 * i + 3], x.w);
+      st[i] = x;
+    }
+    return;
+  }
   if constexpr (epi_base(EPI) == kEpiGelu) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
   }
   if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
+      if (e.q_gain != nullptr) {
+        float gn[32];
+        load_f32x32((col < (e.rope_cols >> 1) ? e.q_gain : e.k_gain) + col % e.head_dim, gn);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= qk_s * gn[j];
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {  // 2 pairs per float4 (cos0, sin0, cos1, sin1)
         const float4 c = in.cs[i];
@@ -336,7 +405,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-  if constexpr (EPI == kEpiGateResid) {
+  if constexpr (EPI == kEpiGateResid || EPI == kEpiBias) {
     if (sa != nullptr) stat_add(*sa, pk, first);
   }
   uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -400,7 +469,13 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
     if (valid) ln = ln_row(p.epi, row);
   }
   StatAcc sa{0.f, 0.f, 0.f};
-  const bool want_stats = EPI == kEpiGateResid && BN == 256 && p.epi.stats_out != nullptr;
+  const bool want_stats =
+      (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
+  float qks[4] = {1.f, 1.f, 1.f, 1.f};
+  if constexpr (epi_base(EPI) == kEpiRope && !INT8) {
+    if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
+      qk_rms_pass_global<BN, EPI>(p.epi, tbase, col0, ln, qks);
+  }
   RowIn in[2];
   uint4 part[2][8];
   if (valid) load_row_in<EPI>(p.epi, row, col0, in[0]);
@@ -433,7 +508,8 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
     }
     if (valid)
       epilogue_chunk<EPI>(p.epi, row, col0 + c * 32, r, in[c & 1], ln,
-                          want_stats ? &sa : nullptr, c == 0);
+                          want_stats ? &sa : nullptr, c == 0,
+                          pick4(qks, (c * 32) / p.epi.head_dim));
   }
   if (want_stats && valid)
     p.epi.stats_out[size_t(row) * (p.epi.ld_out / 256) + col0 / 256] = stat_final(sa);
@@ -478,6 +554,13 @@ __device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, f
     }
     if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq)
       vec[kVecGate + i] = __ldg(e.gate + col);
+    if constexpr (epi_base(EPI) == kEpiRope) {
+      // Q/K RMSNorm gains of the column's head dimension (1 outside q and k, or when off)
+      float gn = 1.0f;
+      if (e.q_gain != nullptr && col < e.rope_cols)
+        gn = __ldg((col < (e.rope_cols >> 1) ? e.q_gain : e.k_gain) + col % e.head_dim);
+      vec[kVecGate + i] = gn;
+    }
   }
 }
 
@@ -512,15 +595,60 @@ __device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, i
   }
 }
 
+// Values before the activation / rotation of a bf16 chunk from staged vectors: acc + bias,
+// or the LN-folded form rstd (acc - mean c) + dv.
+template <int EPI>
+__device__ __forceinline__ void pre_values(const uint32_t (&r)[32], const float* vec,
+                                           const LnRow& ln, float (&v)[32]) {
+  if constexpr (epi_ln_fold(EPI)) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = fmaf(ln.rstd, fmaf(-ln.mu, vec[kVecScale + j], __uint_as_float(r[j])),
+                  vec[kVecBias + j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + vec[kVecBias + j];
+  }
+}
+
+// Q/K RMSNorm, first pass: the reciprocal RMS of each head of this lane's row in a
+// 32-column-chunk tile (heads of head_dim columns; the tile lies inside q, k or v).  The
+// scale of chunk c is qks[c * 32 / head_dim]; the chunks are re-read from TMEM.
+template <int BN, int EPI>
+__device__ __forceinline__ void qk_rms_pass(const GemmEpilogue& e, uint32_t tbase,
+                                            const float* vec, const LnRow& ln,
+                                            float (&qks)[4]) {
+  float ss[4] = {0.f, 0.f, 0.f, 0.f};
+  const int cpd = e.head_dim >> 5;  // chunks per head
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tbase + c * 32, r);
+    tmem_wait_ld(r);
+    float v[32];
+    pre_values<EPI>(r, vec + c * 32, ln, v);
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) s = fmaf(v[j], v[j], s);
+    const int h = c / cpd;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ss[k] += (h == k) ? s : 0.f;
+  }
+  const float inv_hd = 1.0f / static_cast<float>(e.head_dim);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) qks[k] = rsqrtf(fmaf(ss[k], inv_hd, e.ln_eps));
+}
+
 // Epilogue of one 32 x 32 chunk held one row per lane (lane L: row row0 + L, columns col +
 // [0, 32)); vec points at the chunk's first column in the staged vectors.  ln: this lane's
-// row statistics (LN-folded kinds); sa: its running output statistics, or null.
+// row statistics (LN-folded kinds); sa: its running output statistics, or null; qk_s: the
+// Q/K RMSNorm scale of the chunk's head (RoPE kinds with gains).
 template <int EPI>
 __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, int nrows,
                                                int col, const uint32_t (&r)[32],
                                                const RowIn& in, uint4* blk, const float* vec,
                                                int lane, const LnRow& ln, StatAcc* sa,
-                                               bool first) {
+                                               bool first, float qk_s = 1.0f) {
   const bool valid = lane < nrows;
   float v[32];
   if constexpr (EPI == kEpiInt8Deq) {
@@ -540,14 +668,35 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += vec[kVecBias + j];
     }
-  } else if constexpr (epi_ln_fold(EPI)) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      v[j] = fmaf(ln.rstd, fmaf(-ln.mu, vec[kVecScale + j], __uint_as_float(r[j])),
-                  vec[kVecBias + j]);
   } else {
+    pre_values<EPI>(r, vec, ln, v);
+  }
+  if constexpr (EPI == kEpiHeadEuler) {
+    // state += dt * v: the chunk's fp32 rows pass through the block, so each warp
+    // instruction reads and writes 4 whole rows of 128 bytes
+    __syncwarp();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + vec[kVecBias + j];
+    for (int i = 0; i < 8; ++i)
+      blk[blk32(lane, i)] = make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                                       __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int rr = k * 4 + (lane >> 3);
+      if (rr < nrows) {
+        float4* st =
+            reinterpret_cast<float4*>(e.out_f32 + size_t(row0 + rr) * e.ld_out + col) + (lane & 7);
+        const uint4 u = blk[blk32(rr, lane & 7)];
+        float4 x = *st;
+        x.x = fmaf(e.euler_dt, __uint_as_float(u.x), x.x);
+        x.y = fmaf(e.euler_dt, __uint_as_float(u.y), x.y);
+        x.z = fmaf(e.euler_dt, __uint_as_float(u.z), x.z);
+        x.w = fmaf(e.euler_dt, __uint_as_float(u.w), x.w);
+        *st = x;
+      }
+    }
+    __syncwarp();
+    return;
   }
   if constexpr (epi_base(EPI) == kEpiGelu) {
 #pragma unroll
@@ -555,6 +704,10 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
   }
   if constexpr (epi_base(EPI) == kEpiRope) {
     if (col < e.rope_cols) {
+      if (e.q_gain != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= qk_s * vec[kVecGate + j];
+      }
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -598,7 +751,7 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-  if constexpr (EPI == kEpiGateResid) {
+  if constexpr (EPI == kEpiGateResid || EPI == kEpiBias) {
     if (sa != nullptr) stat_add(*sa, pk, first);
   }
   __syncwarp();
@@ -635,7 +788,13 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
     if (lane < nrows) ln = ln_row(p.epi, row0 + lane);
   }
   StatAcc sa{0.f, 0.f, 0.f};
-  const bool want_stats = EPI == kEpiGateResid && BN == 256 && p.epi.stats_out != nullptr;
+  const bool want_stats =
+      (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
+  float qks[4] = {1.f, 1.f, 1.f, 1.f};
+  if constexpr (epi_base(EPI) == kEpiRope && !INT8) {
+    if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
+      qk_rms_pass<BN, EPI>(p.epi, tbase, vec, ln, qks);
+  }
   RowIn in[2];
   uint4 part[2][8];
   load_block_in<EPI>(p.epi, row0, nrows, col0, lane, in[0]);
@@ -667,7 +826,8 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
       }
     }
     epilogue_block<EPI>(p.epi, row0, nrows, col0 + c * 32, r, in[c & 1], blk, vec + c * 32,
-                        lane, ln, want_stats ? &sa : nullptr, c == 0);
+                        lane, ln, want_stats ? &sa : nullptr, c == 0,
+                        pick4(qks, (c * 32) / p.epi.head_dim));
   }
   if (want_stats && lane < nrows)
     p.epi.stats_out[size_t(row0 + lane) * (p.epi.ld_out / 256) + col0 / 256] = stat_final(sa);
@@ -1248,8 +1408,9 @@ int launch_impl(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int tiles = p.m_tiles * p.n_tiles;
   const int sk_ctas = std::min(ctx.num_sms, kMaxSkCtas);
   const long long iters = static_cast<long long>(tiles) * p.k_blocks;
+  // (the Q/K RMSNorm needs whole heads from one accumulator: no split tiles)
   const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
-                     iters >= 4LL * sk_ctas;
+                     iters >= 4LL * sk_ctas && epi.q_gain == nullptr;
   const bool use_sk = sk_ok && (forced_sched() >= 0 ? forced_sched() >= 1
                                                     : want_stream_k(tiles, ctx.num_sms, p.k_blocks));
   if (trace_gemm())
@@ -1338,7 +1499,7 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
   const int sk_tile0 = forced_sched() == 2 ? 0 : hybrid_tile0(tiles, sk_pairs);
   const long long iters = static_cast<long long>(tiles - sk_tile0) * p.k_blocks;
   const bool sk_ok = scratch != nullptr && scratch_bytes >= kScratchBytes &&
-                     iters >= 4LL * sk_pairs;
+                     iters >= 4LL * sk_pairs && epi.q_gain == nullptr;
   const bool use_sk =
       sk_ok && (forced_sched() >= 0 ? forced_sched() >= 1
                                     : want_stream_k(tiles, sk_pairs, p.k_blocks, sk_tile0));
@@ -1469,6 +1630,8 @@ int dispatch_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N,
       return launch_impl<BN, false, kEpiRopeLN>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     case kEpiGeluLN:
       return launch_impl<BN, false, kEpiGeluLN>(ctx, A, B, M, N, K, epi, ws, wsb, s);
+    case kEpiHeadEuler:
+      return launch_impl<BN, false, kEpiHeadEuler>(ctx, A, B, M, N, K, epi, ws, wsb, s);
     default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
   }
 }
@@ -1566,7 +1729,8 @@ int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int
   // Row statistics of the output need a tile that covers a whole 256-column group, and the
   // transposed kernel spreads a token's columns over several warps: 256-wide untransposed
   // tiles for them, and for the LN-folded kinds (row statistics read per row).
-  const bool row_stats = epi.stats_out != nullptr || epi_ln_fold(epi.kind);
+  const bool row_stats =
+      epi.stats_out != nullptr || epi_ln_fold(epi.kind) || epi.q_gain != nullptr;
   if (epi.stats_out != nullptr) tile = M >= 256 ? kPair256 : kSingle256;
   if (tile == kPair256 && !row_stats &&
       want_trans(ctx, M, N, K, scratch != nullptr && scratch_bytes >= kScratchBytes)) {
@@ -1610,6 +1774,10 @@ int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int
       case kEpiGeluLN:
         done = try_pair_bf16<kEpiGeluLN>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
                                          stream, &rc);
+        break;
+      case kEpiHeadEuler:
+        done = try_pair_bf16<kEpiHeadEuler>(bn, ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
+                                            stream, &rc);
         break;
       default: return set_error(-1, "gemm: unknown epilogue %d", epi.kind);
     }

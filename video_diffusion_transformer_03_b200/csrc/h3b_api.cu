@@ -150,6 +150,9 @@ int check_weights(const h3b_block_weights* w) {
   const void* p[8] = {w->w_qkv, w->b_qkv, w->w_o, w->b_o, w->w_fc1, w->b_fc1, w->w_fc2, w->b_fc2};
   for (const void* q : p)
     if (!q || !al16(q)) return set_error(H3B_EINVAL, "block weight pointer NULL or not 16-byte aligned");
+  if ((w->q_norm == nullptr) != (w->k_norm == nullptr) || (w->q_norm && !al16(w->q_norm)) ||
+      (w->k_norm && !al16(w->k_norm)))
+    return set_error(H3B_EINVAL, "q_norm and k_norm: both or neither, 16-byte aligned");
   return H3B_OK;
 }
 
@@ -200,6 +203,9 @@ int block_forward_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_wei
   GemmEpilogue e;
   e.kind = kEpiRope;
   e.bias = reinterpret_cast<const bf16*>(w->b_qkv);
+  e.q_gain = w->q_norm;
+  e.k_gain = w->k_norm;
+  e.ln_eps = d->ln_eps;
   e.rope_cs = rope_cs;
   e.rope_cols = 2 * D;
   e.head_dim = d->head_dim;
@@ -255,6 +261,8 @@ int block_forward_folded_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_bl
   e.kind = kEpiRopeLN;
   e.bias_f32 = w->d_qkv;
   e.fold_c = w->c_qkv;
+  e.q_gain = w->q_norm;
+  e.k_gain = w->k_norm;
   e.stats_in = stats;
   e.stats_parts = D / 256;
   e.ln_eps = d->ln_eps;
@@ -314,11 +322,13 @@ struct StepBufs {
   bf16* x_red;      // [N_red, d]
   float2* stats;    // [N, d / 256] row statistics of the residual (folded blocks)
   float2* stats_red;  // [N_red, d / 256]
+  bf16* lat;        // [N, c_lat] the latent as the patch embedding's operand (latent steps)
   void* arena;      // block arena sized for N tokens
   size_t total;
 };
 
-StepBufs carve_step(const h3b_dims* d, const h3b_grid* g, bool reduce, void* ws) {
+StepBufs carve_step(const h3b_dims* d, const h3b_grid* g, bool reduce, void* ws,
+                    int c_lat = 0) {
   const size_t n = size_t(g->t) * g->h * g->w + g->n_audio;
   const size_t nr = size_t(g->t) * g->h * (g->w / 2) + g->n_audio;
   uint8_t* p = static_cast<uint8_t*>(ws);
@@ -338,9 +348,49 @@ StepBufs carve_step(const h3b_dims* d, const h3b_grid* g, bool reduce, void* ws)
     b.x_red = reinterpret_cast<bf16*>(take(nr * d->d * 2));
     b.stats_red = reinterpret_cast<float2*>(take(nr * (d->d / 256) * sizeof(float2)));
   }
+  if (c_lat > 0) b.lat = reinterpret_cast<bf16*>(take(n * size_t(c_lat) * 2));
   b.arena = take(arena_bytes(d, static_cast<int>(n)));
   b.total = off;
   return b;
+}
+
+// The active blocks in their folded form on b.x_res (row statistics in b.stats), with the
+// token pairing after `reduce_after` executed blocks and the restore at the end: b.x_res
+// then holds x_L.  *stats_valid tells whether b.stats still describes it (not after a
+// restore).
+int folded_stack(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g,
+                 const std::vector<int>& order, const h3b_block_weights* blocks,
+                 const float* mods, int reduce_after, int unpair_bypass, const StepBufs& b,
+                 cudaStream_t s, bool* stats_valid) {
+  const int D = d->d;
+  const int n = g->t * g->h * g->w + g->n_audio;
+  const int n_red = g->t * g->h * (g->w / 2) + g->n_audio;
+  int rc;
+  bf16* cur = b.x_res;
+  float2* cur_stats = b.stats;
+  int cur_n = n;
+  const float* rope = b.rope;
+  for (size_t k = 0; k < order.size(); ++k) {
+    const int blk = order[k];
+    if ((rc = block_forward_folded_impl(ctx, d, &blocks[blk], mods + size_t(blk) * 6 * D, rope,
+                                        cur_n, cur, cur_stats, b.arena, s)))
+      return rc;
+    if (reduce_after > 0 && int(k + 1) == reduce_after && k + 1 < order.size()) {
+      if ((rc = launch_token_pair(b.x_res, b.x_red, g->t, g->h, g->w, g->n_audio, D, s)))
+        return rc;
+      cur = b.x_red;
+      cur_n = n_red;
+      cur_stats = b.stats_red;
+      rope = b.rope_red;
+      if ((rc = launch_row_stats(cur, cur_n, D, cur_stats, s))) return rc;
+    }
+  }
+  *stats_valid = cur != b.x_red;
+  if (cur == b.x_red &&
+      (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
+                                g->w, g->n_audio, D, s)))
+    return rc;
+  return H3B_OK;
 }
 
 int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, int n_blocks,
@@ -373,28 +423,9 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
   if (folded && !order.empty()) {
     // every block reads the raw residual and its row statistics (no LayerNorm pass)
     if ((rc = launch_state_to_residual(x_state, n, D, b.x_res, b.stats, s))) return rc;
-    bf16* cur = b.x_res;
-    float2* cur_stats = b.stats;
-    int cur_n = n;
-    const float* rope = b.rope;
-    for (size_t k = 0; k < order.size(); ++k) {
-      const int blk = order[k];
-      if ((rc = block_forward_folded_impl(ctx, d, &blocks[blk], mods + size_t(blk) * 6 * D, rope,
-                                          cur_n, cur, cur_stats, b.arena, s)))
-        return rc;
-      if (may_reduce && int(k + 1) == reduce_after && k + 1 < order.size()) {
-        if ((rc = launch_token_pair(b.x_res, b.x_red, g->t, g->h, g->w, g->n_audio, D, s)))
-          return rc;
-        cur = b.x_red;
-        cur_n = n_red;
-        cur_stats = b.stats_red;
-        rope = b.rope_red;
-        if ((rc = launch_row_stats(cur, cur_n, D, cur_stats, s))) return rc;
-      }
-    }
-    if (cur == b.x_red &&
-        (rc = launch_token_unpair(b.x_red, b.x_res, unpair_bypass ? b.x_res : nullptr, g->t, g->h,
-                                  g->w, g->n_audio, D, s)))
+    bool stats_valid = false;
+    if ((rc = folded_stack(ctx, d, g, order, blocks, mods, reduce_after, unpair_bypass, b, s,
+                           &stats_valid)))
       return rc;
     if (v_out || r_out)
       return launch_final_euler_keep(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
@@ -437,6 +468,69 @@ int denoise_step_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g, i
     return launch_final_euler_keep(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma,
                                    x_state, v_out, r_out, s);
   return launch_final_euler(b.x_res, n, nv, D, d->ln_eps, final_mod, sigma_next - sigma, x_state, s);
+}
+
+// One Euler step on the per-token latent: patch embedding per stream into the residual
+// (its epilogue writing the row statistics), the folded block stack, the final AdaLN
+// folded into each stream's head with the Euler update in the head's epilogue.
+int denoise_step_latent_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_grid* g,
+                             int n_blocks, const h3b_block_weights* blocks,
+                             const unsigned char* active, const float* mods,
+                             const h3b_latent_heads* hd, int reduce_after, int unpair_bypass,
+                             float sigma, float sigma_next, float* latent, const StepBufs& b,
+                             cudaStream_t s) {
+  const int D = d->d, C = hd->c_lat;
+  const int nv = g->t * g->h * g->w;
+  const int n = nv + g->n_audio;
+  const int parts = D / 256;
+  int rc;
+  if ((rc = launch_rope_table(g->t, g->h, g->w, g->n_audio, g->rope_halved, 0, d->head_dim,
+                              d->rope_split, d->rope_theta, b.rope, s)))
+    return rc;
+  if (reduce_after > 0 &&
+      (rc = launch_rope_table(g->t, g->h, g->w, g->n_audio, g->rope_halved, 1, d->head_dim,
+                              d->rope_split, d->rope_theta, b.rope_red, s)))
+    return rc;
+  if ((rc = launch_f32_to_bf16(latent, static_cast<long long>(n) * C, b.lat, s))) return rc;
+  const int rows[2] = {nv, g->n_audio};
+  const int first[2] = {0, nv};
+  for (int st = 0; st < 2; ++st) {  // patch embedding, video rows then audio rows
+    GemmEpilogue e;
+    e.kind = kEpiBias;
+    e.bias = reinterpret_cast<const bf16*>(hd->b_patch[st]);
+    e.out = b.x_res + size_t(first[st]) * D;
+    e.ld_out = D;
+    e.stats_out = b.stats + size_t(first[st]) * parts;
+    if ((rc = launch_gemm_bf16(ctx, b.lat + size_t(first[st]) * C,
+                               reinterpret_cast<const bf16*>(hd->w_patch[st]), rows[st], D, C, e,
+                               b.arena, 0, s)))
+      return rc;
+  }
+  std::vector<int> order;
+  for (int i = 0; i < n_blocks; ++i)
+    if (!active || active[i]) order.push_back(i);
+  bool stats_valid = true;
+  if (!order.empty() && (rc = folded_stack(ctx, d, g, order, blocks, mods, reduce_after,
+                                           unpair_bypass, b, s, &stats_valid)))
+    return rc;
+  if (!stats_valid && (rc = launch_row_stats(b.x_res, n, D, b.stats, s))) return rc;
+  for (int st = 0; st < 2; ++st) {  // final AdaLN + head + Euler, per stream
+    GemmEpilogue e;
+    e.kind = kEpiHeadEuler;
+    e.bias_f32 = hd->dv_head[st];
+    e.fold_c = hd->c_head[st];
+    e.stats_in = b.stats + size_t(first[st]) * parts;
+    e.stats_parts = parts;
+    e.ln_eps = d->ln_eps;
+    e.out_f32 = latent + size_t(first[st]) * C;
+    e.ld_out = C;
+    e.euler_dt = sigma_next - sigma;
+    if ((rc = launch_gemm_bf16(ctx, b.x_res + size_t(first[st]) * D,
+                               reinterpret_cast<const bf16*>(hd->w_head_fold[st]), rows[st], C, D,
+                               e, b.arena, 0, s)))
+      return rc;
+  }
+  return H3B_OK;
 }
 
 int check_step_args(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
@@ -697,6 +791,46 @@ int h3b_denoise_step(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
   return denoise_step_impl(ctx, dims, grid, n_blocks, blocks, active, mods, final_mod,
                            reduce_after, unpair_bypass, sigma, sigma_next, x_state, b,
                            static_cast<cudaStream_t>(stream));
+}
+
+size_t h3b_denoise_latent_workspace_size(const h3b_dims* dims, const h3b_grid* grid, int reduce,
+                                         int c_lat) {
+  if (check_dims(dims) || check_grid(grid, reduce != 0) || c_lat <= 0 || c_lat % 128) return 0;
+  return carve_step(dims, grid, reduce != 0, nullptr, c_lat).total;
+}
+
+int h3b_denoise_step_latent(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
+                            const h3b_block_weights* blocks, const unsigned char* active,
+                            const float* mods, const h3b_latent_heads* heads, int reduce_after,
+                            int unpair_bypass, float sigma, float sigma_next, float* latent,
+                            void* ws, size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_grid(grid, reduce_after > 0))) return rc;
+  if (!heads || heads->c_lat <= 0 || heads->c_lat % 128 || heads->c_lat > 4096)
+    return set_error(H3B_EINVAL, "denoise_step_latent: c_lat must be a positive multiple of 128");
+  for (int st = 0; st < 2; ++st) {
+    const void* p[6] = {heads->w_patch[st], heads->b_patch[st], heads->w_head_fold[st],
+                        heads->c_head[st], heads->dv_head[st], nullptr};
+    for (int i = 0; i < 5; ++i)
+      if (!p[i] || !al16(p[i]))
+        return set_error(H3B_EINVAL, "denoise_step_latent: head pointer NULL or misaligned");
+  }
+  if (n_blocks < 0 || (n_blocks > 0 && (!blocks || !mods)))
+    return set_error(H3B_EINVAL, "bad block list");
+  for (int i = 0; i < n_blocks; ++i)
+    if ((!active || active[i]) && ((rc = check_weights(&blocks[i])) || (rc = check_fold(&blocks[i]))))
+      return rc;
+  if (!latent || !al16(latent)) return set_error(H3B_EINVAL, "latent NULL or misaligned");
+  const StepBufs need = carve_step(dims, grid, reduce_after > 0, nullptr, heads->c_lat);
+  if (!ws || !al16(ws) || ws_bytes < need.total)
+    return set_error(H3B_EWORKSPACE, "workspace of %zu bytes needed, %zu given", need.total,
+                     ws_bytes);
+  const StepBufs b = carve_step(dims, grid, reduce_after > 0, ws, heads->c_lat);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return denoise_step_latent_impl(ctx, dims, grid, n_blocks, blocks, active, mods, heads,
+                                  reduce_after, unpair_bypass, sigma, sigma_next, latent, b,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 int h3b_denoise_step_keep(const h3b_dims* dims, const h3b_grid* grid, int n_blocks,
@@ -1088,7 +1222,8 @@ int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, 
                      const h3b_bf16* bias, const float* gate, const float* fold_c,
                      const float* fold_dv, const float* stats_in, float* stats_out,
                      float ln_eps, const float* rope_cs, int rope_cols, int head_dim,
-                     h3b_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+                     const float* q_gain, const float* k_gain, h3b_bf16* out, void* ws,
+                     size_t ws_bytes, void* stream) {
   if (M < 0 || K <= 0 || K % 64 || N <= 0 || N % 128)
     return set_error(H3B_EINVAL, "gemm_bf16_ln: K=%d must be a multiple of 64, N=%d of 128", K, N);
   if (!A || !B || !out || !al16(A) || !al16(B) || !al16(out) || (ws && !al16(ws)))
@@ -1113,6 +1248,16 @@ int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, 
     e.rope_cs = rope_cs;
     e.rope_cols = rope_cols;
     e.head_dim = head_dim;
+  } else if (epilogue == H3B_EPI_BIAS_ROPE) {
+    if (!bias || !al16(bias) || !rope_cs || !al16(rope_cs) || (head_dim != 64 && head_dim != 128) ||
+        rope_cols < 0 || rope_cols % head_dim || rope_cols > N)
+      return set_error(H3B_EINVAL, "gemm_bf16_ln: bad bias / RoPE arguments");
+    e.kind = kEpiRope;
+    e.bias = reinterpret_cast<const bf16*>(bias);
+    e.ln_eps = ln_eps;
+    e.rope_cs = rope_cs;
+    e.rope_cols = rope_cols;
+    e.head_dim = head_dim;
   } else if (epilogue == H3B_EPI_GATE_RESID) {
     if (!bias || !gate || !al16(bias) || !al16(gate) || (stats_out && (N % 256 || !al16(stats_out))))
       return set_error(H3B_EINVAL, "gemm_bf16_ln: gated residual needs bias, gate (and N %% 256 == 0 for stats)");
@@ -1123,6 +1268,12 @@ int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, 
   } else {
     return set_error(H3B_EINVAL, "gemm_bf16_ln: epilogue %d", epilogue);
   }
+  if ((q_gain == nullptr) != (k_gain == nullptr) ||
+      (q_gain && (e.kind != kEpiRope && e.kind != kEpiRopeLN)) ||
+      (q_gain && (!al16(q_gain) || !al16(k_gain) || e.rope_cols % 2 || (e.rope_cols / 2) % e.head_dim)))
+    return set_error(H3B_EINVAL, "gemm_bf16_ln: q_gain / k_gain need a RoPE form, both or neither");
+  e.q_gain = q_gain;
+  e.k_gain = k_gain;
   DevCtx ctx;
   if (int rc = get_ctx(&ctx)) return rc;
   return launch_gemm_bf16(ctx, reinterpret_cast<const bf16*>(A), reinterpret_cast<const bf16*>(B),

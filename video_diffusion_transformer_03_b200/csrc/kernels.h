@@ -36,13 +36,16 @@ enum GemmEpi : int {
   // merged from stats_in, then the base epilogue
   kEpiRopeLN = 5,     // out = bf16(rope(pre)) on columns < rope_cols
   kEpiGeluLN = 6,     // out = bf16(gelu_tanh(pre))
+  kEpiHeadEuler = 7,  // out_f32 += euler_dt * pre (fp32 state, in place): a final head
 };
 
 // The base epilogue of a kind (the LN-folded kinds share their base's arithmetic).
 __host__ __device__ constexpr int epi_base(int k) {
   return k == kEpiRopeLN ? kEpiRope : k == kEpiGeluLN ? kEpiGelu : k;
 }
-__host__ __device__ constexpr bool epi_ln_fold(int k) { return k == kEpiRopeLN || k == kEpiGeluLN; }
+__host__ __device__ constexpr bool epi_ln_fold(int k) {
+  return k == kEpiRopeLN || k == kEpiGeluLN || k == kEpiHeadEuler;
+}
 
 struct GemmEpilogue {
   int kind = kEpiBias;
@@ -57,15 +60,23 @@ struct GemmEpilogue {
   const float* row_scale = nullptr;  // int8 path, [M]
   const float* col_scale = nullptr;  // int8 path, [N]
   int32_t* acc_out = nullptr;        // int8 path, [M, N] or null
-  // kEpiGateResid: per row, (mean, M2) of each 256-column group of the stored bf16 output,
-  // [M, ld_out / 256]; or null
+  // kEpiGateResid, kEpiBias: per row, (mean, M2) of each 256-column group of the stored
+  // bf16 output, [M, ld_out / 256]; or null
   float2* stats_out = nullptr;
+  // kEpiHeadEuler: the fp32 state [M, ld_out] updated in place, and the Euler step
+  float* out_f32 = nullptr;
+  float euler_dt = 0.f;
   // LN-folded kinds: the A rows' group statistics [M, stats_parts], the folded weights'
   // row sums c [N] (dv [N] comes in bias_f32) and the LayerNorm epsilon
   const float2* stats_in = nullptr;
   const float* fold_c = nullptr;
   int stats_parts = 0;
   float ln_eps = 1e-6f;
+  // RoPE kinds: per-head RMSNorm of q (columns < rope_cols / 2) and k (up to rope_cols)
+  // before the rotation, gains [head_dim] each (eps = ln_eps); both null = off.  Runs
+  // data-parallel (the norm needs the whole head from one accumulator).
+  const float* q_gain = nullptr;
+  const float* k_gain = nullptr;
 };
 
 // Kernel scratch: one caller buffer per stream, used by one kernel at a time.  Layout:
@@ -139,6 +150,8 @@ int launch_final_euler_keep(const bf16* x_l, int n, int n_video, int d, float ep
 int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float eps,
                             const float* final_mod, float dt_sigma, float* x_state,
                             cudaStream_t stream);
+// dst = bf16(src), n elements (n % 8 == 0)
+int launch_f32_to_bf16(const float* src, long long n, bf16* dst, cudaStream_t stream);
 // x_state += dt * v (n elements, n % 4 == 0)
 int launch_euler_axpy(const float* v, long long n, float dt_sigma, float* x_state,
                       cudaStream_t stream);

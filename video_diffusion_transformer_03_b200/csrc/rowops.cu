@@ -217,6 +217,17 @@ __global__ void __launch_bounds__(128) k_final_euler_ex(const bf16* __restrict__
   }
 }
 
+// dst = bf16(src) over n8 groups of 8 values (the latent as a GEMM operand).
+__global__ void __launch_bounds__(256) k_f32_to_bf16(const float* __restrict__ src, long long n8,
+                                                     bf16* __restrict__ dst) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float f[8];
+    load8f(src + i * 8, f);
+    reinterpret_cast<uint4*>(dst)[i] = pack8(f);
+  }
+}
+
 // x_state += dt * v over n4 float4 elements (a skipped step of whole-velocity reuse).
 __global__ void __launch_bounds__(256) k_euler_axpy(const float4* __restrict__ v, long long n4,
                                                     float dt, float4* __restrict__ xs) {
@@ -604,6 +615,14 @@ int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float 
                              nullptr, r_in, n, n_video, eps, final_mod, dt_sigma, x_state,
                              nullptr, nullptr)));
   return check_launch("core_reuse_final");
+}
+
+int launch_f32_to_bf16(const float* src, long long n, bf16* dst, cudaStream_t stream) {
+  const long long n8 = n / 8;
+  if (n8 <= 0) return 0;
+  const int grid = static_cast<int>(std::min<long long>((n8 + 255) / 256, 148 * 8));
+  k_f32_to_bf16<<<grid, 256, 0, stream>>>(src, n8, dst);
+  return check_launch("f32_to_bf16");
 }
 
 int launch_euler_axpy(const float* v, long long n, float dt_sigma, float* x_state,

@@ -41,10 +41,17 @@ class Grid(ctypes.Structure):
 
 WEIGHT_FIELDS = ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2")
 FOLD_FIELDS = ("w_qkv_fold", "c_qkv", "d_qkv", "w_fc1_fold", "c_fc1", "d_fc1")
+QK_FIELDS = ("q_norm", "k_norm")
 
 
 class BlockWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS + FOLD_FIELDS]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS + FOLD_FIELDS + QK_FIELDS]
+
+
+class LatentHeads(ctypes.Structure):
+    _fields_ = [("c_lat", ctypes.c_int), ("w_patch", ctypes.c_void_p * 2),
+                ("b_patch", ctypes.c_void_p * 2), ("w_head_fold", ctypes.c_void_p * 2),
+                ("c_head", ctypes.c_void_p * 2), ("dv_head", ctypes.c_void_p * 2)]
 
 
 _P = ctypes.c_void_p
@@ -83,6 +90,12 @@ _SIGS = {
     "h3b_denoise_host_pipelined": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                                         ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _I,
                                         _I, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "h3b_denoise_latent_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                                                _I]),
+    "h3b_denoise_step_latent": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
+                                     ctypes.POINTER(BlockWeights), _P, _P,
+                                     ctypes.POINTER(LatentHeads), _I, _I, _F, _F, _P, _P, _SZ,
+                                     _P]),
     "h3b_reuse_schedule": (_I, [_I, _I, _P]),
     "h3b_denoise_step_keep": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                                    ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P,
@@ -94,7 +107,7 @@ _SIGS = {
     "h3b_fc2_int8_row": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "h3b_gemm_bf16": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P]),
     "h3b_gemm_bf16_ln": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _F, _P, _I, _I,
-                              _P, _P, _SZ, _P]),
+                              _P, _P, _P, _P, _SZ, _P]),
     "h3b_attention": (_I, [_P, _I, _I, _I, _P, _P, _SZ, _P]),
     "h3b_layer_mask": (_I, [_P, _I, _I, _I, _P]),
 }
@@ -173,8 +186,13 @@ def make_block_weights(p) -> BlockWeights:
     if folded:
         for k in FOLD_FIELDS:
             _dev(p[k], torch.bfloat16 if k.startswith("w_") else torch.float32, k)
+    qk = all(p.get(k) is not None for k in QK_FIELDS)
+    if qk:
+        for k in QK_FIELDS:
+            _dev(p[k], torch.float32, k)
     return BlockWeights(*[_ptr(p[k]) for k in WEIGHT_FIELDS],
-                        *[_ptr(p[k]) if folded else None for k in FOLD_FIELDS])
+                        *[_ptr(p[k]) if folded else None for k in FOLD_FIELDS],
+                        *[_ptr(p[k]) if qk else None for k in QK_FIELDS])
 
 
 def gemm_workspace_size() -> int:
@@ -357,6 +375,36 @@ def denoise_step(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active,
     del keep
 
 
+def make_latent_heads(c_lat: int, t) -> LatentHeads:
+    """t: mapping with per-stream lists of device tensors w_patch, b_patch (bf16),
+    w_head_fold (bf16), c_head, dv_head (fp32), each of length 2 (video, audio)."""
+    h = LatentHeads()
+    h.c_lat = c_lat
+    for name in ("w_patch", "b_patch", "w_head_fold", "c_head", "dv_head"):
+        arr = getattr(h, name)
+        for st in range(2):
+            arr[st] = _ptr(t[name][st])
+    return h
+
+
+def denoise_latent_workspace_size(dims: Dims, grid: Grid, reduce: bool, c_lat: int) -> int:
+    return lib.h3b_denoise_latent_workspace_size(ctypes.byref(dims), ctypes.byref(grid),
+                                                 int(bool(reduce)), c_lat)
+
+
+def denoise_step_latent(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], active, mods,
+                        heads: LatentHeads, reduce_after: int, unpair_bypass: bool, sigma: float,
+                        sigma_next: float, latent, ws, stream=None) -> None:
+    _dev(latent, torch.float32, "latent")
+    arr = _blocks_array(blocks)
+    keep, mask = _mask_array(active, len(blocks))
+    _check(lib.h3b_denoise_step_latent(ctypes.byref(dims), ctypes.byref(grid), len(blocks), arr,
+                                       mask, _ptr(mods), ctypes.byref(heads), reduce_after,
+                                       int(bool(unpair_bypass)), sigma, sigma_next, _ptr(latent),
+                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+    del keep
+
+
 def reuse_schedule(steps: int, every: int) -> np.ndarray:
     """Host policy: which of `steps` Euler steps run the model (h3b_reuse_schedule)."""
     out = (ctypes.c_ubyte * max(steps, 1))()
@@ -465,17 +513,18 @@ def gemm_bf16(A, B, epilogue, bias, out, gate=None, rope_cs=None, rope_cols=0, h
 
 def gemm_bf16_ln(A, B, epilogue, out, bias=None, gate=None, fold_c=None, fold_dv=None,
                  stats_in=None, stats_out=None, ln_eps=1e-6, rope_cs=None, rope_cols=0,
-                 head_dim=128, ws=None, stream=None) -> None:
+                 head_dim=128, q_gain=None, k_gain=None, ws=None, stream=None) -> None:
     """The folded block's GEMM forms (h3b_gemm_bf16_ln): EPI_LN_ROPE / EPI_LN_GELU read the
-    raw residual A with its row statistics stats_in; EPI_GATE_RESID may write stats_out."""
+    raw residual A with its row statistics stats_in; EPI_GATE_RESID may write stats_out;
+    the RoPE forms take optional Q/K RMSNorm gains."""
     _dev(A, torch.bfloat16, "A"); _dev(B, torch.bfloat16, "B"); _dev(out, torch.bfloat16, "out")
     M, K = A.shape
     N = B.shape[0]
     wp, wb = _wsargs(ws)
     _check(lib.h3b_gemm_bf16_ln(_ptr(A), _ptr(B), M, N, K, epilogue, _ptr(bias), _ptr(gate),
                                 _ptr(fold_c), _ptr(fold_dv), _ptr(stats_in), _ptr(stats_out),
-                                ln_eps, _ptr(rope_cs), rope_cols, head_dim, _ptr(out), wp, wb,
-                                _stream(stream)))
+                                ln_eps, _ptr(rope_cs), rope_cols, head_dim, _ptr(q_gain),
+                                _ptr(k_gain), _ptr(out), wp, wb, _stream(stream)))
 
 
 def attention(qkv, n_heads, head_dim, out, ws=None, stream=None) -> None:

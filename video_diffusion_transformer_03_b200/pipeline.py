@@ -64,8 +64,33 @@ class DiTDenoiser:
             mask = h3b.layer_mask(self.mods.cpu().numpy(), cfg.active_count)
             self.active = [bool(m) for m in mask]
         self.reduce = cfg.reduce_after > 0
-        self.ws = h3b.workspace(h3b.denoise_workspace_size(self.dims, self.grid, self.reduce),
-                                self.device)
+        self.latent = cfg.latent_channels > 0
+        if self.latent:
+            # patch embedding and heads per stream; each head gets its stream's final AdaLN
+            # folded in (the blocks must be folded too)
+            if not fold:
+                raise ValueError("the latent step runs the folded block form")
+            hp = {k: v.to(self.device) for k, v in synth.head_params(cfg, gen_device).items()}
+            self.host_heads = {k: v.cpu() for k, v in hp.items()} if keep_host_params else None
+            self.heads_t = {"w_patch": [hp["w_patch"][s].contiguous() for s in range(2)],
+                            "b_patch": [hp["b_patch"][s].contiguous() for s in range(2)],
+                            "w_head_fold": [], "c_head": [], "dv_head": []}
+            for st in range(2):
+                w, b = hp["w_head"][st].contiguous(), hp["b_head"][st].contiguous()
+                wo = torch.empty_like(w)
+                c = torch.empty(w.shape[0], dtype=torch.float32, device=self.device)
+                dv = torch.empty_like(c)
+                h3b.fold_adaln(w, b, self.final_mod[st, 0].contiguous(),
+                               self.final_mod[st, 1].contiguous(), wo, c, dv)
+                self.heads_t["w_head_fold"].append(wo)
+                self.heads_t["c_head"].append(c)
+                self.heads_t["dv_head"].append(dv)
+            self.heads = h3b.make_latent_heads(cfg.latent_channels, self.heads_t)
+            nbytes = h3b.denoise_latent_workspace_size(self.dims, self.grid, self.reduce,
+                                                       cfg.latent_channels)
+        else:
+            nbytes = h3b.denoise_workspace_size(self.dims, self.grid, self.reduce)
+        self.ws = h3b.workspace(nbytes, self.device)
 
     @property
     def n_tokens(self) -> int:
@@ -76,7 +101,14 @@ class DiTDenoiser:
         return 1.0 - i / s, 1.0 - (i + 1) / s
 
     def step(self, x_state: torch.Tensor, i: int, stream=None) -> None:
+        """One Euler step on x_state: [N, d] model-space state, or the [N, C] latent for a
+        latent workload."""
         sg, sn = self.sigmas(i)
+        if self.latent:
+            h3b.denoise_step_latent(self.dims, self.grid, self.weights, self.active, self.mods,
+                                    self.heads, self.cfg.reduce_after, self.cfg.unpair_bypass,
+                                    sg, sn, x_state, self.ws, stream)
+            return
         h3b.denoise_step(self.dims, self.grid, self.weights, self.active, self.mods,
                          self.final_mod, self.cfg.reduce_after, self.cfg.unpair_bypass, sg, sn,
                          x_state, self.ws, stream)

@@ -33,8 +33,10 @@ PARAM_STD = 0.02
 
 # Order of the per-block tensors; the index is part of each tensor's seed.
 BLOCK_TENSORS = ("w_qkv", "b_qkv", "w_o", "b_o", "w_fc1", "b_fc1", "w_fc2", "b_fc2",
-                 "w_ada", "b_ada")
+                 "w_ada", "b_ada", "q_norm", "k_norm")
+QK_GAIN_STD = 0.1  # Q/K RMSNorm gains ~ 1 + N(0, 0.1)
 _FINAL_TENSORS = ("w_fin", "b_fin")
+_HEAD_TENSORS = ("w_patch", "b_patch", "w_head", "b_head")
 _COND_IDX = 100
 _NOISE_IDX = 101
 _INT8_IDX = {"act": 200, "w": 201, "gate": 202, "resid": 203, "bias": 204}
@@ -62,6 +64,9 @@ class DiTConfig:
     n_active: Optional[int] = None      # layer thinning: active blocks (None = all)
     rope_halved: bool = False           # spatial RoPE coordinates halved
     unpair_bypass: bool = True          # bypass restore (False: duplicate)
+    qk_norm: bool = False               # per-head Q/K RMSNorm gains in every block
+    latent_channels: int = 0            # > 0: the state is a per-token latent of this many
+                                        # channels, with patch embedding and final heads
 
     @property
     def n_video(self) -> int:
@@ -116,6 +121,21 @@ CONFIGS: Dict[str, DiTConfig] = {
     # 768x1344: 11 latent frames of 24x42 tokens + 256 audio tokens, 50 blocks, 4 steps
     "dit768x1344": _c("dit768x1344", n_blocks=50, grid=(11, 24, 42), n_audio=256, steps=4,
                       run_steps=4, seed=3, **_BIG),
+    # the 512x512 workload with per-head Q/K RMSNorm before RoPE in every block (the
+    # QKV-tile RMS normalisation of the pages' int8 path); same weights as dit512 otherwise
+    "dit512_qknorm": _c("dit512_qknorm", n_blocks=8, grid=(6, 16, 16), n_audio=64, steps=4,
+                        run_steps=4, seed=1, qk_norm=True, **_BIG),
+    # the 512x512 workload on a 128-channel per-token latent: patch embedding and the
+    # final heads (AdaLN folded into the head) around the same 8 blocks
+    "dit512_latent": _c("dit512_latent", n_blocks=8, grid=(6, 16, 16), n_audio=64, steps=4,
+                        run_steps=4, seed=1, latent_channels=128, **_BIG),
+    "tiny_latent": _c("tiny_latent", d=256, n_heads=4, head_dim=64, d_ff=1024, c_dim=256,
+                      rope_split=(16, 24, 24), n_blocks=1, grid=(2, 4, 4), n_audio=8,
+                      steps=4, run_steps=2, seed=0, latent_channels=128),
+    # the tiny workload with Q/K RMSNorm
+    "tiny_qknorm": _c("tiny_qknorm", d=256, n_heads=4, head_dim=64, d_ff=1024, c_dim=256,
+                      rope_split=(16, 24, 24), n_blocks=1, grid=(2, 4, 4), n_audio=8,
+                      steps=4, run_steps=1, seed=0, qk_norm=True),
 }
 
 INT8_CONFIG = Int8Config(name="fc2_int8_row", M=8192, K=12288, n_out=3072, seed=4)
@@ -136,13 +156,20 @@ def _param(shape, seed, block, idx, device, std=PARAM_STD) -> torch.Tensor:
 
 
 def block_params(cfg: DiTConfig, block: int, device="cpu") -> Dict[str, torch.Tensor]:
-    """Parameters of one block, weights as [out, in] row-major bf16."""
+    """Parameters of one block, weights as [out, in] row-major bf16; with cfg.qk_norm also
+    the Q/K RMSNorm gains q_norm, k_norm [head_dim] (1 + N(0, 0.1), bf16-valued fp32)."""
     d, f, c = cfg.d, cfg.d_ff, cfg.c_dim
     shapes = {"w_qkv": (3 * d, d), "b_qkv": (3 * d,), "w_o": (d, d), "b_o": (d,),
               "w_fc1": (f, d), "b_fc1": (f,), "w_fc2": (d, f), "b_fc2": (d,),
               "w_ada": (6 * d, c), "b_ada": (6 * d,)}
-    return {name: _param(shapes[name], cfg.seed, block, i, device)
-            for i, name in enumerate(BLOCK_TENSORS)}
+    out = {name: _param(shapes[name], cfg.seed, block, i, device)
+           for i, name in enumerate(BLOCK_TENSORS) if name in shapes}
+    if cfg.qk_norm:
+        for name in ("q_norm", "k_norm"):
+            i = BLOCK_TENSORS.index(name)
+            z = _randn((cfg.head_dim,), _seed(cfg.seed, block, i), device)
+            out[name] = (1.0 + QK_GAIN_STD * z).to(torch.bfloat16).float()
+    return out
 
 
 def final_params(cfg: DiTConfig, device="cpu") -> Dict[str, torch.Tensor]:
@@ -150,6 +177,21 @@ def final_params(cfg: DiTConfig, device="cpu") -> Dict[str, torch.Tensor]:
     d, c = cfg.d, cfg.c_dim
     return {"w_fin": _param((2, 2 * d, c), cfg.seed, -1, 0, device),
             "b_fin": _param((2, 2 * d), cfg.seed, -1, 1, device)}
+
+
+def head_params(cfg: DiTConfig, device="cpu") -> Dict[str, torch.Tensor]:
+    """Patch embedding and final heads of a latent workload, one per stream (video, audio):
+    w_patch [2, d, C], b_patch [2, d], w_head [2, C, d], b_head [2, C], bf16 N(0, 0.02)."""
+    d, C = cfg.d, cfg.latent_channels
+    shapes = {"w_patch": (2, d, C), "b_patch": (2, d), "w_head": (2, C, d), "b_head": (2, C)}
+    return {name: _param(shapes[name], cfg.seed, -2, i, device)
+            for i, name in enumerate(_HEAD_TENSORS)}
+
+
+def latent_state(cfg: DiTConfig, device="cpu") -> torch.Tensor:
+    """Initial latent [N, C] ~ N(0, 1) as fp32 holding bf16-representable values."""
+    x = _randn((cfg.n_tokens, cfg.latent_channels), _seed(cfg.seed, -2, _NOISE_IDX), device)
+    return x.to(torch.bfloat16).float()
 
 
 def conditioning(cfg: DiTConfig, device="cpu") -> torch.Tensor:
