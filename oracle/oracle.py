@@ -576,3 +576,76 @@ def denoise_latent(lat0, blocks, mods, final_mod, heads, grid, n_audio: int, n_h
         v = final_head(x_l, final_mod, nv, eps, heads["w_head"], heads["b_head"], dt)
         lat = euler_update(lat, v, sig[i], sig[i + 1], dt)
     return lat
+
+
+# --------------------------------------------------------------------------------------
+# f3: grouped int8 MLP and int8 QKV
+# --------------------------------------------------------------------------------------
+def quantize_groups(a, group: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Symmetric int8 quantisation with one fp32 scale per row and per `group` consecutive
+    columns ([dothoosh] "The powerful int8 path": the FC2 input has one scale per 1024
+    channels).  Each (row, group) follows quantize_rows' rule.  Returns q [M, K] int8 and
+    scales [M, K / group] fp32."""
+    a = np.asarray(a, np.float32)
+    m, k = a.shape
+    assert k % group == 0
+    g = a.reshape(m * (k // group), group)
+    q, s = quantize_rows(g)
+    return q.reshape(m, k), s.reshape(m, k // group)
+
+
+def int8_grouped_matmul(q, s_a, w_q, w_scale, group: int, dt=F64) -> np.ndarray:
+    """y[m, n] = w_scale[n] sum_g s_a[m, g] acc_g[m, n] with the exact integer group sums
+    acc_g = sum over the group's k of q[m, k] w_q[n, k]."""
+    m, k = q.shape
+    y = np.zeros((m, w_q.shape[0]), dt)
+    for gi in range(k // group):
+        sl = slice(gi * group, (gi + 1) * group)
+        acc = int_matmul(q[:, sl], w_q[:, sl]).astype(dt)
+        y += np.asarray(s_a[:, gi], dt)[:, None] * acc
+    return y * np.asarray(w_scale, dt)[None, :]
+
+
+def int8_linear_rows(a, w_q, w_scale, bias=None, dt=F64) -> np.ndarray:
+    """Linear layer on int8 operands with one scale per activation row and per weight
+    output channel: y = (q_a w_q^T) s_a s_w (+ b), q_a, s_a = quantize_rows(a)."""
+    q, s = quantize_rows(a)
+    y = int_matmul(q, w_q).astype(dt) * np.asarray(s, dt)[:, None] * np.asarray(w_scale, dt)[None, :]
+    if bias is not None:
+        y = y + np.asarray(bias, dt)[None, :]
+    return y
+
+
+def block_forward_int8(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int, split,
+                       theta: float, eps: float, group: int = 1024, rows=None,
+                       dt=F64) -> np.ndarray:
+    """block_forward with the int8 path of [dothoosh] "The powerful int8 path": the QKV and
+    FC1 inputs (the AdaLN outputs) quantised per token row, the FC2 input (the GELU
+    output) per token and per `group` channels, weights per output channel
+    (w["w_qkv_q"], w["s_qkv"], ...: quantize_rows of the bf16 weights); the attention and
+    the output projection stay bf16.  The quantisation acts on fp32 values of the
+    activations (the GPU quantises its fp32 epilogue values)."""
+    x = np.asarray(x, dt)
+    mod = np.asarray(mod, dt)
+    n, d = x.shape
+    hd = d // n_heads
+    sel = np.arange(n) if rows is None else np.asarray(rows)
+    h = modulate(layer_norm(x, eps, dt), mod[0], mod[1], dt)
+    qkv = int8_linear_rows(h.astype(np.float32), w["w_qkv_q"], w["s_qkv"],
+                           np.asarray(w["b_qkv"], dt), dt)
+    q = qkv[sel, :d].reshape(len(sel), n_heads, hd)
+    k = qkv[:, d:2 * d].reshape(n, n_heads, hd)
+    v = qkv[:, 2 * d:].reshape(n, n_heads, hd)
+    if w.get("q_norm") is not None:
+        q = rms_norm(q, w["q_norm"], eps, dt)
+        k = rms_norm(k, w["k_norm"], eps, dt)
+    k = rope_rotate(k, pos, split, theta, dt)
+    q = rope_rotate(q, np.asarray(pos)[sel], split, theta, dt)
+    o = attention(q, k, v, dt=dt).reshape(len(sel), d)
+    x1 = gated_residual(x[sel], mod[2], o @ np.asarray(w["w_o"], dt).T + np.asarray(w["b_o"], dt), dt)
+    h2 = modulate(layer_norm(x1, eps, dt), mod[3], mod[4], dt)
+    g = gelu_tanh(int8_linear_rows(h2.astype(np.float32), w["w_fc1_q"], w["s_fc1"],
+                                   np.asarray(w["b_fc1"], dt), dt), dt)
+    qg, sg = quantize_groups(g.astype(np.float32), group)
+    y = int8_grouped_matmul(qg, sg, w["w_fc2_q"], w["s_fc2"], group, dt) + np.asarray(w["b_fc2"], dt)
+    return gated_residual(x1, mod[5], y, dt)

@@ -801,3 +801,49 @@ def test_latent_loop_constant_head_closed_form():
     want[:nv] += -0.75 * vv
     want[nv:] += -0.75 * va
     assert np.allclose(got, want, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- grouped int8
+def test_quantize_groups_is_rows_per_group():
+    a = (RNG.standard_normal((5, 12)) * [1, 1, 1, 1, 10, 10, 10, 10, 0, 0, 0, 0]).astype(np.float32)
+    q, s = O.quantize_groups(a, 4)
+    assert q.shape == (5, 12) and s.shape == (5, 3)
+    for g in range(3):
+        qg, sg = O.quantize_rows(a[:, 4 * g:4 * g + 4])
+        assert np.array_equal(q[:, 4 * g:4 * g + 4], qg) and np.array_equal(s[:, g], sg)
+    assert np.all(s[:, 2] == 0) and np.all(q[:, 8:] == 0)         # a zero group
+    assert np.all(np.max(np.abs(q[:, :8].astype(int).reshape(5, 2, 4)), axis=2) == 127)
+
+
+def test_int8_grouped_matmul_bruteforce_and_single_group():
+    qa = RNG.integers(-127, 128, (3, 8)).astype(np.int8)
+    wq = RNG.integers(-127, 128, (2, 8)).astype(np.int8)
+    sa = RNG.uniform(0.01, 0.1, (3, 2)).astype(np.float32)
+    sw = RNG.uniform(0.001, 0.01, 2).astype(np.float32)
+    y = O.int8_grouped_matmul(qa, sa, wq, sw, 4)
+    for m in range(3):
+        for n in range(2):
+            ref = sum(float(sa[m, k // 4]) * int(qa[m, k]) * int(wq[n, k]) for k in range(8))
+            assert abs(y[m, n] - ref * float(sw[n])) < 1e-12
+    # one group spanning K is the row-scaled product
+    y1 = O.int8_grouped_matmul(qa, sa[:, :1], wq, sw, 8)
+    ref = O.int_matmul(qa, wq) * sa[:, :1].astype(float) * sw[None, :].astype(float)
+    assert np.allclose(y1, ref, atol=1e-14)
+
+
+def test_int8_block_close_to_bf16_block_and_exact_parts():
+    w, mod = _tiny_block(seed=51)
+    for name in ("qkv", "fc1", "fc2"):
+        w[f"w_{name}_q"], w[f"s_{name}"] = O.quantize_rows(w[f"w_{name}"].astype(np.float32))
+    grid = (2, 2, 4)
+    x = RNG.standard_normal((16 + 3, 64))
+    pos = O.rope_positions(grid, 3)
+    ref, _ = O.block_forward(x, w, mod, pos, 2, (8, 12, 12), 1e4, 1e-6)
+    got = O.block_forward_int8(x, w, mod, pos, 2, (8, 12, 12), 1e4, 1e-6, group=64)
+    # quantisation noise only: the int8 update stays close to the float update
+    assert rel_l2(got - x, ref - x) < 3e-2
+    # zero gates: identity, as in the float block
+    mz = mod.copy()
+    mz[2] = 0
+    mz[5] = 0
+    assert np.array_equal(O.block_forward_int8(x, w, mz, pos, 2, (8, 12, 12), 1e4, 1e-6, 64), x)
