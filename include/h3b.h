@@ -450,6 +450,58 @@ int h3b_fc2_int8_row(const h3b_bf16* act, int M, int K, int n_out, const int8_t*
                      h3b_bf16* resid, int8_t* act_q, float* row_scale, int32_t* acc_out,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- int8 block path */
+/* Weights of one block on the int8 path (dothoosh.com, "The powerful int8 path": int8
+ * MLP with dynamic activation quantisation and per-output-channel weight scales, the FC2
+ * input with one scale per 1024 channels, quantised QKV).  Weights [out, in] int8 from
+ * h3b_quantize_rows of the bf16 weights, with their per-output-channel scales [out] fp32.
+ * The biases, the output projection and the Q/K norm gains come from h3b_block_weights. */
+typedef struct h3b_int8_block {
+  const int8_t* w_qkv_q;   /* [3d, d] */
+  const float* s_qkv;      /* [3d] */
+  const int8_t* w_fc1_q;   /* [d_ff, d] */
+  const float* s_fc1;      /* [d_ff] */
+  const int8_t* w_fc2_q;   /* [d, d_ff] */
+  const float* s_fc2;      /* [d] */
+} h3b_int8_block;
+
+/* Bytes of workspace h3b_block_forward_int8 needs (0 on bad arguments; d_ff % 1024). */
+size_t h3b_workspace_size_int8(const h3b_dims* dims, int n_tokens);
+
+/* One DiT block on the int8 path:
+ *   hq, hs = quantise_rows(LN(x)(1 + scale_msa) + shift_msa)      (one fused kernel)
+ *   qkv    = rope(rmsnorm?((hq w_qkv_q^T) hs s_qkv + b_qkv))          (int8 GEMM epilogue)
+ *   o      = attention (bf16);  x = x + gate_msa (o W_o^T + b_o)  (bf16)
+ *   hq, hs = quantise_rows(LN(x)(1 + scale_mlp) + shift_mlp)
+ *   g      = GELU((hq w_fc1_q^T) hs s_fc1 + b_fc1)                   (bf16)
+ *   gq, gs = quantise_groups(g), one scale per row and 1024 channels
+ *   x      = x + gate_mlp (s_fc2 sum_groups gs acc_group + b_fc2)   (grouped int8 GEMM)
+ * Quantisation: the rule of h3b_quantize_rows.  mod [6, d] fp32; x [n_tokens, d] bf16
+ * in/out; ws: h3b_workspace_size_int8 bytes.  All device.  d_ff % 1024 == 0. */
+int h3b_block_forward_int8(const h3b_dims* dims, const h3b_block_weights* w,
+                           const h3b_int8_block* wq, const float* mod, const float* rope_cs,
+                           int n_tokens, h3b_bf16* x, void* ws, size_t ws_bytes, void* stream);
+
+/* h = LN(x)(1 + scale) + shift (fp32) quantised per row: q [n_tokens, d] int8,
+ * q_scale [n_tokens] fp32 (the rule of h3b_quantize_rows); x bf16.  All device. */
+int h3b_ln_modulate_q8(const h3b_bf16* x, int n_tokens, int d, float eps, const float* shift,
+                       const float* scale, int8_t* q, float* q_scale, void* stream);
+
+/* The rule of h3b_quantize_rows applied to every 1024-column group of every row:
+ * a [rows, cols] bf16, q [rows, cols] int8, scale [rows, cols / 1024] fp32; cols % 1024
+ * == 0.  All device. */
+int h3b_quantize_groups(const h3b_bf16* a, int rows, int cols, int8_t* q, float* scale,
+                        void* stream);
+
+/* The grouped int8 FC2 with gated residual:
+ *   resid = bf16(resid + gate (w_scale[n] sum_g a_scale[m, g] acc_g[m, n] + bias[n])),
+ *   acc_g = the exact int32 product of group g (1024 K columns) of A [M, K] and w_q [N, K].
+ * a_scale [M, K / 1024], w_scale, gate [N] fp32; bias [N] bf16 or NULL; resid [M, N]
+ * bf16 in/out.  All device.  K % 1024 == 0, N % 128 == 0. */
+int h3b_gemm_i8_grouped(const int8_t* A, const float* a_scale, int M, int K, int N,
+                        const int8_t* w_q, const float* w_scale, const h3b_bf16* bias,
+                        const float* gate, h3b_bf16* resid, void* stream);
+
 /* ---------------------------------------------------------------- single kernels */
 /* The projection GEMM used by the block: out = A B^T with an epilogue.
  * A [M, K] bf16, B [N, K] bf16 (device), K % 64 == 0, N % 128 == 0.

@@ -185,9 +185,11 @@ __device__ __forceinline__ void load_f32x32(const float* src, float (&v)[32]) {
   }
 }
 
-// Row statistics an LN-folded epilogue applies to its row: mean and 1 / sqrt(var + eps).
+// Per-row scalars of an epilogue row: for the LN-folded kinds the mean and
+// 1 / sqrt(var + eps); for the int8 kinds the activation row scale rs.
 struct LnRow {
   float mu, rstd;
+  float rs = 0.f;
 };
 
 // Merge a row's group statistics (mean, M2 of each 256-column group, in group order) into
@@ -244,7 +246,7 @@ struct RowIn {
 
 template <int EPI>
 __device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int col, RowIn& in) {
-  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+  if constexpr (epi_gated(EPI)) {
     const uint4* s = reinterpret_cast<const uint4*>(e.out + size_t(row) * e.ld_out + col);
 #pragma unroll
     for (int i = 0; i < 4; ++i) in.res[i] = s[i];  // coherent: this kernel rewrites it
@@ -283,7 +285,18 @@ __device__ __forceinline__ void qk_rms_pass_global(const GemmEpilogue& e, uint32
     tmem_wait_ld(r);
     float v[32];
     const int col = col0 + c * 32;
-    if constexpr (epi_ln_fold(EPI)) {
+    if constexpr (epi_int8(EPI)) {
+      float cs[32], b[32];
+      load_f32x32(e.col_scale + col, cs);
+      if (e.bias_f32)
+        load_f32x32(e.bias_f32 + col, b);
+      else
+        load_bf16x32(e.bias + col, b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), ln.rs), cs[j]) +
+               b[j];
+    } else if constexpr (epi_ln_fold(EPI)) {
       float cv[32], dv[32];
       load_f32x32(e.fold_c + col, cv);
       load_f32x32(e.bias_f32 + col, dv);
@@ -317,7 +330,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
                                                const LnRow& ln, StatAcc* sa, bool first,
                                                float qk_s = 1.0f) {
   float v[32];
-  if constexpr (EPI == kEpiInt8Deq) {
+  if constexpr (epi_int8(EPI)) {
     const float rs = __ldg(e.row_scale + row);
     float cs[32];
     load_f32x32(e.col_scale + col, cs);
@@ -331,9 +344,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), rs), cs[j]);
-    if (e.bias_f32) {
+    if (e.bias_f32 || e.bias) {
       float b[32];
-      load_f32x32(e.bias_f32 + col, b);
+      if (e.bias_f32)
+        load_f32x32(e.bias_f32 + col, b);
+      else
+        load_bf16x32(e.bias + col, b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += b[j];
     }
@@ -388,7 +404,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
     }
   }
   bf16* dst = e.out + size_t(row) * e.ld_out + col;
-  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+  if constexpr (epi_gated(EPI)) {
     float g[32];
     load_f32x32(e.gate + col, g);
 #pragma unroll
@@ -471,8 +487,9 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
   StatAcc sa{0.f, 0.f, 0.f};
   const bool want_stats =
       (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
+  if constexpr (epi_int8(EPI)) ln.rs = valid ? __ldg(p.epi.row_scale + row) : 0.f;
   float qks[4] = {1.f, 1.f, 1.f, 1.f};
-  if constexpr (epi_base(EPI) == kEpiRope && !INT8) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
       qk_rms_pass_global<BN, EPI>(p.epi, tbase, col0, ln, qks);
   }
@@ -542,8 +559,14 @@ __device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, f
   for (int k = 0; k < NV / 32; ++k) {
     const int i = k * 32 + lane;
     const int col = col0 + i;
-    if constexpr (EPI == kEpiInt8Deq) {
-      vec[kVecBias + i] = e.bias_f32 ? __ldg(e.bias_f32 + col) : 0.0f;
+    if constexpr (epi_int8(EPI) || EPI == kEpiI8GroupGate) {
+      float bv = 0.0f;
+      if (e.bias_f32)
+        bv = __ldg(e.bias_f32 + col);
+      else if (e.bias)
+        bv = __uint_as_float(static_cast<uint32_t>(
+                 __ldg(reinterpret_cast<const unsigned short*>(e.bias) + col)) << 16);
+      vec[kVecBias + i] = bv;
       vec[kVecScale + i] = __ldg(e.col_scale + col);
     } else if constexpr (epi_ln_fold(EPI)) {
       vec[kVecBias + i] = __ldg(e.bias_f32 + col);   // dv
@@ -552,7 +575,7 @@ __device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, f
       const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(e.bias) + col);
       vec[kVecBias + i] = __uint_as_float(b << 16);
     }
-    if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq)
+    if constexpr (epi_gated(EPI))
       vec[kVecGate + i] = __ldg(e.gate + col);
     if constexpr (epi_base(EPI) == kEpiRope) {
       // Q/K RMSNorm gains of the column's head dimension (1 outside q and k, or when off)
@@ -570,7 +593,7 @@ __device__ __forceinline__ void stage_vectors(const GemmEpilogue& e, int col0, f
 template <int EPI>
 __device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, int nrows,
                                               int col, int lane, RowIn& in) {
-  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+  if constexpr (epi_gated(EPI)) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int r = k * 8 + (lane >> 2);
@@ -600,7 +623,13 @@ __device__ __forceinline__ void load_block_in(const GemmEpilogue& e, int row0, i
 template <int EPI>
 __device__ __forceinline__ void pre_values(const uint32_t (&r)[32], const float* vec,
                                            const LnRow& ln, float (&v)[32]) {
-  if constexpr (epi_ln_fold(EPI)) {
+  if constexpr (epi_int8(EPI)) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), ln.rs),
+                       vec[kVecScale + j]) +
+             vec[kVecBias + j];
+  } else if constexpr (epi_ln_fold(EPI)) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       v[j] = fmaf(ln.rstd, fmaf(-ln.mu, vec[kVecScale + j], __uint_as_float(r[j])),
@@ -651,7 +680,11 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
                                                bool first, float qk_s = 1.0f) {
   const bool valid = lane < nrows;
   float v[32];
-  if constexpr (EPI == kEpiInt8Deq) {
+  if constexpr (EPI == kEpiI8GroupGate) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      v[j] = __fmul_rn(__uint_as_float(r[j]), vec[kVecScale + j]) + vec[kVecBias + j];
+  } else if constexpr (epi_int8(EPI)) {
     const float rs = valid ? __ldg(e.row_scale + row0 + lane) : 0.0f;
     if (e.acc_out && valid) {
       int4* dst = reinterpret_cast<int4*>(e.acc_out + size_t(row0 + lane) * e.ld_out + col);
@@ -730,7 +763,7 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
       }
     }
   }
-  if constexpr (EPI == kEpiGateResid || EPI == kEpiInt8Deq) {
+  if constexpr (epi_gated(EPI)) {
     __syncwarp();
 #pragma unroll
     for (int k = 0; k < 4; ++k) blk[blk16(k * 8 + (lane >> 2), lane & 3)] = in.res[k];
@@ -790,8 +823,9 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
   StatAcc sa{0.f, 0.f, 0.f};
   const bool want_stats =
       (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
+  if constexpr (epi_int8(EPI)) ln.rs = lane < nrows ? __ldg(p.epi.row_scale + row0 + lane) : 0.f;
   float qks[4] = {1.f, 1.f, 1.f, 1.f};
-  if constexpr (epi_base(EPI) == kEpiRope && !INT8) {
+  if constexpr (epi_base(EPI) == kEpiRope) {
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
       qk_rms_pass<BN, EPI>(p.epi, tbase, vec, ln, qks);
   }
@@ -1337,6 +1371,241 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Grouped int8 pair GEMM: the A operand carries one scale per row and per group of 1024 K
+// columns (the int8 MLP's FC2 input), so the group products cannot share one integer
+// accumulator.  Pair tiles of 256 x 128, data-parallel.  TMEM (per CTA, 128 lanes): two
+// int32 group accumulators (columns 0-127 and 128-255) and the fp32 running sum (256-383).
+// The MMA issuer fills accumulator g & 1 with group g's products (the accumulation
+// restarts at each group) and signals gfull; the epilogue warps fold it into the sum,
+// sum += float(acc_g) * s_a[row, g], and hand the accumulator back (gempty), so the fold
+// of group g overlaps the products of group g + 1.  After a tile's last group the same
+// warps run the staged epilogue on the sum.
+constexpr int kGroupK = 1024;
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_gemm_pair_grouped(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int BN = 128;
+  using Cfg = PairCfg<BN>;
+  constexpr int STAGES = Cfg::kStages;
+  constexpr uint32_t HA = Cfg::kABytes;
+  constexpr uint32_t HB = Cfg::kBBytes;
+  constexpr uint32_t IDESC = idesc_s8(256, BN);
+  constexpr int K_STEPS = kTileBytesK / 32;
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kSumCol = 256;
+  constexpr int KB_PER_GROUP = kGroupK / 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * HA;
+  uint8_t* sEpi = sB + STAGES * HB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB + Cfg::kStageOut);
+  uint64_t* empty = full + STAGES;
+  uint64_t* gfull = empty + STAGES;
+  uint64_t* gempty = gfull + 2;
+  uint64_t* drain = gempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int groups = p.k_blocks / KB_PER_GROUP;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&gfull[b], 1);
+      mbar_init(&gempty[b], 8);  // four epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+  const uint32_t gempty0 = mapa_shared(smem_u32(gempty), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer (both)
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[STAGES];
+#pragma unroll
+      for (int st = 0; st < STAGES; ++st) armed[st] = -1;
+      bool ok = true;
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        int mb, nb;
+        tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrGemmWait)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (HA + HB));
+          const uint32_t fb = full0 + stage * 8;
+          tma_load_2d_pair(sA + stage * HA, &tmA, fb, kb * 128, mb * 256 + rank * 128);
+          tma_load_2d_pair(sB + stage * HB, &tmB, fb, kb * 128,
+                           nb * BN + static_cast<int>(rank) * (BN / 2));
+          armed[stage] = static_cast<int>(phase);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int st = 0; st < STAGES; ++st)
+          if (armed[st] >= 0) drain_wait(&full[st], static_cast<uint32_t>(armed[st]));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------------- MMA issuer (even CTA)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int gi = 0;  // groups issued by this pair so far
+      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+        for (int g = 0; g < groups && ok; ++g, ++gi) {
+          const int buf = gi & 1;
+          const uint32_t use = static_cast<uint32_t>(gi >> 1);
+          if (!wait_bar(&gempty[buf], (use & 1u) ^ 1u, abort_flag, p.err, kErrGemmWait)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+          for (int kb = 0; kb < KB_PER_GROUP; ++kb) {
+            if (!wait_bar(&full[stage], phase, abort_flag, p.err, kErrGemmWait)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + stage * HA);
+            const uint32_t b0 = smem_u32(sB + stage * HB);
+#pragma unroll
+            for (int k = 0; k < K_STEPS; ++k)
+              umma_i8_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
+                           sdesc_sw128(b0 + k * 32, 16, 1024), IDESC,
+                           (kb > 0 || k > 0) ? 1u : 0u);
+            tc_commit_pair_mc(&empty[stage], 0x3);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (ok) tc_commit_pair_mc(&gfull[buf], 0x3);
+        }
+      }
+      tc_commit_pair(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ fold + epilogue
+    const int quarter = warp & 3;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint4* blk = reinterpret_cast<uint4*>(sEpi + quarter * kWarpStage);
+    float* vec = reinterpret_cast<float*>(sEpi + quarter * kWarpStage + 4096);
+    int gi = 0;
+    bool ok = true;
+    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+      int mb, nb;
+      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      stage_vectors<EPI, BN>(p.epi, nb * BN, vec, lane);
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int row = row0 + lane;
+      const uint32_t sum_addr = tmem_base + lane_addr + kSumCol;
+      for (int g = 0; g < groups; ++g, ++gi) {
+        const int buf = gi & 1;
+        const uint32_t use = static_cast<uint32_t>(gi >> 1);
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(&gfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait));
+        if (!ok) break;
+        tc_fence_after();
+        const float sa = row < p.M ? __ldg(p.epi.row_scale + size_t(row) * groups + g) : 0.f;
+        const uint32_t acc_addr = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(acc_addr + c * 32, a);
+          tmem_wait_ld(a);
+          uint32_t sm[32];
+          if (g > 0) {
+            tmem_ld32(sum_addr + c * 32, sm);
+            tmem_wait_ld(sm);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              sm[j] = __float_as_uint(fmaf(static_cast<float>(static_cast<int32_t>(a[j])), sa,
+                                           __uint_as_float(sm[j])));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              sm[j] = __float_as_uint(__fmul_rn(static_cast<float>(static_cast<int32_t>(a[j])), sa));
+          }
+          tmem_st32(sum_addr + c * 32, sm);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {  // the group accumulator may be refilled
+          if (rank == 0)
+            mbar_arrive(&gempty[buf]);
+          else
+            mbar_arrive_cluster(gempty0 + buf * 8);
+        }
+      }
+      if (!ok) break;
+      __syncwarp();  // staged vectors visible to every lane
+      const int nrows = p.M - row0;
+      RowIn in[2];
+      load_block_in<EPI>(p.epi, row0, nrows, nb * BN, lane, in[0]);
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(sum_addr + c * 32, r);
+        if (c + 1 < BN / 32) load_block_in<EPI>(p.epi, row0, nrows, nb * BN + (c + 1) * 32, lane, in[(c + 1) & 1]);
+        tmem_wait_ld(r);
+        epilogue_block<EPI>(p.epi, row0, nrows, nb * BN + c * 32, r, in[c & 1], blk, vec + c * 32,
+                            lane, LnRow{0.f, 1.f}, nullptr, false);
+      }
+      tc_fence_before();
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 std::atomic<unsigned long long> g_sk_seq{0};
 bool trace_gemm();
 int forced_sched();
@@ -1788,28 +2057,91 @@ int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int
   return dispatch_bf16<128>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
 }
 
-int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
+template <int EPI>
+int launch_i8_kind(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
                    const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                    cudaStream_t stream) {
-  if (M <= 0) return 0;
   const int tile = choose_tile(M, N);
   if (tile == kPair256 || tile == kPair128) {
     int rc = 0;
     const int r = tile == kPair256
-                      ? launch_pair<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch,
-                                                            scratch_bytes, stream, &rc)
-                      : launch_pair<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch,
-                                                            scratch_bytes, stream, &rc);
+                      ? launch_pair<256, true, EPI>(ctx, A, B, M, N, K, epi, scratch,
+                                                    scratch_bytes, stream, &rc)
+                      : launch_pair<128, true, EPI>(ctx, A, B, M, N, K, epi, scratch,
+                                                    scratch_bytes, stream, &rc);
     if (r == 0) return rc;
   }
   if (tile == kSingle128 || N % 256 != 0)
-    return launch_impl<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
-                                               stream);
-  if (N % 256 == 0)
-    return launch_impl<256, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
-                                               stream);
-  return launch_impl<128, true, kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes,
-                                             stream);
+    return launch_impl<128, true, EPI>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+  return launch_impl<256, true, EPI>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+}
+
+int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
+                   const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                   cudaStream_t stream) {
+  if (M <= 0) return 0;
+  switch (epi.kind) {
+    case kEpiInt8Deq:
+      return launch_i8_kind<kEpiInt8Deq>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+    case kEpiI8Rope:
+      return launch_i8_kind<kEpiI8Rope>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+    case kEpiI8Gelu:
+      return launch_i8_kind<kEpiI8Gelu>(ctx, A, B, M, N, K, epi, scratch, scratch_bytes, stream);
+    default: return set_error(-1, "gemm_i8: unknown epilogue %d", epi.kind);
+  }
+}
+
+int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N,
+                           int K, const GemmEpilogue& epi, cudaStream_t stream) {
+  if (M <= 0) return 0;
+  if (epi.kind != kEpiI8GroupGate || K % kGroupK || N % 128)
+    return set_error(-1, "gemm_i8_grouped: K=%d must be a multiple of %d, N=%d of 128", K, kGroupK, N);
+  using Cfg = PairCfg<128>;
+  auto kernel = k_gemm_pair_grouped<kEpiI8GroupGate>;
+  static std::atomic<uint32_t> attr_done{0};
+  const uint32_t bit = 1u << (ctx.device & 31);
+  if (!(attr_done.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Cfg::kSmem));
+    if (e != cudaSuccess)
+      return set_error(-3, "gemm_i8_grouped: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_done.fetch_or(bit);
+  }
+  static std::atomic<int> cap_cache[64];
+  int cap = cap_cache[ctx.device & 63].load();
+  if (cap <= 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (ctx.num_sms / 2));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = Cfg::kSmem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return set_error(-3, "gemm_i8_grouped: no resident CTA pair");
+    }
+    cap = std::min(n, ctx.num_sms / 2);
+    cap_cache[ctx.device & 63].store(cap);
+  }
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(M), uint64_t(K), uint64_t(K),
+                    128, 128) ||
+      !make_tmap_2d(&tb, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, uint64_t(N), uint64_t(K), uint64_t(K),
+                    64, 128))
+    return set_error(-3, "gemm_i8_grouped: cuTensorMapEncodeTiled failed (M=%d N=%d K=%d)", M, N, K);
+  GemmParams p{};
+  p.M = M;
+  p.N = N;
+  p.k_blocks = K / 128;
+  p.m_tiles = (M + 255) / 256;
+  p.n_tiles = N / 128;
+  p.epi = epi;
+  p.err = ctx.err_flag;
+  const int tiles = p.m_tiles * p.n_tiles;
+  if (trace_gemm())
+    std::fprintf(stderr, "h3b gemm i8 grouped M=%d N=%d K=%d tiles=%d cap=%d\n", M, N, K, tiles,
+                 cap);
+  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  return check_launch("gemm_i8_grouped");
 }
 
 }  // namespace h3b

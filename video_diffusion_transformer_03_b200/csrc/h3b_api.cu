@@ -313,6 +313,100 @@ int block_forward_folded_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_bl
                           b.gemm_scratch, gemm_scratch_bytes(), s);
 }
 
+// Buffers of the int8 block after the shared arena: the quantised AdaLN output [n, d] and
+// its row scales [n], the quantised GELU output [n, d_ff] and its group scales
+// [n, d_ff / 1024].
+struct Int8Bufs {
+  int8_t* hq;
+  float* hs;
+  int8_t* gq;
+  float* gs;
+  size_t total;
+};
+
+Int8Bufs carve_int8(const h3b_dims* d, int n, void* base) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  Int8Bufs b{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* q = p ? p + off : nullptr;
+    off += a256(bytes);
+    return q;
+  };
+  b.hq = reinterpret_cast<int8_t*>(take(size_t(n) * d->d));
+  b.hs = reinterpret_cast<float*>(take(size_t(n) * 4));
+  b.gq = reinterpret_cast<int8_t*>(take(size_t(n) * d->d_ff));
+  b.gs = reinterpret_cast<float*>(take(size_t(n) * (d->d_ff / 1024) * 4));
+  b.total = off;
+  return b;
+}
+
+// The block on the int8 path (dothoosh.com, "The powerful int8 path"): the AdaLN outputs
+// quantised per row inside the LayerNorm kernel, int8 QKV and FC1 with per-row and
+// per-output-channel scales (RoPE / GELU in their epilogues), the GELU output quantised
+// per 1024-channel group, and the grouped int8 FC2 with the gated residual; attention and
+// the output projection stay bf16.
+int block_forward_int8_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_block_weights* w,
+                            const h3b_int8_block* q, const float* mod, const float* rope_cs,
+                            int n, bf16* x, void* arena, cudaStream_t s) {
+  const int D = d->d;
+  const BlockBufs b = carve_block(d, n, arena);
+  const Int8Bufs ib = carve_int8(d, n, static_cast<uint8_t*>(arena) + arena_bytes(d, n));
+  int rc;
+  if ((rc = launch_ln_modulate_q8(x, n, D, d->ln_eps, mod, mod + D, ib.hq, ib.hs, s))) return rc;
+  GemmEpilogue e;
+  e.kind = kEpiI8Rope;
+  e.bias = reinterpret_cast<const bf16*>(w->b_qkv);
+  e.row_scale = ib.hs;
+  e.col_scale = q->s_qkv;
+  e.q_gain = w->q_norm;
+  e.k_gain = w->k_norm;
+  e.ln_eps = d->ln_eps;
+  e.rope_cs = rope_cs;
+  e.rope_cols = 2 * D;
+  e.head_dim = d->head_dim;
+  e.out = b.qkv;
+  e.ld_out = 3 * D;
+  if ((rc = launch_gemm_i8(ctx, ib.hq, q->w_qkv_q, n, 3 * D, D, e, b.gemm_scratch,
+                           gemm_scratch_bytes(), s)))
+    return rc;
+  if ((rc = launch_attention(ctx, b.qkv, n, d->n_heads, d->head_dim, b.attn, b.gemm_scratch,
+                             gemm_scratch_bytes(), s)))
+    return rc;
+  e = GemmEpilogue();
+  e.kind = kEpiGateResid;
+  e.bias = reinterpret_cast<const bf16*>(w->b_o);
+  e.gate = mod + 2 * D;
+  e.out = x;
+  e.ld_out = D;
+  if ((rc = launch_gemm_bf16(ctx, b.attn, reinterpret_cast<const bf16*>(w->w_o), n, D, D, e,
+                             b.gemm_scratch, gemm_scratch_bytes(), s)))
+    return rc;
+  if ((rc = launch_ln_modulate_q8(x, n, D, d->ln_eps, mod + 3 * D, mod + 4 * D, ib.hq, ib.hs, s)))
+    return rc;
+  e = GemmEpilogue();
+  e.kind = kEpiI8Gelu;
+  e.bias = reinterpret_cast<const bf16*>(w->b_fc1);
+  e.row_scale = ib.hs;
+  e.col_scale = q->s_fc1;
+  e.out = b.g;
+  e.ld_out = d->d_ff;
+  if ((rc = launch_gemm_i8(ctx, ib.hq, q->w_fc1_q, n, d->d_ff, D, e, b.gemm_scratch,
+                           gemm_scratch_bytes(), s)))
+    return rc;
+  if ((rc = launch_quantize_groups(b.g, n, d->d_ff, ib.gq, ib.gs, s))) return rc;
+  e = GemmEpilogue();
+  e.kind = kEpiI8GroupGate;
+  e.bias = reinterpret_cast<const bf16*>(w->b_fc2);
+  e.row_scale = ib.gs;
+  e.act_groups = d->d_ff / 1024;
+  e.col_scale = q->s_fc2;
+  e.gate = mod + 5 * D;
+  e.out = x;
+  e.ld_out = D;
+  return launch_gemm_i8_grouped(ctx, ib.gq, q->w_fc2_q, n, D, d->d_ff, e, s);
+}
+
 // Workspace of one denoise step.
 struct StepBufs {
   bf16* x_res;      // [N, d] residual stream (bf16)
@@ -721,6 +815,83 @@ int h3b_block_forward_folded(const h3b_dims* dims, const h3b_block_weights* w, c
   return block_forward_folded_impl(ctx, dims, w, mod, rope_cs, n_tokens, reinterpret_cast<bf16*>(x),
                                    reinterpret_cast<float2*>(stats), ws,
                                    static_cast<cudaStream_t>(stream));
+}
+
+size_t h3b_workspace_size_int8(const h3b_dims* dims, int n_tokens) {
+  if (check_dims(dims) || n_tokens < 0 || dims->d_ff % 1024) return 0;
+  return arena_bytes(dims, n_tokens) + carve_int8(dims, n_tokens, nullptr).total;
+}
+
+int h3b_block_forward_int8(const h3b_dims* dims, const h3b_block_weights* w,
+                           const h3b_int8_block* wq, const float* mod, const float* rope_cs,
+                           int n_tokens, h3b_bf16* x, void* ws, size_t ws_bytes, void* stream) {
+  int rc;
+  if ((rc = check_dims(dims)) || (rc = check_weights(w))) return rc;
+  if (dims->d_ff % 1024)
+    return set_error(H3B_EINVAL, "block_forward_int8: d_ff=%d must be a multiple of 1024", dims->d_ff);
+  if (n_tokens < 0 || n_tokens > (1 << 24)) return set_error(H3B_EINVAL, "n_tokens=%d", n_tokens);
+  if (!wq) return set_error(H3B_EINVAL, "block_forward_int8: int8 weights NULL");
+  const void* ptrs[6] = {wq->w_qkv_q, wq->s_qkv, wq->w_fc1_q, wq->s_fc1, wq->w_fc2_q, wq->s_fc2};
+  for (const void* p : ptrs)
+    if (!p || !al16(p)) return set_error(H3B_EINVAL, "block_forward_int8: int8 weight NULL or misaligned");
+  if (!mod || !rope_cs || !x || !al16(mod) || !al16(rope_cs) || !al16(x))
+    return set_error(H3B_EINVAL, "block_forward_int8: NULL or misaligned pointer");
+  const size_t need = arena_bytes(dims, n_tokens) + carve_int8(dims, n_tokens, nullptr).total;
+  if (!ws || !al16(ws) || ws_bytes < need)
+    return set_error(H3B_EWORKSPACE, "block_forward_int8: workspace of %zu bytes needed, %zu given",
+                     need, ws_bytes);
+  DevCtx ctx;
+  if ((rc = get_ctx(&ctx))) return rc;
+  return block_forward_int8_impl(ctx, dims, w, wq, mod, rope_cs, n_tokens,
+                                 reinterpret_cast<bf16*>(x), ws, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_quantize_groups(const h3b_bf16* a, int rows, int cols, int8_t* q, float* scale,
+                        void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 1024)
+    return set_error(H3B_EINVAL, "quantize_groups: cols=%d must be a positive multiple of 1024", cols);
+  if (!a || !q || !scale || !al16(a) || !al16(q) || !al16(scale))
+    return set_error(H3B_EINVAL, "quantize_groups: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_quantize_groups(reinterpret_cast<const bf16*>(a), rows, cols, q, scale,
+                                static_cast<cudaStream_t>(stream));
+}
+
+int h3b_ln_modulate_q8(const h3b_bf16* x, int n_tokens, int d, float eps, const float* shift,
+                       const float* scale, int8_t* q, float* q_scale, void* stream) {
+  if (n_tokens < 0 || d <= 0 || d % 256 || d > 4096)
+    return set_error(H3B_EINVAL, "ln_modulate_q8: d=%d must be a multiple of 256 <= 4096", d);
+  if (!x || !q || !q_scale || !shift || !scale || !al16(x) || !al16(q) || !al16(shift) ||
+      !al16(scale))
+    return set_error(H3B_EINVAL, "ln_modulate_q8: NULL or misaligned pointer");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  return launch_ln_modulate_q8(reinterpret_cast<const bf16*>(x), n_tokens, d, eps, shift, scale,
+                               q, q_scale, static_cast<cudaStream_t>(stream));
+}
+
+int h3b_gemm_i8_grouped(const int8_t* A, const float* a_scale, int M, int K, int N,
+                        const int8_t* w_q, const float* w_scale, const h3b_bf16* bias,
+                        const float* gate, h3b_bf16* resid, void* stream) {
+  if (M < 0 || K <= 0 || K % 1024 || N <= 0 || N % 128)
+    return set_error(H3B_EINVAL, "gemm_i8_grouped: K=%d must be a multiple of 1024, N=%d of 128", K, N);
+  const void* ptrs[6] = {A, a_scale, w_q, w_scale, gate, resid};
+  for (const void* p : ptrs)
+    if (!p || !al16(p)) return set_error(H3B_EINVAL, "gemm_i8_grouped: NULL or misaligned pointer");
+  if (bias && !al16(bias)) return set_error(H3B_EINVAL, "gemm_i8_grouped: misaligned bias");
+  DevCtx ctx;
+  if (int rc = get_ctx(&ctx)) return rc;
+  GemmEpilogue e;
+  e.kind = kEpiI8GroupGate;
+  e.bias = reinterpret_cast<const bf16*>(bias);
+  e.row_scale = a_scale;
+  e.act_groups = K / 1024;
+  e.col_scale = w_scale;
+  e.gate = gate;
+  e.out = reinterpret_cast<bf16*>(resid);
+  e.ld_out = N;
+  return launch_gemm_i8_grouped(ctx, A, w_q, M, N, K, e, static_cast<cudaStream_t>(stream));
 }
 
 int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,

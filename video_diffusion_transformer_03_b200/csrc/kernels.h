@@ -37,11 +37,28 @@ enum GemmEpi : int {
   kEpiRopeLN = 5,     // out = bf16(rope(pre)) on columns < rope_cols
   kEpiGeluLN = 6,     // out = bf16(gelu_tanh(pre))
   kEpiHeadEuler = 7,  // out_f32 += euler_dt * pre (fp32 state, in place): a final head
+  // int8 operands with one scale per A row (row_scale [M]) and per B row (col_scale [N]):
+  // pre = (float(acc) * row_scale) * col_scale + bias_f32, then the base epilogue
+  kEpiI8Rope = 8,     // out = bf16(rope(pre)) on columns < rope_cols
+  kEpiI8Gelu = 9,     // out = bf16(gelu_tanh(pre))
+  // grouped int8 (launch_gemm_i8_grouped): acc is the fp32 sum over K groups of
+  // float(acc_g) * row_scale[m, g]; out = bf16(out + gate * (acc * col_scale + bias_f32))
+  kEpiI8GroupGate = 10,
 };
 
 // The base epilogue of a kind (the LN-folded kinds share their base's arithmetic).
 __host__ __device__ constexpr int epi_base(int k) {
-  return k == kEpiRopeLN ? kEpiRope : k == kEpiGeluLN ? kEpiGelu : k;
+  return (k == kEpiRopeLN || k == kEpiI8Rope) ? kEpiRope
+         : (k == kEpiGeluLN || k == kEpiI8Gelu) ? kEpiGelu
+                                                 : k;
+}
+// Kinds whose accumulator is int32 with row and column scales.
+__host__ __device__ constexpr bool epi_int8(int k) {
+  return k == kEpiInt8Deq || k == kEpiI8Rope || k == kEpiI8Gelu;
+}
+// Kinds that add a gated branch to the residual held in `out`.
+__host__ __device__ constexpr bool epi_gated(int k) {
+  return k == kEpiGateResid || k == kEpiInt8Deq || k == kEpiI8GroupGate;
 }
 __host__ __device__ constexpr bool epi_ln_fold(int k) {
   return k == kEpiRopeLN || k == kEpiGeluLN || k == kEpiHeadEuler;
@@ -77,6 +94,8 @@ struct GemmEpilogue {
   // data-parallel (the norm needs the whole head from one accumulator).
   const float* q_gain = nullptr;
   const float* k_gain = nullptr;
+  // kEpiI8GroupGate: groups of 1024 K columns; row_scale is [M, act_groups]
+  int act_groups = 0;
 };
 
 // Kernel scratch: one caller buffer per stream, used by one kernel at a time.  Layout:
@@ -109,10 +128,15 @@ int set_gemm_override(int tile, int sched, int trans);
 int launch_gemm_bf16(const DevCtx& ctx, const bf16* A, const bf16* B, int M, int N, int K,
                      const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream);
-// Same for int8 inputs (int32 accumulate, kEpiInt8Deq).  K % 128 == 0, N % 128 == 0.
+// Same for int8 inputs (int32 accumulate; kEpiInt8Deq, kEpiI8Rope, kEpiI8Gelu).
+// K % 128 == 0, N % 128 == 0.
 int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N, int K,
                    const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                    cudaStream_t stream);
+// Grouped int8 product (kEpiI8GroupGate): one A scale per row and 1024-column group.
+// K % 1024 == 0, N % 128 == 0.
+int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N,
+                           int K, const GemmEpilogue& epi, cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention (tcgen05)
 // scratch (>= gemm_scratch_bytes(), or null) enables the persistent split schedule:
@@ -150,6 +174,14 @@ int launch_final_euler_keep(const bf16* x_l, int n, int n_video, int d, float ep
 int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float eps,
                             const float* final_mod, float dt_sigma, float* x_state,
                             cudaStream_t stream);
+// h = LN(x)(1 + scale) + shift quantised to int8 with one scale per row (q [n, d],
+// q_scale [n]); the quantisation rule of launch_quantize_rows
+int launch_ln_modulate_q8(const bf16* x, int n, int d, float eps, const float* shift,
+                          const float* scale, int8_t* q, float* q_scale, cudaStream_t stream);
+// int8 quantisation with one scale per row and 1024-column group: q [rows, cols],
+// scale [rows, cols / 1024]; cols % 1024 == 0
+int launch_quantize_groups(const bf16* a, int rows, int cols, int8_t* q, float* scale,
+                           cudaStream_t stream);
 // dst = bf16(src), n elements (n % 8 == 0)
 int launch_f32_to_bf16(const float* src, long long n, bf16* dst, cudaStream_t stream);
 // x_state += dt * v (n elements, n % 4 == 0)

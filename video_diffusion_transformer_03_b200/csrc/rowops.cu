@@ -110,6 +110,91 @@ __global__ void __launch_bounds__(128) k_ln_modulate(const void* __restrict__ xi
   }
 }
 
+// Symmetric int8 code of v with inv = 127 / absmax (IEEE fp32 multiply, round to nearest
+// even, clamp): the rule of k_quantize_rows.
+__device__ __forceinline__ uint32_t q8x4(float a, float b, float c, float d, float inv) {
+  const int qa = max(-127, min(127, __float2int_rn(__fmul_rn(a, inv))));
+  const int qb = max(-127, min(127, __float2int_rn(__fmul_rn(b, inv))));
+  const int qc = max(-127, min(127, __float2int_rn(__fmul_rn(c, inv))));
+  const int qd = max(-127, min(127, __float2int_rn(__fmul_rn(d, inv))));
+  return (static_cast<uint32_t>(qa) & 0xFFu) | ((static_cast<uint32_t>(qb) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(qc) & 0xFFu) << 16) | ((static_cast<uint32_t>(qd) & 0xFFu) << 24);
+}
+
+// LayerNorm + AdaLN fused with the int8 quantisation of its output (the int8 path's input
+// to QKV and FC1): h = LN(x)(1 + scale) + shift in fp32, then one scale per row,
+// absmax / 127, and q = clamp(rne(h * (127 / absmax))).  The row stays in registers.
+template <int NV>
+__global__ void __launch_bounds__(128) k_ln_modulate_q8(const bf16* __restrict__ x, int n,
+                                                        float eps, const float* __restrict__ shift,
+                                                        const float* __restrict__ scale,
+                                                        int8_t* __restrict__ q,
+                                                        float* __restrict__ q_scale) {
+  constexpr int D = NV * 256;
+  const int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const int lane = threadIdx.x & 31;
+  float v[NV][8];
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+    unpack8(__ldg(reinterpret_cast<const uint4*>(x + size_t(row) * D + (i * 32 + lane) * 8)), v[i]);
+  float mean, rstd;
+  row_stats<NV>(v, D, eps, mean, rstd);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int col = (i * 32 + lane) * 8;
+    float sh[8], sc[8];
+    load8f(shift + col, sh);
+    load8f(scale + col, sc);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[i][k] = fmaf((v[i][k] - mean) * rstd, 1.0f + sc[k], sh[k]);
+      amax = fmaxf(amax, fabsf(v[i][k]));
+    }
+  }
+  amax = warp_max(amax);
+  const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int col = (i * 32 + lane) * 8;
+    reinterpret_cast<uint2*>(q + size_t(row) * D + col)[0] =
+        make_uint2(q8x4(v[i][0], v[i][1], v[i][2], v[i][3], inv),
+                   q8x4(v[i][4], v[i][5], v[i][6], v[i][7], inv));
+  }
+  if (lane == 0) q_scale[row] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
+// Group quantisation: a warp per (row, 1024-column group) of a [rows, cols] bf16 matrix,
+// the rule of k_quantize_rows within each group; scale [rows, cols / 1024].
+__global__ void __launch_bounds__(256) k_quantize_groups(const bf16* __restrict__ a, int rows,
+                                                         int cols, int8_t* __restrict__ q,
+                                                         float* __restrict__ scale) {
+  constexpr int G = 1024;
+  const int groups = cols / G;
+  const long long gw = blockIdx.x * 8ll + (threadIdx.x >> 5);
+  if (gw >= static_cast<long long>(rows) * groups) return;
+  const int row = static_cast<int>(gw / groups), g = static_cast<int>(gw % groups);
+  const int lane = threadIdx.x & 31;
+  const uint4* src = reinterpret_cast<const uint4*>(a + size_t(row) * cols + size_t(g) * G);
+  float v[4][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    unpack8(__ldg(src + i * 32 + lane), v[i]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(v[i][k]));
+  }
+  amax = warp_max(amax);
+  const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  uint2* dst = reinterpret_cast<uint2*>(q + size_t(row) * cols + size_t(g) * G);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    dst[i * 32 + lane] = make_uint2(q8x4(v[i][0], v[i][1], v[i][2], v[i][3], inv),
+                                    q8x4(v[i][4], v[i][5], v[i][6], v[i][7], inv));
+  if (lane == 0) scale[size_t(row) * groups + g] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
 // v = LN(x_l)(1 + scale_s) + shift_s (s = video below n_video, else audio);
 // x_state += dt * v.
 template <int NV>
@@ -615,6 +700,24 @@ int launch_core_reuse_final(const float* r_in, int n, int n_video, int d, float 
                              nullptr, r_in, n, n_video, eps, final_mod, dt_sigma, x_state,
                              nullptr, nullptr)));
   return check_launch("core_reuse_final");
+}
+
+int launch_ln_modulate_q8(const bf16* x, int n, int d, float eps, const float* shift,
+                          const float* scale, int8_t* q, float* q_scale, cudaStream_t stream) {
+  if (n <= 0) return 0;
+  const int grid = (n + kRowWarps - 1) / kRowWarps;
+  H3B_NV_SWITCH(d / 256, (k_ln_modulate_q8<NV><<<grid, 32 * kRowWarps, 0, stream>>>(
+                             x, n, eps, shift, scale, q, q_scale)));
+  return check_launch("ln_modulate_q8");
+}
+
+int launch_quantize_groups(const bf16* a, int rows, int cols, int8_t* q, float* scale,
+                           cudaStream_t stream) {
+  const long long warps = static_cast<long long>(rows) * (cols / 1024);
+  if (warps <= 0) return 0;
+  k_quantize_groups<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(a, rows, cols, q,
+                                                                               scale);
+  return check_launch("quantize_groups");
 }
 
 int launch_f32_to_bf16(const float* src, long long n, bf16* dst, cudaStream_t stream) {

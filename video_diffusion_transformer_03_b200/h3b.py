@@ -54,6 +54,11 @@ class LatentHeads(ctypes.Structure):
                 ("c_head", ctypes.c_void_p * 2), ("dv_head", ctypes.c_void_p * 2)]
 
 
+class Int8Block(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_qkv_q", "s_qkv", "w_fc1_q", "s_fc1", "w_fc2_q", "s_fc2")]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
@@ -96,6 +101,12 @@ _SIGS = {
                                      ctypes.POINTER(BlockWeights), _P, _P,
                                      ctypes.POINTER(LatentHeads), _I, _I, _F, _F, _P, _P, _SZ,
                                      _P]),
+    "h3b_workspace_size_int8": (_SZ, [ctypes.POINTER(Dims), _I]),
+    "h3b_block_forward_int8": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(BlockWeights),
+                                    ctypes.POINTER(Int8Block), _P, _P, _I, _P, _P, _SZ, _P]),
+    "h3b_ln_modulate_q8": (_I, [_P, _I, _I, _F, _P, _P, _P, _P, _P]),
+    "h3b_quantize_groups": (_I, [_P, _I, _I, _P, _P, _P]),
+    "h3b_gemm_i8_grouped": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "h3b_reuse_schedule": (_I, [_I, _I, _P]),
     "h3b_denoise_step_keep": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                                    ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P,
@@ -403,6 +414,51 @@ def denoise_step_latent(dims: Dims, grid: Grid, blocks: Sequence[BlockWeights], 
                                        int(bool(unpair_bypass)), sigma, sigma_next, _ptr(latent),
                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
     del keep
+
+
+def quantize_block_int8(p, stream=None):
+    """Int8 weights of one block (device tensors) from its bf16 weights p: per-output-
+    channel quantize_rows of w_qkv, w_fc1, w_fc2.  Returns (tensors, Int8Block)."""
+    t = {}
+    for name in ("qkv", "fc1", "fc2"):
+        w = p["w_" + name]
+        t["w_%s_q" % name] = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+        t["s_" + name] = torch.empty(w.shape[0], dtype=torch.float32, device=w.device)
+        quantize_rows(w, t["w_%s_q" % name], t["s_" + name], stream)
+    return t, Int8Block(*[_ptr(t[k]) for k in ("w_qkv_q", "s_qkv", "w_fc1_q", "s_fc1",
+                                                 "w_fc2_q", "s_fc2")])
+
+
+def workspace_size_int8(dims: Dims, n_tokens: int) -> int:
+    return lib.h3b_workspace_size_int8(ctypes.byref(dims), n_tokens)
+
+
+def block_forward_int8(dims: Dims, weights: BlockWeights, wq: Int8Block, mod, rope_cs, x, ws,
+                       stream=None) -> None:
+    _dev(x, torch.bfloat16, "x"); _dev(mod, torch.float32, "mod")
+    _check(lib.h3b_block_forward_int8(ctypes.byref(dims), ctypes.byref(weights), ctypes.byref(wq),
+                                      _ptr(mod), _ptr(rope_cs), x.shape[0], _ptr(x), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def ln_modulate_q8(x, eps, shift, scale, q, q_scale, stream=None) -> None:
+    _dev(x, torch.bfloat16, "x"); _dev(q, torch.int8, "q"); _dev(q_scale, torch.float32, "q_scale")
+    _check(lib.h3b_ln_modulate_q8(_ptr(x), x.shape[0], x.shape[1], eps, _ptr(shift), _ptr(scale),
+                                  _ptr(q), _ptr(q_scale), _stream(stream)))
+
+
+def quantize_groups(a, q, scale, stream=None) -> None:
+    _dev(a, torch.bfloat16, "a"); _dev(q, torch.int8, "q"); _dev(scale, torch.float32, "scale")
+    _check(lib.h3b_quantize_groups(_ptr(a), a.shape[0], a.shape[1], _ptr(q), _ptr(scale),
+                                   _stream(stream)))
+
+
+def gemm_i8_grouped(A, a_scale, w_q, w_scale, bias, gate, resid, stream=None) -> None:
+    _dev(A, torch.int8, "A"); _dev(w_q, torch.int8, "w_q"); _dev(resid, torch.bfloat16, "resid")
+    M, K = A.shape
+    _check(lib.h3b_gemm_i8_grouped(_ptr(A), _ptr(a_scale), M, K, w_q.shape[0], _ptr(w_q),
+                                   _ptr(w_scale), _ptr(bias), _ptr(gate), _ptr(resid),
+                                   _stream(stream)))
 
 
 def reuse_schedule(steps: int, every: int) -> np.ndarray:
