@@ -416,6 +416,45 @@ def time_gemm_widths(dev, peaks, reps=10):
     return res
 
 
+def time_attention_forms(dev, peaks, reps=10):
+    """Attention alone at the 512x512 (1,600 tokens) and 768x1344 (11,344 tokens) shapes,
+    24 heads x 128, split schedule, in both kernel forms (one or two query tiles per CTA);
+    CUDA-graph replays of `reps` launches."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b
+    g = torch.Generator(device=dev).manual_seed(5)
+    ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
+    res = {}
+    for n in (1600, 11344):
+        d = 24 * 128
+        qkv = torch.randn(n, 3 * d, generator=g, device=dev).to(torch.bfloat16)
+        out = torch.empty(n, d, dtype=torch.bfloat16, device=dev)
+        for name, v in (("two_tile", h3b.ATTN_TWO_TILES), ("one_tile", h3b.ATTN_ONE_TILE)):
+            with h3b.attention_variant(v):
+                for _ in range(3):
+                    h3b.attention(qkv, 24, 128, out, ws=ws)
+                torch.cuda.synchronize(dev)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for _ in range(reps):
+                        h3b.attention(qkv, 24, 128, out, ws=ws)
+            graph.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            del graph
+            ms = e0.elapsed_time(e1) / reps
+            tf = 4 * n * n * d / (ms * 1e-3) / 1e12
+            res[f"{name}_{n}"] = {"us": ms * 1e3, "tflops": tf, "frac": tf / peaks["bf16_tflops"]}
+        del qkv, out
+    h3b.sync_status()
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_denoise(cfg_name, dev, reps, warm=1):
     """Device time of complete denoises of another workload (graph replays)."""
     import torch
@@ -711,6 +750,7 @@ def run_gpu(args):
         for name, reps in (("dit512_tokred", 20), ("dit768x1344", 2)):
             if name != args.config:
                 also[name] = time_denoise(name, dev, reps)
+        also["attention_forms"] = time_attention_forms(dev, peaks)
         also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
         also["gemm_widths"] = time_gemm_widths(dev, peaks)

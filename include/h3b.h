@@ -185,6 +185,12 @@ int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, in
  * captured. */
 int h3b_set_gemm_override(int tile, int sched, int trans);
 
+/* Select the attention kernel's form for later launches of this process, for tests and
+ * measurements: 0 automatic (the default: two 128-query tiles per CTA sharing each K/V
+ * tile, one softmax warpgroup each), 1 one query tile per CTA, 2 two tiles.  Returns
+ * H3B_OK or H3B_EINVAL. */
+int h3b_set_attention_variant(int variant);
+
 /* ---------------------------------------------------------------- hot-path steps */
 /* AdaLN modulation vectors: mod[j] = sum_k w[j, k] c[k] + b[j], j < n_out.
  * w [n_out, c_dim] bf16, b [n_out] bf16, c [c_dim] bf16, mod [n_out] fp32 (all device).
@@ -546,8 +552,10 @@ int h3b_gemm_bf16_ln(const h3b_bf16* A, const h3b_bf16* B, int M, int N, int K, 
  * n_heads head_dim] bf16 (device).  out = softmax(q k^T / sqrt(head_dim)) v per head.
  * ws: NULL, or 16-byte aligned device scratch of h3b_gemm_workspace_size() bytes (the
  * same scratch the GEMM calls take; one kernel at a time per buffer).  With it the work
- * is split evenly over the SMs (a query tile may be finished by two CTAs, merged through
- * the scratch); without it, one CTA per (head, 128-query tile).  A smaller ws is ignored. */
+ * is split evenly over the SMs (a query block may be finished by two CTAs, merged through
+ * the scratch); without it, one CTA per (head, query block).  A query block is 256 rows
+ * (two 128-row tiles sharing each K/V load; see h3b_set_attention_variant).  A smaller
+ * ws is ignored. */
 int h3b_attention(const h3b_bf16* qkv, int n_tokens, int n_heads, int head_dim,
                   h3b_bf16* out, void* ws, size_t ws_bytes, void* stream);
 

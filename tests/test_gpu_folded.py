@@ -115,10 +115,13 @@ def test_folded_block_vs_oracle(name):
         tol = _update_tol(cfg, params, c, x)
         eu = rel_l2(got - xin, xo - xin)
         assert eu <= tol, f"update rel-L2 {eu:.3e} > {tol:.3e}"
-    # the statistics the FC2 epilogue wrote describe the stored output
+    # the statistics the FC2 epilogue wrote describe the output before its bf16 rounding:
+    # against those of the stored output they differ by the rounding only (each value moves
+    # by at most 2^-9 of itself, averaging out over a 256-column group)
     s, r = st.numpy().astype(np.float64), st_ref.numpy().astype(np.float64)
-    assert np.max(np.abs(s[..., 0] - r[..., 0])) < 1e-5 * (1 + np.max(np.abs(r[..., 0])))
-    assert rel_l2(s[..., 1], r[..., 1]) < 1e-5
+    scale = np.sqrt(r[..., 1] / 256.0) + np.abs(r[..., 0])
+    assert np.max(np.abs(s[..., 0] - r[..., 0]) / scale) < 2e-3
+    assert rel_l2(s[..., 1], r[..., 1]) < 2e-3
 
 
 def test_folded_block_close_to_unfolded_block():
@@ -235,14 +238,18 @@ def test_gate_resid_gemm_writes_row_statistics(M, N, K):
                      gate=g.to(DEV), stats_out=st, ws=ws)
     h3b.gemm_bf16(A.to(DEV), B.to(DEV), h3b.EPI_GATE_RESID, bias.to(DEV), plain, gate=g.to(DEV),
                   ws=ws)
-    ref = torch.empty_like(st)
-    h3b.row_stats(out, ref)
     h3b.sync_status()
     # the output is that of the plain gated-residual epilogue, bit for bit
     assert torch.equal(out, plain)
-    s, r = st.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64)
-    assert np.max(np.abs(s[..., 0] - r[..., 0])) < 1e-5 * (1 + np.max(np.abs(r[..., 0])))
-    assert rel_l2(s[..., 1], r[..., 1]) < 1e-5
+    # the statistics are those of the exact (unrounded) output, per 256-column group
+    want = O.gated_residual(np64(resid), np64(g), np64(A) @ np64(B).T + np64(bias))
+    gr = want.reshape(M, N // 256, 256)
+    mean = gr.mean(axis=2)
+    m2 = ((gr - mean[..., None]) ** 2).sum(axis=2)
+    s = st.cpu().numpy().astype(np.float64)
+    scale = np.sqrt(m2 / 256.0) + np.abs(mean)
+    assert np.max(np.abs(s[..., 0] - mean) / scale) < 2e-3
+    assert rel_l2(s[..., 1], m2) < 2e-3
 
 
 def test_ln_folded_gemm_large_row_offset():

@@ -246,24 +246,28 @@ def _attention_want(qkv, n, heads, hd):
     return O.attention(q, k, v).reshape(n, d)
 
 
+@pytest.mark.parametrize("variant", [h3b.ATTN_TWO_TILES, h3b.ATTN_ONE_TILE],
+                         ids=["two-tile", "one-tile"])
 @pytest.mark.parametrize("split", [False, True], ids=["per-unit", "split"])
 @pytest.mark.parametrize("n,heads,hd,std", ATTN_CASES)
-def test_attention(n, heads, hd, std, split):
+def test_attention(n, heads, hd, std, split, variant):
     d = heads * hd
     qkv = rnd((n, 3 * d), std, seed=n + heads)
     out = torch.empty((n, d), dtype=torch.bfloat16, device=DEV)
     ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV) if split else None
-    h3b.attention(qkv.to(DEV), heads, hd, out, ws=ws)
-    _sync()
+    with h3b.attention_variant(variant):
+        h3b.attention(qkv.to(DEV), heads, hd, out, ws=ws)
+        _sync()
     want = _attention_want(qkv, n, heads, hd)
     got = np64(out)
     assert rel_l2(got, want) < 1e-2
     assert _worst_unit_rel_l2(got, want, heads, hd) < 2e-2
 
 
-def test_attention_split_is_repeatable_and_matches_per_unit_closely():
-    # the same scratch over and over (flags are handed back at zero after each merge)
-    n, heads, hd = 520, 40, 128
+@pytest.mark.parametrize("n,heads,hd", [(520, 40, 128), (1600, 24, 128), (700, 30, 64)])
+def test_attention_split_is_repeatable_and_matches_per_unit_closely(n, heads, hd):
+    # the same scratch over and over (flags are handed back at zero after each merge); the
+    # two-tile form parks the lower part of a cut block's O in bf16
     d = heads * hd
     qkv = rnd((n, 3 * d), 2.0, seed=11).to(DEV)
     ws = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV)
@@ -278,6 +282,12 @@ def test_attention_split_is_repeatable_and_matches_per_unit_closely():
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     # a cut unit differs from the uncut one only by the merge's rounding
     assert rel_l2(np64(outs[0]), np64(ref)) < 4e-3
+    # and the one-tile form agrees with the two-tile form closely
+    one = torch.empty_like(ref)
+    with h3b.attention_variant(h3b.ATTN_ONE_TILE):
+        h3b.attention(qkv, heads, hd, one, ws=ws)
+        _sync()
+    assert rel_l2(np64(one), np64(ref)) < 4e-3
 
 
 def test_attention_uniform_keys_average_values():

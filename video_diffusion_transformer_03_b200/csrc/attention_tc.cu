@@ -547,6 +547,572 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+
+// ============================================================================ two-tile form
+// The unit is (head, 256-query block): two 128-query tiles that share every K and V tile
+// load, each with its own softmax warpgroup, so the two softmax streams overlap each
+// other and the tensor core (one softmax warpgroup per CTA was the critical path).
+// Roles (384 threads, three warpgroups):
+//   warpgroup 0  warp 0 TMA producer, warp 1 MMA issuer, warps 2-3 idle (88 registers);
+//   warpgroup 1  softmax of query tile 0 (rows 0-127 of the unit), 208 registers;
+//   warpgroup 2  softmax of query tile 1 (rows 128-255), 208 registers (the split adds up
+//                to the 384 x 168 registers the CTA is launched with).
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512): one score buffer per tile,
+// so S_j+1 of a tile is computed as soon as its softmax has read S_j into registers.
+// Shared memory: Q0, Q1, P0, P1 and a 3-slot ring of K/V tiles loaded in the order the
+// tensor core consumes them (K_j+1 before V_j).  Per step the MMA thread issues S0, S1 of
+// key tile j, then O0 += P0 V, O1 += P1 V of key tile j - 1 (at a unit's first step, the
+// previous unit's last P V goes first).  A query block whose second tile starts past the
+// last token skips that tile (its MMAs and its softmax).  The split schedule is that of
+// the one-tile form, with the parked running state of both tiles (O in bf16, (max, sum)
+// in fp32).
+constexpr int kRing = 3;
+
+template <int HD>
+struct Attn2Cfg {
+  static constexpr int kNBox = HD / 64;
+  static constexpr uint32_t kQBytes = kNBox * kBox;   // one 128-row tile
+  static constexpr uint32_t kKVBytes = kNBox * kBox;
+  static constexpr uint32_t kPBytes = 2 * kBox;
+  static constexpr size_t kSmem = 1024 + 2 * size_t(kQBytes) + 2 * size_t(kPBytes) +
+                                  size_t(kRing) * kKVBytes + 512;
+  static_assert(kSmem <= 232448, "two-tile attention shared memory above 227 KB");
+};
+
+struct Attn2Params {
+  int n, d, n_kv, n_qb;  // tokens, n_heads * head_dim, key tiles, 256-query blocks per head
+  long long steps;       // units * n_kv
+  float scale_log2;
+  bf16* out;
+  uint4* part_o;         // [gridDim.x][2 tiles][head_dim / 8][128] uint4 (8 bf16)
+  float2* part_ml;       // [gridDim.x][2 tiles][128]
+  unsigned long long* flags;  // [gridDim.x][2 tiles][4]
+  unsigned long long seq;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ Range cta_range2(const Attn2Params& p) {
+  Range r;
+  r.begin = p.steps * static_cast<long long>(blockIdx.x) / static_cast<long long>(gridDim.x);
+  r.end = p.steps * static_cast<long long>(blockIdx.x + 1) / static_cast<long long>(gridDim.x);
+  r.u_first = static_cast<int>(r.begin / p.n_kv);
+  r.u_last = static_cast<int>((r.end - 1) / p.n_kv);
+  return r;
+}
+
+__device__ __forceinline__ void segment2(const Attn2Params& p, const Range& r, int k, int& unit,
+                                         int& j0, int& j1) {
+  unit = r.u_last - k;
+  const long long base = static_cast<long long>(unit) * p.n_kv;
+  j0 = static_cast<int>(r.begin > base ? r.begin - base : 0ll);
+  j1 = static_cast<int>(r.end - base < p.n_kv ? r.end - base : static_cast<long long>(p.n_kv));
+}
+
+// Whether the unit's second query tile holds any token.
+__device__ __forceinline__ bool tile1_valid(const Attn2Params& p, int unit) {
+  return (unit % p.n_qb) * 256 + 128 < p.n;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(384, 1)
+    k_attention_tc2(const __grid_constant__ CUtensorMap tm, const Attn2Params p) {
+  using Cfg = Attn2Cfg<HD>;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false);
+  constexpr uint32_t IDESC_PV = idesc_bf16(128, HD, true);
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kOCol = 256;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                          // 2 tiles
+  uint8_t* sP = sQ + 2 * Cfg::kQBytes;         // 2 tiles
+  uint8_t* sKV = sP + 2 * Cfg::kPBytes;        // kRing slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kRing * Cfg::kKVBytes);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [kRing]
+  uint64_t* kv_empty = bars + 5;  // [kRing]
+  uint64_t* s_full = bars + 8;    // [2 tiles]
+  uint64_t* s_free = bars + 10;   // [2]
+  uint64_t* p_full = bars + 12;   // [2]
+  uint64_t* p_free = bars + 14;   // [2]
+  uint64_t* o_empty = bars + 16;  // [2]
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Range rg = cta_range2(p);
+  const int n_seg = rg.u_last - rg.u_first + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&s_free[w], 4);
+      mbar_init(&p_full[w], 4);
+      mbar_init(&p_free[w], 1);
+      mbar_init(&o_empty[w], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_map(&tm);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    regs_dealloc<88>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------------ producer
+      // Loads in the MMA's consumption order: per step t, K(t) then V(t - 1), except at a
+      // unit's first step (not the walk's first), where V(t - 1) goes first; the Q tiles
+      // of a unit before its first K.
+      bool ok = true;
+      int slot = 0;
+      uint32_t ring_phase = 0;
+      int armed[kRing] = {-1, -1, -1};
+      int q_armed = -1;
+      const long long total = rg.end - rg.begin;
+      int ks = 0, js = 0, js0 = 0, js1 = 0, unit_s = 0;  // step t's segment and key tile
+      int kp = 0, jp = 0, jp0 = 0, jp1 = 0, unit_p = 0;  // step t - 1's
+      segment2(p, rg, 0, unit_s, js0, js1);
+      js = js0;
+      segment2(p, rg, 0, unit_p, jp0, jp1);
+      jp = jp0;
+      auto load = [&](int x, int y) -> bool {
+        if (!wait_bar(&kv_empty[slot], ring_phase ^ 1u, abort_flag, p.err, kErrAttnWait))
+          return false;
+        mbar_arrive_expect_tx(&kv_full[slot], Cfg::kKVBytes);
+#pragma unroll
+        for (int b = 0; b < Cfg::kNBox; ++b)
+          tma_load_2d(sKV + slot * Cfg::kKVBytes + b * kBox, &tm, &kv_full[slot], x + 64 * b, y);
+        armed[slot] = static_cast<int>(ring_phase);
+        if (++slot == kRing) {
+          slot = 0;
+          ring_phase ^= 1u;
+        }
+        return true;
+      };
+      auto load_k = [&]() -> bool {  // K of step t, and the unit's Q tiles first
+        const int head = unit_s / p.n_qb, qb = unit_s % p.n_qb;
+        if (js == js0) {
+          if (ks > 0 && !wait_bar(q_empty, static_cast<uint32_t>(ks - 1) & 1u, abort_flag, p.err,
+                                  kErrAttnWait))
+            return false;
+          mbar_arrive_expect_tx(q_full, 2 * Cfg::kQBytes);
+#pragma unroll
+          for (int w = 0; w < 2; ++w)
+#pragma unroll
+            for (int b = 0; b < Cfg::kNBox; ++b)
+              tma_load_2d(sQ + w * Cfg::kQBytes + b * kBox, &tm, q_full, head * HD + 64 * b,
+                          qb * 256 + w * 128);
+          q_armed = ks & 1;
+        }
+        if (!load(p.d + head * HD, js * 128)) return false;
+        if (++js == js1 && ++ks < n_seg) {
+          segment2(p, rg, ks, unit_s, js0, js1);
+          js = js0;
+        }
+        return true;
+      };
+      auto load_v = [&]() -> bool {  // V of step t - 1
+        const int head = unit_p / p.n_qb;
+        if (!load(2 * p.d + head * HD, jp * 128)) return false;
+        if (++jp == jp1 && ++kp < n_seg) {
+          segment2(p, rg, kp, unit_p, jp0, jp1);
+          jp = jp0;
+        }
+        return true;
+      };
+      for (long long t = 0; t <= total && ok; ++t) {
+        const bool first = t >= 1 && t < total && js == js0;
+        if (first) ok = load_v() && load_k();
+        else ok = (t >= total || load_k()) && (t < 1 || load_v());
+      }
+      if (!ok) {
+        if (q_armed >= 0) drain_wait(q_full, static_cast<uint32_t>(q_armed));
+        for (int s = 0; s < kRing; ++s)
+          if (armed[s] >= 0) drain_wait(&kv_full[s], static_cast<uint32_t>(armed[s]));
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      int slot = 0;
+      uint32_t ring_phase = 0;
+      int cnt[2] = {0, 0};    // S products issued per tile (= P V products, one behind)
+      int pvc[2] = {0, 0};    // P V products issued per tile
+      int units_done[2] = {0, 0};
+      int ks = 0, js = 0, js0 = 0, js1 = 0, unit_s = 0;
+      int kp = 0, jp = 0, jp0 = 0, jp1 = 0, unit_p = 0;
+      segment2(p, rg, 0, unit_s, js0, js1);
+      js = js0;
+      segment2(p, rg, 0, unit_p, jp0, jp1);
+      jp = jp0;
+      auto ring_take = [&](int& s_out) -> bool {
+        if (!wait_bar(&kv_full[slot], ring_phase, abort_flag, p.err, kErrAttnWait)) return false;
+        s_out = slot;
+        if (++slot == kRing) {
+          slot = 0;
+          ring_phase ^= 1u;
+        }
+        return true;
+      };
+      auto issue_s = [&]() -> bool {
+        const bool v1 = tile1_valid(p, unit_s);
+        if (js == js0 &&
+            !wait_bar(q_full, static_cast<uint32_t>(ks) & 1u, abort_flag, p.err, kErrAttnWait))
+          return false;
+        int ksl;
+        if (!ring_take(ksl)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sKV + ksl * Cfg::kKVBytes);
+        for (int w = 0; w < (v1 ? 2 : 1); ++w) {
+          if (cnt[w] >= 1 && !wait_bar(&s_free[w], static_cast<uint32_t>(cnt[w] - 1) & 1u,
+                                       abort_flag, p.err, kErrAttnWait))
+            return false;
+          tc_fence_after();
+          const uint32_t q0 = smem_u32(sQ + w * Cfg::kQBytes);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+            umma_f16(tmem + w * 128, sdesc_sw128(q0 + off, 16, 1024),
+                     sdesc_sw128(k0 + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[w]);
+          ++cnt[w];
+        }
+        tc_commit(&kv_empty[ksl]);
+        if (++js == js1) {
+          tc_commit(q_empty);
+          if (++ks < n_seg) {
+            segment2(p, rg, ks, unit_s, js0, js1);
+            js = js0;
+          }
+        }
+        return true;
+      };
+      auto issue_pv = [&]() -> bool {
+        const bool v1 = tile1_valid(p, unit_p);
+        const bool first = jp == jp0;
+        int vsl;
+        if (!ring_take(vsl)) return false;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sKV + vsl * Cfg::kKVBytes);
+        for (int w = 0; w < (v1 ? 2 : 1); ++w) {
+          // the tile's previous unit must have read O out before it is overwritten
+          if (first && units_done[w] > 0 &&
+              !wait_bar(&o_empty[w], static_cast<uint32_t>(units_done[w] - 1) & 1u, abort_flag,
+                        p.err, kErrAttnWait))
+            return false;
+          if (!wait_bar(&p_full[w], static_cast<uint32_t>(pvc[w]) & 1u, abort_flag, p.err,
+                        kErrAttnWait))
+            return false;
+          tc_fence_after();
+          const uint32_t p0 = smem_u32(sP + w * Cfg::kPBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t poff = (kk >> 2) * kBox + (kk & 3) * 32;
+            umma_f16(tmem + kOCol + w * 128, sdesc_sw128(p0 + poff, 16, 1024),
+                     sdesc_sw128(v0 + kk * 2048, kBox, 1024), IDESC_PV,
+                     (!first || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&p_free[w]);
+          ++pvc[w];
+        }
+        tc_commit(&kv_empty[vsl]);
+        if (++jp == jp1) {
+          units_done[0] += 1;
+          if (v1) units_done[1] += 1;
+          if (++kp < n_seg) {
+            segment2(p, rg, kp, unit_p, jp0, jp1);
+            jp = jp0;
+          }
+        }
+        return true;
+      };
+      const long long total = rg.end - rg.begin;
+      for (long long t = 0; t <= total; ++t) {
+        const bool pv_first = t >= 1 && t < total && js == js0;
+        if (pv_first && !issue_pv()) break;
+        if (t < total && !issue_s()) break;
+        if (t >= 1 && !pv_first && !issue_pv()) break;
+      }
+      tc_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    regs_alloc<208>();
+    // ------------------------------------------------------------------ softmax (tile w)
+    const int w = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem + lane_addr + w * 128;
+    const uint32_t o_addr = tmem + lane_addr + kOCol + w * 128;
+    const float sl2 = p.scale_log2;
+    uint8_t* pbuf = sP + w * Cfg::kPBytes + row * 128;
+    bool ok = true;
+    int c = 0;  // steps of this tile so far
+    for (int k = 0; k < n_seg && ok; ++k) {
+      int unit, j0, j1;
+      segment2(p, rg, k, unit, j0, j1);
+      if (w == 1 && !tile1_valid(p, unit)) continue;
+      float m_used = -INFINITY;
+      float l = 0.f;
+      for (int j = j0; j < j1; ++j, ++c) {
+        const uint32_t ph = static_cast<uint32_t>(c) & 1u;
+        ok = __all_sync(0xffffffffu, wait_bar(&s_full[w], ph, abort_flag, p.err, kErrAttnWait));
+        if (!ok) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t r[128];
+          tmem_ld128_sync(s_addr, r);
+#pragma unroll
+          for (int q = 0; q < 128; ++q) s[q] = __uint_as_float(r[q]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[w]);
+        if ((j + 1) * 128 > p.n) {
+          const int valid = p.n - j * 128;
+#pragma unroll
+          for (int q = 0; q < 128; ++q)
+            if (q >= valid) s[q] = -INFINITY;
+        }
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          m8[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+          for (int q = 16; q < 128; q += 16) m8[i] = max3(m8[i], s[q + i], s[q + 8 + i]);
+        }
+        const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
+                              fmaxf(m8[6], m8[7]));
+        const float mxs = mx * sl2;
+        if (j == j0) {
+          m_used = mxs;
+        } else {
+          const bool need = mxs > m_used + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            // O must hold every earlier P V product of this unit before it is rescaled
+            ok = __all_sync(0xffffffffu, wait_bar(&p_free[w], static_cast<uint32_t>(c - 1) & 1u,
+                                                  abort_flag, p.err, kErrAttnWait));
+            if (!ok) break;
+            tc_fence_after();
+            const float alpha = need ? ex2_approx(m_used - mxs) : 1.0f;
+#pragma unroll
+            for (int cc = 0; cc < HD / 32; ++cc) {
+              uint32_t r[32];
+              tmem_ld32(o_addr + cc * 32, r);
+              tmem_wait_ld(r);
+#pragma unroll
+              for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+              tmem_st32(o_addr + cc * 32, r);
+            }
+            tmem_wait_st();
+            l *= alpha;
+            if (need) m_used = mxs;
+          }
+        }
+        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < 128; ++q) {
+          const float e = ex2_approx(fmaf(s[q], sl2, -m_used));
+          sum8[q & 7] += e;
+          s[q] = e;
+        }
+#pragma unroll
+        for (int i = 4; i > 0; i >>= 1)
+#pragma unroll
+          for (int q = 0; q < i; ++q) sum8[q] += sum8[q + i];
+        l += sum8[0];
+        if (c >= 1) {  // the tile's P buffer is free once its previous P V has completed
+          ok = __all_sync(0xffffffffu, wait_bar(&p_free[w], static_cast<uint32_t>(c - 1) & 1u,
+                                                abort_flag, p.err, kErrAttnWait));
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int c16 = 0; c16 < 16; ++c16) {
+          uint4 u;
+          u.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
+          u.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
+          u.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
+          u.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
+          const int chunk = (c16 & 7) ^ (row & 7);
+          *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kBox + chunk * 16) = u;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[w]);
+      }
+      if (!ok) break;
+      // ---- end of the unit: O holds every P V product once the last one completes
+      ok = __all_sync(0xffffffffu, wait_bar(&p_free[w], static_cast<uint32_t>(c - 1) & 1u,
+                                            abort_flag, p.err, kErrAttnWait));
+      if (!ok) break;
+      tc_fence_after();
+      const int head = unit / p.n_qb, qb = unit % p.n_qb;
+      const int part = static_cast<int>(blockIdx.x) * 2 + w;
+      if (j1 < p.n_kv) {
+        // lower part of a split unit: park the running state for the owner (next CTA)
+        uint4* po = p.part_o + size_t(part) * (HD / 8) * 128 + row;
+#pragma unroll 1
+        for (int cc = 0; cc < HD / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + cc * 32, r);
+          tmem_wait_ld(r);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            __stcg(po + size_t(cc * 4 + i) * 128,
+                   make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]), __uint_as_float(r[8 * i + 1])),
+                              pack_bf16x2(__uint_as_float(r[8 * i + 2]), __uint_as_float(r[8 * i + 3])),
+                              pack_bf16x2(__uint_as_float(r[8 * i + 4]), __uint_as_float(r[8 * i + 5])),
+                              pack_bf16x2(__uint_as_float(r[8 * i + 6]), __uint_as_float(r[8 * i + 7]))));
+        }
+        __stcg(p.part_ml + size_t(part) * 128 + row, make_float2(m_used, l));
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_u64(p.flags + part * 4 + quarter, p.seq);
+      } else {
+        float wa = 0.f, wb = 1.f;
+        const uint4* po = nullptr;
+        if (j0 > 0) {
+          const int src = part - 2;  // the same tile of the previous CTA
+          ok = __all_sync(0xffffffffu,
+                          wait_flag(p.flags + src * 4 + quarter, p.seq, abort_flag, p.err));
+          if (!ok) break;
+          const float2 ml = __ldcg(p.part_ml + size_t(src) * 128 + row);
+          const float m = fmaxf(ml.x, m_used);
+          wa = ex2_approx(ml.x - m);
+          wb = ex2_approx(m_used - m);
+          l = ml.y * wa + l * wb;
+          po = p.part_o + size_t(src) * (HD / 8) * 128 + row;
+        }
+        const float inv_l = 1.0f / l;
+        wa *= inv_l;
+        wb *= inv_l;
+        const int grow = qb * 256 + w * 128 + row;
+#pragma unroll
+        for (int cc = 0; cc < HD / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(o_addr + cc * 32, r);
+          tmem_wait_ld(r);
+          float o[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(r[q]) * wb;
+          if (po != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 a = __ldcg(po + size_t(cc * 4 + i) * 128);
+              const float2 a0 = unpack_bf16x2(a.x), a1 = unpack_bf16x2(a.y);
+              const float2 a2 = unpack_bf16x2(a.z), a3 = unpack_bf16x2(a.w);
+              o[8 * i + 0] = fmaf(a0.x, wa, o[8 * i + 0]);
+              o[8 * i + 1] = fmaf(a0.y, wa, o[8 * i + 1]);
+              o[8 * i + 2] = fmaf(a1.x, wa, o[8 * i + 2]);
+              o[8 * i + 3] = fmaf(a1.y, wa, o[8 * i + 3]);
+              o[8 * i + 4] = fmaf(a2.x, wa, o[8 * i + 4]);
+              o[8 * i + 5] = fmaf(a2.y, wa, o[8 * i + 5]);
+              o[8 * i + 6] = fmaf(a3.x, wa, o[8 * i + 6]);
+              o[8 * i + 7] = fmaf(a3.y, wa, o[8 * i + 7]);
+            }
+          }
+          if (grow < p.n) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(p.out + size_t(grow) * p.d + head * HD + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16x2(o[8 * i + 0], o[8 * i + 1]);
+              u.y = pack_bf16x2(o[8 * i + 2], o[8 * i + 3]);
+              u.z = pack_bf16x2(o[8 * i + 4], o[8 * i + 5]);
+              u.w = pack_bf16x2(o[8 * i + 6], o[8 * i + 7]);
+              dst[i] = u;
+            }
+          }
+        }
+        if (po != nullptr) {
+          __syncwarp();
+          if (lane == 0) p.flags[(part - 2) * 4 + quarter] = 0ull;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[w]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int HD>
+int launch_hd2(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, void* scratch,
+               size_t scratch_bytes, cudaStream_t stream) {
+  using Cfg = Attn2Cfg<HD>;
+  const int d = heads * HD;
+  CUtensorMap tm;
+  if (!make_tmap_2d(&tm, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint64_t(n), uint64_t(3 * d),
+                    uint64_t(3 * d) * 2, 128, 64))
+    return set_error(-3, "attention: cuTensorMapEncodeTiled failed (n=%d d=%d)", n, d);
+  auto kernel = k_attention_tc2<HD>;
+  static std::atomic<uint32_t> attr_done{0};
+  const uint32_t bit = 1u << (ctx.device & 31);
+  if (!(attr_done.load() & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Cfg::kSmem));
+    if (e != cudaSuccess)
+      return set_error(-3, "attention: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    attr_done.fetch_or(bit);
+  }
+  Attn2Params p = {};
+  p.n = n;
+  p.d = d;
+  p.n_kv = (n + 127) / 128;
+  p.n_qb = (n + 255) / 256;
+  const long long units = static_cast<long long>(p.n_qb) * heads;
+  p.steps = units * p.n_kv;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(HD)));
+  p.out = out;
+  p.err = ctx.err_flag;
+  long long grid = units;
+  if (scratch != nullptr && scratch_bytes >= kScratchBytes) {
+    static_assert(size_t(kMaxSkCtas) * 2 * 128 * (128 * 2 + 8) <= kSkFlagsOffset,
+                  "two-tile attention partial states must fit the slot area");
+    static_assert(size_t(kMaxSkCtas) * 2 * 4 * 8 <= kScratchBytes - kSkFlagsOffset,
+                  "two-tile attention flags must fit the flag area");
+    grid = std::min<long long>(units, std::min(ctx.num_sms, kMaxSkCtas));
+    uint8_t* base = static_cast<uint8_t*>(scratch);
+    p.part_o = reinterpret_cast<uint4*>(base);
+    p.part_ml = reinterpret_cast<float2*>(base + size_t(kMaxSkCtas) * 2 * 128 * HD * 2);
+    p.flags = reinterpret_cast<unsigned long long*>(base + kSkFlagsOffset);
+    p.seq = next_scratch_seq();
+  }
+  if (grid > 0x7fffffffll) return set_error(-1, "attention: %lld units", units);
+  kernel<<<static_cast<unsigned>(grid), 384, Cfg::kSmem, stream>>>(tm, p);
+  return check_launch("attention");
+}
+
 template <int HD>
 int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, void* scratch,
               size_t scratch_bytes, cudaStream_t stream) {
@@ -597,14 +1163,26 @@ int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, v
 
 }  // namespace
 
+std::atomic<int> g_attn_variant{0};
+
+int set_attention_variant(int v) {
+  if (v < 0 || v > 2) return -1;
+  g_attn_variant.store(v);
+  return 0;
+}
+
 int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_heads,
                      int head_dim, bf16* out, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream) {
   if (n_tokens <= 0) return 0;
+  // two query tiles per CTA unless the one-tile form is asked for
+  const bool two = g_attn_variant.load(std::memory_order_relaxed) != 1;
   if (head_dim == 128)
-    return launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+    return two ? launch_hd2<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
+               : launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
   if (head_dim == 64)
-    return launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+    return two ? launch_hd2<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
+               : launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
   return set_error(-1, "attention: head_dim %d unsupported (64 or 128)", head_dim);
 }
 

@@ -215,21 +215,27 @@ struct StatAcc {
   float k, s1, s2;
 };
 
-// Add 32 stored values (16 packed bf16 pairs) of this lane's row; `first` marks the
-// tile's first chunk, whose first value becomes the shift.
-__device__ __forceinline__ void stat_add(StatAcc& a, const uint32_t (&pk)[16], bool first) {
+// Add 32 output values of this lane's row (the fp32 values the bf16 output rounds: the
+// statistics then describe the residual before its storage rounding, as the LayerNorm of
+// the unrounded sum would); `first` marks the tile's first chunk, whose first value
+// becomes the shift.  Two independent partial sums keep the dependency chains short.
+__device__ __forceinline__ void stat_add(StatAcc& a, const float (&v)[32], bool first) {
   if (first) {
-    a.k = __uint_as_float(pk[0] << 16);
+    a.k = v[0];
     a.s1 = 0.f;
     a.s2 = 0.f;
   }
+  float s1a = 0.f, s1b = 0.f, s2a = 0.f, s2b = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float lo = __uint_as_float(pk[i] << 16) - a.k;
-    const float hi = __uint_as_float(pk[i] & 0xFFFF0000u) - a.k;
-    a.s1 += lo + hi;
-    a.s2 = fmaf(lo, lo, fmaf(hi, hi, a.s2));
+    const float x0 = v[2 * i] - a.k, x1 = v[2 * i + 1] - a.k;
+    s1a += x0;
+    s1b += x1;
+    s2a = fmaf(x0, x0, s2a);
+    s2b = fmaf(x1, x1, s2b);
   }
+  a.s1 += s1a + s1b;
+  a.s2 += s2a + s2b;
 }
 
 // The tile row's group statistics (mean, M2) over its 256 columns.
@@ -260,6 +266,19 @@ __device__ __forceinline__ void load_row_in(const GemmEpilogue& e, int row, int 
       for (int i = 0; i < 8; ++i) in.cs[i] = __ldg(cs + i);
     }
   }
+}
+
+// The per-row scalars an epilogue row needs (LN-folded kinds: the merged statistics; int8
+// kinds: the activation row scale), read before the accumulator is ready so that their
+// latency overlaps the tile's MMAs.
+template <int EPI>
+__device__ __forceinline__ LnRow row_scalars(const GemmEpilogue& e, int row, bool valid) {
+  LnRow ln{0.f, 1.f};
+  if constexpr (epi_ln_fold(EPI)) {
+    if (valid) ln = ln_row(e, row);
+  }
+  if constexpr (epi_int8(EPI)) ln.rs = valid ? __ldg(e.row_scale + row) : 0.f;
+  return ln;
 }
 
 // a[i] for i in 0..3 without indexing a register array by a runtime value.
@@ -422,7 +441,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmEpilogue& e, int row, i
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
   if constexpr (EPI == kEpiGateResid || EPI == kEpiBias) {
-    if (sa != nullptr) stat_add(*sa, pk, first);
+    if (sa != nullptr) stat_add(*sa, v, first);
   }
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -475,19 +494,15 @@ __device__ __forceinline__ void add_part(uint32_t (&r)[32], const uint4 (&part)[
 template <int BN, bool INT8, int EPI>
 __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbase, int row,
                                               int row_in_tile, int col0, int src_lo,
-                                              int src_hi, int stride, int off) {
+                                              int src_hi, int stride, int off, LnRow ln_in) {
   constexpr int NC = BN / 32;
   const bool valid = row < p.M;
   const bool has_part = src_lo < src_hi;
   const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
-  LnRow ln{0.f, 1.f};
-  if constexpr (epi_ln_fold(EPI)) {
-    if (valid) ln = ln_row(p.epi, row);
-  }
+  LnRow ln = ln_in;
   StatAcc sa{0.f, 0.f, 0.f};
   const bool want_stats =
       (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
-  if constexpr (epi_int8(EPI)) ln.rs = valid ? __ldg(p.epi.row_scale + row) : 0.f;
   float qks[4] = {1.f, 1.f, 1.f, 1.f};
   if constexpr (epi_base(EPI) == kEpiRope) {
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
@@ -785,7 +800,7 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
   if constexpr (EPI == kEpiGateResid || EPI == kEpiBias) {
-    if (sa != nullptr) stat_add(*sa, pk, first);
+    if (sa != nullptr) stat_add(*sa, v, first);
   }
   __syncwarp();
 #pragma unroll
@@ -811,19 +826,14 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
                                                    int row0, int row_in_tile, int col0,
                                                    int src_lo, int src_hi, int stride,
                                                    int off, uint4* blk, const float* vec,
-                                                   int lane) {
+                                                   int lane, LnRow ln) {
   constexpr int NC = BN / 32;
   const int nrows = p.M - row0;
   const bool has_part = src_lo < src_hi;
   const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
-  LnRow ln{0.f, 1.f};
-  if constexpr (epi_ln_fold(EPI)) {
-    if (lane < nrows) ln = ln_row(p.epi, row0 + lane);
-  }
   StatAcc sa{0.f, 0.f, 0.f};
   const bool want_stats =
       (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
-  if constexpr (epi_int8(EPI)) ln.rs = lane < nrows ? __ldg(p.epi.row_scale + row0 + lane) : 0.f;
   float qks[4] = {1.f, 1.f, 1.f, 1.f};
   if constexpr (epi_base(EPI) == kEpiRope) {
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
@@ -1047,11 +1057,12 @@ __global__ void __launch_bounds__(192, 1)
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int row = mb * kBM + row_in_tile;
+      const LnRow ln_pre = row_scalars<EPI>(p.epi, row, row < p.M);
       bool ok = wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int row = mb * kBM + row_in_tile;
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
       if (kb1 < p.k_blocks) {
         // stream-K contributor: park the partial tile in this CTA's slot
@@ -1087,7 +1098,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       epilogue_unit<BN, INT8, EPI>(p, tbase, row, row_in_tile, nb * BN, c_lo,
-                                   static_cast<int>(blockIdx.x), 1, 0);
+                                   static_cast<int>(blockIdx.x), 1, 0, ln_pre);
       // hand the consumed flags back at zero, so a replay of this launch (same sequence
       // value, e.g. from a CUDA graph) waits for its own contributors again
       __syncwarp();
@@ -1298,6 +1309,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                                vec, lane);
       else
         stage_vectors<EPI, BN>(p.epi, nb * BN, vec, lane);
+      const int row_pre = mb * 256 + static_cast<int>(rank) * 128 + row_in_tile;
+      const LnRow ln_pre = row_scalars<EPI>(p.epi, row_pre, !TRANS && row_pre < p.M);
       bool ok = wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -1345,7 +1358,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                                      quarter * 32, nb * BN, blk, vec);
       else
         epilogue_unit_pair<BN, INT8, EPI>(p, tbase, row - lane, row_in_tile, nb * BN, c_lo,
-                                          pair, 2, static_cast<int>(rank), blk, vec, lane);
+                                          pair, 2, static_cast<int>(rank), blk, vec, lane,
+                                          ln_pre);
       __syncwarp();
       if (lane == 0)
         for (int src = c_lo; src < pair; ++src)

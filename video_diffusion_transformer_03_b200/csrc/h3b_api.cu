@@ -702,6 +702,12 @@ int h3b_set_gemm_override(int tile, int sched, int trans) {
   return H3B_OK;
 }
 
+int h3b_set_attention_variant(int variant) {
+  if (set_attention_variant(variant))
+    return set_error(H3B_EINVAL, "set_attention_variant: %d (0, 1 or 2)", variant);
+  return H3B_OK;
+}
+
 size_t h3b_workspace_size(const h3b_dims* dims, int n_tokens) {
   if (check_dims(dims) || n_tokens < 0) return 0;
   return arena_bytes(dims, n_tokens);

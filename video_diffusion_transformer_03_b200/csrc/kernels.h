@@ -145,6 +145,10 @@ int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_hea
                      int head_dim, bf16* out, void* scratch, size_t scratch_bytes,
                      cudaStream_t stream);
 
+// Attention form for later launches: 0 automatic (two query tiles per CTA), 1 one tile,
+// 2 two tiles; -1 on a bad value.
+int set_attention_variant(int v);
+
 // ---------------------------------------------------------------- row kernels
 int launch_ln_modulate(const bf16* x, int n, int d, float eps, const float* shift,
                        const float* scale, bf16* h, cudaStream_t stream);

@@ -74,6 +74,7 @@ _SIGS = {
     "h3b_denoise_workspace_size": (_SZ, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I]),
     "h3b_gemm_schedule": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int), _I]),
     "h3b_set_gemm_override": (_I, [_I, _I, _I]),
+    "h3b_set_attention_variant": (_I, [_I]),
     "h3b_adaln_modulation": (_I, [_P, _P, _P, _I, _I, _P, _P]),
     "h3b_rope_table": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I, _P, _P]),
     "h3b_ln_modulate": (_I, [_P, _I, _I, _F, _P, _P, _P, _P]),
@@ -234,6 +235,29 @@ def set_gemm_override(tile: int = -1, sched: int = -1, trans: int = -1) -> None:
     """Force the GEMM tile configuration / schedule / transposed kernel for later launches
     of this process (tests and measurements); -1 restores the automatic choice."""
     _check(lib.h3b_set_gemm_override(tile, sched, trans))
+
+
+ATTN_AUTO, ATTN_ONE_TILE, ATTN_TWO_TILES = 0, 1, 2
+
+
+def set_attention_variant(variant: int) -> None:
+    """Attention form for later launches (tests and measurements)."""
+    _check(lib.h3b_set_attention_variant(variant))
+
+
+class attention_variant:
+    """Context manager around set_attention_variant that restores the automatic form."""
+
+    def __init__(self, variant: int):
+        self.variant = variant
+
+    def __enter__(self):
+        set_attention_variant(self.variant)
+        return self
+
+    def __exit__(self, *exc):
+        set_attention_variant(ATTN_AUTO)
+        return False
 
 
 class gemm_override:
