@@ -69,6 +69,8 @@ def parse_args(argv=None):
                     help="skip the secondary measurements of the other workloads")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying a CUDA graph")
+    ap.add_argument("--attn-variant", type=int, default=0,
+                    help="attention form: 0 automatic, 1 one query tile per CTA, 2 two tiles")
     ap.add_argument("--replica-check", action="store_true",
                     help="CPU only: run the replica plumbing (gloo barrier, max over ranks, "
                          "job rate) through the same launcher and print what every rank saw")
@@ -416,6 +418,86 @@ def time_gemm_widths(dev, peaks, reps=10):
     return res
 
 
+def time_reuse(cfg_name, dev, reps=10):
+    """Whole denoises under the reuse policies (host loop over the C ABI captured as one
+    CUDA graph): ms per denoise and fresh model evaluations, for whole-velocity and
+    core-residual reuse with period 2 and 3."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    from video_diffusion_transformer_03_b200.pipeline import DiTDenoiser
+    cfg = synth.CONFIGS[cfg_name]
+    model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
+    x = synth.latent_noise(cfg, device=str(dev))
+    res = {}
+    for mode in ("velocity", "core"):
+        for every in (2, 3):
+            fresh = model.run_reuse(x, every, mode)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                model.run_reuse(x, every, mode)
+            graph.replay()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            del graph
+            res[f"{mode}{every}"] = {"ms_per_denoise": e0.elapsed_time(e1) / reps,
+                                     "fresh_evaluations": fresh, "steps": cfg.steps}
+    h3b.sync_status()
+    del model
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_int8_block(dev, peaks, reps=20):
+    """One DiT block of the 512x512 workload on the int8 path (h3b_block_forward_int8)
+    against the bf16 block (h3b_block_forward), CUDA-graph replays of `reps` blocks."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b, synth
+    from video_diffusion_transformer_03_b200.pipeline import dims_of, grid_of
+    cfg = synth.CONFIGS["dit512"]
+    dims, grid = dims_of(cfg), grid_of(cfg)
+    n = cfg.n_tokens
+    p = {k: v.to(dev) for k, v in synth.block_params(cfg, 0, device=str(dev)).items()}
+    mod = torch.empty((6, cfg.d), dtype=torch.float32, device=dev)
+    h3b.adaln_modulation(p.pop("w_ada"), p.pop("b_ada"), synth.conditioning(cfg, str(dev)), mod)
+    tq, wq = h3b.quantize_block_int8(p)
+    w = h3b.make_block_weights(p)
+    cs = torch.empty((n, cfg.head_dim // 2, 2), dtype=torch.float32, device=dev)
+    h3b.rope_table(dims, grid, False, cs)
+    x = synth.latent_noise(cfg, device=str(dev)).to(torch.bfloat16)
+    h = torch.empty_like(x)
+    ws8 = h3b.workspace(h3b.workspace_size_int8(dims, n), dev)
+    ws = h3b.workspace(h3b.workspace_size(dims, n), dev)
+    forms = {"int8": lambda: h3b.block_forward_int8(dims, w, wq, mod, cs, x, ws8),
+             "bf16": lambda: h3b.block_forward(dims, w, mod, mod, cs, x, h, ws, True)}
+    res = {}
+    for name, fn in forms.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(reps):
+                fn()
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        del graph
+        res[name + "_block_us"] = e0.elapsed_time(e1) / reps * 1e3
+    h3b.sync_status()
+    del p, tq, x, ws8, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_attention_forms(dev, peaks, reps=10):
     """Attention alone at the 512x512 (1,600 tokens) and 768x1344 (11,344 tokens) shapes,
     24 heads x 128, split schedule, in both kernel forms (one or two query tiles per CTA);
@@ -463,7 +545,8 @@ def time_denoise(cfg_name, dev, reps, warm=1):
     cfg = synth.CONFIGS[cfg_name]
     model = DiTDenoiser(cfg, device=str(dev), gen_device=str(dev))
     counts, _ = workload_counts(cfg, model.active)
-    x = synth.latent_noise(cfg, device=str(dev))
+    x = (synth.latent_state(cfg, device=str(dev)) if cfg.latent_channels
+         else synth.latent_noise(cfg, device=str(dev)))
     for _ in range(warm):
         model.run(x)
     graph = model.capture(x)
@@ -623,6 +706,8 @@ def run_gpu(args):
     barrier, max_over_ranks = replicas.barrier, replicas.max
 
     peaks, peak_src = load_peaks()
+    if args.attn_variant:
+        h3b.set_attention_variant(args.attn_variant)
     if args.kernel in ("fc2_int8_row", "token_pairing"):  # workloads outside the block
         res = (time_int8_fc2(dev, peaks, reps=args.reps) if args.kernel == "fc2_int8_row"
                else time_token_pairing(dev, peaks, reps=args.reps))
@@ -747,9 +832,12 @@ def run_gpu(args):
         del graph
         graph = None
         also = {}
-        for name, reps in (("dit512_tokred", 20), ("dit768x1344", 2)):
+        for name, reps in (("dit512_tokred", 20), ("dit768x1344", 2), ("dit512_latent", 20),
+                           ("dit512_qknorm", 20)):
             if name != args.config:
                 also[name] = time_denoise(name, dev, reps)
+        also["reuse_dit512"] = time_reuse("dit512", dev)
+        also["int8_block_dit512"] = time_int8_block(dev, peaks)
         also["attention_forms"] = time_attention_forms(dev, peaks)
         also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
