@@ -623,8 +623,9 @@ def block_forward_int8(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int, spli
     FC1 inputs (the AdaLN outputs) quantised per token row, the FC2 input (the GELU
     output) per token and per `group` channels, weights per output channel
     (w["w_qkv_q"], w["s_qkv"], ...: quantize_rows of the bf16 weights); the attention and
-    the output projection stay bf16.  The quantisation acts on fp32 values of the
-    activations (the GPU quantises its fp32 epilogue values)."""
+    the output projection stay bf16.  The QKV and FC1 inputs are quantised from fp32 values
+    (in the LayerNorm kernel, before any storage); the FC2 input from the stored bf16 GELU
+    output."""
     x = np.asarray(x, dt)
     mod = np.asarray(mod, dt)
     n, d = x.shape
@@ -646,6 +647,8 @@ def block_forward_int8(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int, spli
     h2 = modulate(layer_norm(x1, eps, dt), mod[3], mod[4], dt)
     g = gelu_tanh(int8_linear_rows(h2.astype(np.float32), w["w_fc1_q"], w["s_fc1"],
                                    np.asarray(w["b_fc1"], dt), dt), dt)
-    qg, sg = quantize_groups(g.astype(np.float32), group)
+    # the FC2 input is quantised as it is stored, in bf16 (the activations of the int8
+    # FC2 workload are bf16 too)
+    qg, sg = quantize_groups(round_to_bf16(g), group)
     y = int8_grouped_matmul(qg, sg, w["w_fc2_q"], w["s_fc2"], group, dt) + np.asarray(w["b_fc2"], dt)
     return gated_residual(x1, mod[5], y, dt)
