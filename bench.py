@@ -511,7 +511,8 @@ def time_attention_forms(dev, peaks, reps=10):
         d = 24 * 128
         qkv = torch.randn(n, 3 * d, generator=g, device=dev).to(torch.bfloat16)
         out = torch.empty(n, d, dtype=torch.bfloat16, device=dev)
-        for name, v in (("two_tile", h3b.ATTN_TWO_TILES), ("one_tile", h3b.ATTN_ONE_TILE)):
+        for name, v in (("two_tile", h3b.ATTN_TWO_TILES), ("one_tile", h3b.ATTN_ONE_TILE),
+                        ("two_tile_poly", h3b.ATTN_TWO_TILES_POLY)):
             with h3b.attention_variant(v):
                 for _ in range(3):
                     h3b.attention(qkv, 24, 128, out, ws=ws)

@@ -187,8 +187,9 @@ int h3b_set_gemm_override(int tile, int sched, int trans);
 
 /* Select the attention kernel's form for later launches of this process, for tests and
  * measurements: 0 automatic (the default: two 128-query tiles per CTA sharing each K/V
- * tile, one softmax warpgroup each), 1 one query tile per CTA, 2 two tiles.  Returns
- * H3B_OK or H3B_EINVAL. */
+ * tile, one softmax warpgroup each), 1 one query tile per CTA, 2 two tiles, 3 two tiles
+ * with a quarter of the exponentials on the FMA pipe (a cubic on the reduced argument)
+ * instead of the MUFU unit.  Returns H3B_OK or H3B_EINVAL. */
 int h3b_set_attention_variant(int variant);
 
 /* ---------------------------------------------------------------- hot-path steps */

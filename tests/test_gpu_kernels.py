@@ -246,8 +246,9 @@ def _attention_want(qkv, n, heads, hd):
     return O.attention(q, k, v).reshape(n, d)
 
 
-@pytest.mark.parametrize("variant", [h3b.ATTN_TWO_TILES, h3b.ATTN_ONE_TILE],
-                         ids=["two-tile", "one-tile"])
+@pytest.mark.parametrize("variant", [h3b.ATTN_TWO_TILES, h3b.ATTN_ONE_TILE,
+                                     h3b.ATTN_TWO_TILES_POLY],
+                         ids=["two-tile", "one-tile", "two-tile-poly"])
 @pytest.mark.parametrize("split", [False, True], ids=["per-unit", "split"])
 @pytest.mark.parametrize("n,heads,hd,std", ATTN_CASES)
 def test_attention(n, heads, hd, std, split, variant):

@@ -553,9 +553,9 @@ __global__ void __launch_bounds__(192, 1)
 // load, each with its own softmax warpgroup, so the two softmax streams overlap each
 // other and the tensor core (one softmax warpgroup per CTA was the critical path).
 // Roles (384 threads, three warpgroups):
-//   warpgroup 0  warp 0 TMA producer, warp 1 MMA issuer, warps 2-3 idle (88 registers);
-//   warpgroup 1  softmax of query tile 0 (rows 0-127 of the unit), 208 registers;
-//   warpgroup 2  softmax of query tile 1 (rows 128-255), 208 registers (the split adds up
+//   warpgroup 0  warp 0 TMA producer, warp 1 MMA issuer, warps 2-3 idle (104 registers);
+//   warpgroup 1  softmax of query tile 0 (rows 0-127 of the unit), 200 registers;
+//   warpgroup 2  softmax of query tile 1 (rows 128-255), 200 registers (the split adds up
 //                to the 384 x 168 registers the CTA is launched with).
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512): one score buffer per tile,
 // so S_j+1 of a tile is computed as soon as its softmax has read S_j into registers.
@@ -567,6 +567,22 @@ __global__ void __launch_bounds__(192, 1)
 // the one-tile form, with the parked running state of both tiles (O in bf16, (max, sum)
 // in fp32).
 constexpr int kRing = 3;
+
+// 2^x on the FMA and integer pipes (the MUFU unit has 16 results per clock per SM and is
+// shared by both softmax warpgroups): x = n + f with n the nearest integer (added to
+// 1.5 * 2^23, x's integer part lands in the low mantissa bits) and f in [-0.5, 0.5];
+// 2^f from a cubic fitted to minimise the relative error on that interval (Remez
+// exchange; max relative error 7.5e-5, below the 2^-9 of the bf16 P it feeds); 2^n added
+// to the exponent field.  x is clamped to -125 so the result stays normal.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.05517166853f, f, 0.24261112511f), f, 0.69326096773f), f,
+                       0.99992805719f);
+  return __int_as_float(__float_as_int(p) + static_cast<int>(static_cast<unsigned>(n) << 23));
+}
 
 template <int HD>
 struct Attn2Cfg {
@@ -613,7 +629,8 @@ __device__ __forceinline__ bool tile1_valid(const Attn2Params& p, int unit) {
   return (unit % p.n_qb) * 256 + 128 < p.n;
 }
 
-template <int HD>
+// POLY: every fourth exponential of a score row on the FMA pipe (exp2_poly).
+template <int HD, bool POLY>
 __global__ void __launch_bounds__(384, 1)
     k_attention_tc2(const __grid_constant__ CUtensorMap tm, const Attn2Params p) {
   using Cfg = Attn2Cfg<HD>;
@@ -676,7 +693,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    regs_dealloc<88>();
+    regs_dealloc<104>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------------ producer
       // Loads in the MMA's consumption order: per step t, K(t) then V(t - 1), except at a
@@ -855,7 +872,7 @@ __global__ void __launch_bounds__(384, 1)
       drain_wait(drain, 0);
     }
   } else {
-    regs_alloc<208>();
+    regs_alloc<200>();
     // ------------------------------------------------------------------ softmax (tile w)
     const int w = (warp - 4) >> 2;
     const int quarter = warp & 3;
@@ -904,35 +921,22 @@ __global__ void __launch_bounds__(384, 1)
         const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]),
                               fmaxf(m8[6], m8[7]));
         const float mxs = mx * sl2;
+        // lazy rescale: the running max moves only when the tile max exceeds it by more
+        // than 8; O is rescaled below, once the scores are dead (after P is stored)
+        float alpha = 1.0f;
+        bool need = false;
         if (j == j0) {
           m_used = mxs;
-        } else {
-          const bool need = mxs > m_used + 8.0f;
-          if (__any_sync(0xffffffffu, need)) {
-            // O must hold every earlier P V product of this unit before it is rescaled
-            ok = __all_sync(0xffffffffu, wait_bar(&p_free[w], static_cast<uint32_t>(c - 1) & 1u,
-                                                  abort_flag, p.err, kErrAttnWait));
-            if (!ok) break;
-            tc_fence_after();
-            const float alpha = need ? ex2_approx(m_used - mxs) : 1.0f;
-#pragma unroll
-            for (int cc = 0; cc < HD / 32; ++cc) {
-              uint32_t r[32];
-              tmem_ld32(o_addr + cc * 32, r);
-              tmem_wait_ld(r);
-#pragma unroll
-              for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
-              tmem_st32(o_addr + cc * 32, r);
-            }
-            tmem_wait_st();
-            l *= alpha;
-            if (need) m_used = mxs;
-          }
+        } else if (mxs > m_used + 8.0f) {
+          need = true;
+          alpha = ex2_approx(m_used - mxs);
+          m_used = mxs;
         }
         float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int q = 0; q < 128; ++q) {
-          const float e = ex2_approx(fmaf(s[q], sl2, -m_used));
+          const float x = fmaf(s[q], sl2, -m_used);
+          const float e = (POLY && (q & 3) == 3) ? exp2_poly(x) : ex2_approx(x);
           sum8[q & 7] += e;
           s[q] = e;
         }
@@ -940,8 +944,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 4; i > 0; i >>= 1)
 #pragma unroll
           for (int q = 0; q < i; ++q) sum8[q] += sum8[q + i];
-        l += sum8[0];
-        if (c >= 1) {  // the tile's P buffer is free once its previous P V has completed
+        l = fmaf(l, alpha, sum8[0]);
+        if (c >= 1) {
+          // the tile's P buffer is free, and O complete, once its previous P V has finished
           ok = __all_sync(0xffffffffu, wait_bar(&p_free[w], static_cast<uint32_t>(c - 1) & 1u,
                                                 abort_flag, p.err, kErrAttnWait));
           if (!ok) break;
@@ -955,6 +960,21 @@ __global__ void __launch_bounds__(384, 1)
           u.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
           const int chunk = (c16 & 7) ^ (row & 7);
           *reinterpret_cast<uint4*>(pbuf + (c16 >> 3) * kBox + chunk * 16) = u;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds every earlier P V product of the unit (the wait above) and the next one
+          // is not released yet: scale it to the new running max
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < HD / 32; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(o_addr + cc * 32, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+            tmem_st32(o_addr + cc * 32, r);
+          }
+          tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1066,7 +1086,7 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int HD>
+template <int HD, bool POLY>
 int launch_hd2(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, void* scratch,
                size_t scratch_bytes, cudaStream_t stream) {
   using Cfg = Attn2Cfg<HD>;
@@ -1075,7 +1095,7 @@ int launch_hd2(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, 
   if (!make_tmap_2d(&tm, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint64_t(n), uint64_t(3 * d),
                     uint64_t(3 * d) * 2, 128, 64))
     return set_error(-3, "attention: cuTensorMapEncodeTiled failed (n=%d d=%d)", n, d);
-  auto kernel = k_attention_tc2<HD>;
+  auto kernel = k_attention_tc2<HD, POLY>;
   static std::atomic<uint32_t> attr_done{0};
   const uint32_t bit = 1u << (ctx.device & 31);
   if (!(attr_done.load() & bit)) {
@@ -1166,7 +1186,7 @@ int launch_hd(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, v
 std::atomic<int> g_attn_variant{0};
 
 int set_attention_variant(int v) {
-  if (v < 0 || v > 2) return -1;
+  if (v < 0 || v > 3) return -1;
   g_attn_variant.store(v);
   return 0;
 }
@@ -1176,13 +1196,18 @@ int launch_attention(const DevCtx& ctx, const bf16* qkv, int n_tokens, int n_hea
                      cudaStream_t stream) {
   if (n_tokens <= 0) return 0;
   // two query tiles per CTA unless the one-tile form is asked for
-  const bool two = g_attn_variant.load(std::memory_order_relaxed) != 1;
-  if (head_dim == 128)
-    return two ? launch_hd2<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
-               : launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
-  if (head_dim == 64)
-    return two ? launch_hd2<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
-               : launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+  const int v = g_attn_variant.load(std::memory_order_relaxed);
+  const bool poly = v == 3;
+  if (head_dim == 128) {
+    if (v == 1) return launch_hd<128>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+    return poly ? launch_hd2<128, true>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
+                : launch_hd2<128, false>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+  }
+  if (head_dim == 64) {
+    if (v == 1) return launch_hd<64>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+    return poly ? launch_hd2<64, true>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream)
+                : launch_hd2<64, false>(ctx, qkv, n_tokens, n_heads, out, scratch, scratch_bytes, stream);
+  }
   return set_error(-1, "attention: head_dim %d unsupported (64 or 128)", head_dim);
 }
 

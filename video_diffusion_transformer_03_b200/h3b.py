@@ -237,7 +237,7 @@ def set_gemm_override(tile: int = -1, sched: int = -1, trans: int = -1) -> None:
     _check(lib.h3b_set_gemm_override(tile, sched, trans))
 
 
-ATTN_AUTO, ATTN_ONE_TILE, ATTN_TWO_TILES = 0, 1, 2
+ATTN_AUTO, ATTN_ONE_TILE, ATTN_TWO_TILES, ATTN_TWO_TILES_POLY = 0, 1, 2, 3
 
 
 def set_attention_variant(variant: int) -> None:
