@@ -644,6 +644,10 @@ def block_forward_int8(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int, spli
     q = rope_rotate(q, np.asarray(pos)[sel], split, theta, dt)
     o = attention(q, k, v, dt=dt).reshape(len(sel), d)
     x1 = gated_residual(x[sel], mod[2], o @ np.asarray(w["w_o"], dt).T + np.asarray(w["b_o"], dt), dt)
+    # the residual is stored in bf16 between the two halves ([dothoosh] "DiT fusions and
+    # memory management": the bf16-rounded residual feeds the MLP's AdaLN); the FC1 input
+    # codes are decided on the LayerNorm of that stored value
+    x1 = round_to_bf16(x1).astype(dt)
     h2 = modulate(layer_norm(x1, eps, dt), mod[3], mod[4], dt)
     g = gelu_tanh(int8_linear_rows(h2.astype(np.float32), w["w_fc1_q"], w["s_fc1"],
                                    np.asarray(w["b_fc1"], dt), dt), dt)
