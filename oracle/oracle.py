@@ -646,9 +646,10 @@ def block_forward_int8(x, w: Dict[str, np.ndarray], mod, pos, n_heads: int, spli
     x1 = gated_residual(x[sel], mod[2], o @ np.asarray(w["w_o"], dt).T + np.asarray(w["b_o"], dt), dt)
     # the residual is stored in bf16 between the two halves ([dothoosh] "DiT fusions and
     # memory management": the bf16-rounded residual feeds the MLP's AdaLN); the FC1 input
-    # codes are decided on the LayerNorm of that stored value
-    x1 = round_to_bf16(x1).astype(dt)
-    h2 = modulate(layer_norm(x1, eps, dt), mod[3], mod[4], dt)
+    # codes are decided on the LayerNorm of that stored value.  The gated residual add
+    # keeps x1 itself, so zero gates still give the identity on any input.
+    x1_stored = round_to_bf16(x1).astype(dt)
+    h2 = modulate(layer_norm(x1_stored, eps, dt), mod[3], mod[4], dt)
     g = gelu_tanh(int8_linear_rows(h2.astype(np.float32), w["w_fc1_q"], w["s_fc1"],
                                    np.asarray(w["b_fc1"], dt), dt), dt)
     # the FC2 input is quantised as it is stored, in bf16 (the activations of the int8
