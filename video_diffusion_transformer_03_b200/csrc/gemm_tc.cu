@@ -307,10 +307,14 @@ __device__ __forceinline__ void qk_rms_pass_global(const GemmEpilogue& e, uint32
     if constexpr (epi_int8(EPI)) {
       float cs[32], b[32];
       load_f32x32(e.col_scale + col, cs);
-      if (e.bias_f32)
+      if (e.bias_f32) {
         load_f32x32(e.bias_f32 + col, b);
-      else
+      } else if (e.bias) {
         load_bf16x32(e.bias + col, b);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) b[j] = 0.0f;
+      }
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), ln.rs), cs[j]) +
@@ -712,7 +716,7 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
     for (int j = 0; j < 32; ++j)
       v[j] = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), rs),
                        vec[kVecScale + j]);
-    if (e.bias_f32) {
+    if (e.bias_f32 || e.bias) {  // staged as fp32 from either form
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += vec[kVecBias + j];
     }
