@@ -553,19 +553,27 @@ __global__ void __launch_bounds__(192, 1)
 // load, each with its own softmax warpgroup, so the two softmax streams overlap each
 // other and the tensor core (one softmax warpgroup per CTA was the critical path).
 // Roles (384 threads, three warpgroups):
-//   warpgroup 0  warp 0 TMA producer, warp 1 MMA issuer, warps 2-3 idle (104 registers);
-//   warpgroup 1  softmax of query tile 0 (rows 0-127 of the unit), 200 registers;
-//   warpgroup 2  softmax of query tile 1 (rows 128-255), 200 registers (the split adds up
-//                to the 384 x 168 registers the CTA is launched with).
+//   warpgroup 0  warp 0 TMA producer; warps 1 and 2 MMA issuers of query tiles 0 and 1
+//                (one thread each, on different SMSPs); warp 3 idle;
+//   warpgroup 1  softmax of query tile 0 (rows 0-127 of the unit);
+//   warpgroup 2  softmax of query tile 1 (rows 128-255).
+// The softmax fits the 168 registers a thread is launched with; the polynomial-exp2 form
+// needs more and moves registers from warpgroup 0 (104) to the softmax (200), which adds
+// up to the 384 x 168 of the launch.
+// The tensor pipe keeps almost nothing queued behind the MMA it is executing, so any time
+// an issuing thread spends between two MMAs (barrier waits, fences, commits, address
+// arithmetic) leaves it idle: each 8-step product is issued from one asm block, and two
+// issuers, one per tile, keep the pipe fed while either of them waits.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512): one score buffer per tile,
 // so S_j+1 of a tile is computed as soon as its softmax has read S_j into registers.
 // Shared memory: Q0, Q1, P0, P1 and a 3-slot ring of K/V tiles loaded in the order the
-// tensor core consumes them (K_j+1 before V_j).  Per step the MMA thread issues S0, S1 of
-// key tile j, then O0 += P0 V, O1 += P1 V of key tile j - 1 (at a unit's first step, the
-// previous unit's last P V goes first).  A query block whose second tile starts past the
-// last token skips that tile (its MMAs and its softmax).  The split schedule is that of
-// the one-tile form, with the parked running state of both tiles (O in bf16, (max, sum)
-// in fp32).
+// tensor core consumes them (K_j+1 before V_j); both issuers release every slot (the empty
+// barriers count two arrivals).  Per step an issuer issues S of key tile j, then O += P V of
+// key tile j - 1 (at a unit's first step, the previous unit's last P V goes first).  A
+// query block whose second tile starts past the last token skips that tile (its MMAs and
+// its softmax).  The split schedule is that of the one-tile form, with the parked running
+// state of both tiles (O in bf16, (max, sum) in fp32).
+
 constexpr int kRing = 3;
 
 // 2^x on the FMA and integer pipes (the MUFU unit has 16 results per clock per SM and is
@@ -655,8 +663,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = bars + 12;   // [2]
   uint64_t* p_free = bars + 14;   // [2]
   uint64_t* o_empty = bars + 16;  // [2]
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* drain = bars + 18;    // [2 issuers]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -666,10 +674,10 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, 2);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
@@ -678,7 +686,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&p_free[w], 1);
       mbar_init(&o_empty[w], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -693,7 +702,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    regs_dealloc<104>();
+    if constexpr (POLY) regs_dealloc<104>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------------ producer
       // Loads in the MMA's consumption order: per step t, K(t) then V(t - 1), except at a
@@ -766,19 +775,31 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < kRing; ++s)
           if (armed[s] >= 0) drain_wait(&kv_full[s], static_cast<uint32_t>(armed[s]));
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
+      // ------------------------------------------------------------------ MMA issuers
+      // Warp 1 issues tile 0's products, warp 2 tile 1's (different SMSPs): each walks the
+      // same steps and ring slots, so while one thread waits on a barrier the other feeds
+      // the tensor pipe, and neither tile's chain waits on the other's.  Both commit every
+      // ring slot and the Q buffer (their empty barriers count two arrivals).
+      const int w = warp - 1;
       int slot = 0;
       uint32_t ring_phase = 0;
-      int cnt[2] = {0, 0};    // S products issued per tile (= P V products, one behind)
-      int pvc[2] = {0, 0};    // P V products issued per tile
-      int units_done[2] = {0, 0};
+      int cnt = 0;         // S products issued for this tile (P V products run one behind)
+      int pvc = 0;         // P V products issued
+      int units_done = 0;  // units whose last P V was issued (tile present)
       int ks = 0, js = 0, js0 = 0, js1 = 0, unit_s = 0;
       int kp = 0, jp = 0, jp0 = 0, jp1 = 0, unit_p = 0;
       segment2(p, rg, 0, unit_s, js0, js1);
       js = js0;
       segment2(p, rg, 0, unit_p, jp0, jp1);
       jp = jp0;
+      // (pinned here: hoisted above the role split they would stay live through the softmax)
+      const uint64_t q_desc = opaque_u64(sdesc_sw128(smem_u32(sQ + w * Cfg::kQBytes), 16, 1024));
+      const uint64_t p_desc = opaque_u64(sdesc_sw128(smem_u32(sP + w * Cfg::kPBytes), 16, 1024));
+      const uint64_t k_desc0 = opaque_u64(sdesc_sw128(smem_u32(sKV), 16, 1024));
+      const uint64_t v_desc0 = opaque_u64(sdesc_sw128(smem_u32(sKV), kBox, 1024));
+      const uint32_t s_tmem = tmem + w * 128;
+      const uint32_t o_tmem = tmem + kOCol + w * 128;
       auto ring_take = [&](int& s_out) -> bool {
         if (!wait_bar(&kv_full[slot], ring_phase, abort_flag, p.err, kErrAttnWait)) return false;
         s_out = slot;
@@ -789,28 +810,24 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       auto issue_s = [&]() -> bool {
-        const bool v1 = tile1_valid(p, unit_s);
+        const bool here = w == 0 || tile1_valid(p, unit_s);
         if (js == js0 &&
             !wait_bar(q_full, static_cast<uint32_t>(ks) & 1u, abort_flag, p.err, kErrAttnWait))
           return false;
         int ksl;
         if (!ring_take(ksl)) return false;
-        tc_fence_after();
-        const uint32_t k0 = smem_u32(sKV + ksl * Cfg::kKVBytes);
-        for (int w = 0; w < (v1 ? 2 : 1); ++w) {
-          if (cnt[w] >= 1 && !wait_bar(&s_free[w], static_cast<uint32_t>(cnt[w] - 1) & 1u,
-                                       abort_flag, p.err, kErrAttnWait))
+        if (here) {
+          if (cnt >= 1 && !wait_bar(&s_free[w], static_cast<uint32_t>(cnt - 1) & 1u,
+                                    abort_flag, p.err, kErrAttnWait))
             return false;
           tc_fence_after();
-          const uint32_t q0 = smem_u32(sQ + w * Cfg::kQBytes);
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_f16(tmem + w * 128, sdesc_sw128(q0 + off, 16, 1024),
-                     sdesc_sw128(k0 + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-          }
+          const uint64_t k_desc = k_desc0 + static_cast<uint64_t>(ksl) * (Cfg::kKVBytes >> 4);
+          if constexpr (HD == 128)
+            umma_f16_x8_kk<kBox / 16>(s_tmem, q_desc, k_desc, IDESC_S, 0u);
+          else
+            umma_f16_x4_kk(s_tmem, q_desc, k_desc, IDESC_S, 0u);
           tc_commit(&s_full[w]);
-          ++cnt[w];
+          ++cnt;
         }
         tc_commit(&kv_empty[ksl]);
         if (++js == js1) {
@@ -823,37 +840,29 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       auto issue_pv = [&]() -> bool {
-        const bool v1 = tile1_valid(p, unit_p);
+        const bool here = w == 0 || tile1_valid(p, unit_p);
         const bool first = jp == jp0;
         int vsl;
         if (!ring_take(vsl)) return false;
-        tc_fence_after();
-        const uint32_t v0 = smem_u32(sKV + vsl * Cfg::kKVBytes);
-        for (int w = 0; w < (v1 ? 2 : 1); ++w) {
+        if (here) {
           // the tile's previous unit must have read O out before it is overwritten
-          if (first && units_done[w] > 0 &&
-              !wait_bar(&o_empty[w], static_cast<uint32_t>(units_done[w] - 1) & 1u, abort_flag,
+          if (first && units_done > 0 &&
+              !wait_bar(&o_empty[w], static_cast<uint32_t>(units_done - 1) & 1u, abort_flag,
                         p.err, kErrAttnWait))
             return false;
-          if (!wait_bar(&p_full[w], static_cast<uint32_t>(pvc[w]) & 1u, abort_flag, p.err,
+          if (!wait_bar(&p_full[w], static_cast<uint32_t>(pvc) & 1u, abort_flag, p.err,
                         kErrAttnWait))
             return false;
           tc_fence_after();
-          const uint32_t p0 = smem_u32(sP + w * Cfg::kPBytes);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t poff = (kk >> 2) * kBox + (kk & 3) * 32;
-            umma_f16(tmem + kOCol + w * 128, sdesc_sw128(p0 + poff, 16, 1024),
-                     sdesc_sw128(v0 + kk * 2048, kBox, 1024), IDESC_PV,
-                     (!first || kk > 0) ? 1u : 0u);
-          }
+          umma_f16_x8_kmn<kBox / 16>(
+              o_tmem, p_desc, v_desc0 + static_cast<uint64_t>(vsl) * (Cfg::kKVBytes >> 4),
+              IDESC_PV, first ? 0u : 1u);
           tc_commit(&p_free[w]);
-          ++pvc[w];
+          ++pvc;
         }
         tc_commit(&kv_empty[vsl]);
         if (++jp == jp1) {
-          units_done[0] += 1;
-          if (v1) units_done[1] += 1;
+          if (here) ++units_done;
           if (++kp < n_seg) {
             segment2(p, rg, kp, unit_p, jp0, jp1);
             jp = jp0;
@@ -868,11 +877,11 @@ __global__ void __launch_bounds__(384, 1)
         if (t < total && !issue_s()) break;
         if (t >= 1 && !pv_first && !issue_pv()) break;
       }
-      tc_commit(drain);
-      drain_wait(drain, 0);
+      tc_commit(&drain[w]);
+      drain_wait(&drain[w], 0);
     }
   } else {
-    regs_alloc<200>();
+    if constexpr (POLY) regs_alloc<200>();
     // ------------------------------------------------------------------ softmax (tile w)
     const int w = (warp - 4) >> 2;
     const int quarter = warp & 3;
