@@ -1248,10 +1248,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------------- MMA issuer (even CTA)
+      // Each stage's four K steps are issued from one asm block: the tensor pipe queues
+      // little behind the MMA it executes, so instructions between MMAs can idle it.
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int local = 0;
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 16, 1024);
       Sched sc;
       sched_init(p, sc, pair, npairs);
       int tile, kb0, kb1;
@@ -1267,18 +1271,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * HA);
-          const uint32_t b0 = smem_u32(sB + stage * HB);
-#pragma unroll
-          for (int k = 0; k < K_STEPS; ++k) {
-            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
-            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
-            if constexpr (INT8)
-              umma_i8_pair(d_tmem, ad, bd, IDESC, acc);
-            else
-              umma_f16_pair(d_tmem, ad, bd, IDESC, acc);
-          }
+          static_assert(K_STEPS == 4, "one stage is four K steps of 32 bytes");
+          umma_pair_x4<INT8>(d_tmem, a_desc0 + static_cast<uint64_t>(stage) * (HA >> 4),
+                             b_desc0 + static_cast<uint64_t>(stage) * (HB >> 4), IDESC,
+                             kb > kb0 ? 1u : 0u);
           tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
