@@ -668,7 +668,7 @@ __device__ __forceinline__ void qk_rms_pass(const GemmEpilogue& e, uint32_t tbas
                                             float (&qks)[4]) {
   float ss[4] = {0.f, 0.f, 0.f, 0.f};
   const int cpd = e.head_dim >> 5;  // chunks per head
-#pragma unroll
+#pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
@@ -843,6 +843,9 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
       qk_rms_pass<BN, EPI>(p.epi, tbase, vec, ln, qks);
   }
+  // The chunk loop is unrolled by two only (the double buffers alternate at even and odd
+  // chunks): fully unrolled, the epilogue of a 256-wide tile is large enough that its warps
+  // stall on instruction fetch.
   RowIn in[2];
   uint4 part[2][8];
   load_block_in<EPI>(p.epi, row0, nrows, col0, lane, in[0]);
@@ -850,7 +853,7 @@ __device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[0][i] = __ldcg(first + size_t(i) * kBM);
   }
-#pragma unroll
+#pragma unroll 2
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
