@@ -519,7 +519,7 @@ __device__ __forceinline__ void epilogue_unit(const GemmParams& p, uint32_t tbas
 #pragma unroll
     for (int i = 0; i < 8; ++i) part[0][i] = __ldcg(first + size_t(i) * kBM);
   }
-#pragma unroll
+#pragma unroll 2
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
@@ -897,7 +897,7 @@ __device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_
   float* stage = reinterpret_cast<float*>(blk);
   RowIn in[2];
   load_block_in<EPI>(p.epi, tok0, p.tokens - tok0, feat0, lane, in[0]);
-#pragma unroll
+#pragma unroll 2
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
@@ -1600,7 +1600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int nrows = p.M - row0;
       RowIn in[2];
       load_block_in<EPI>(p.epi, row0, nrows, nb * BN, lane, in[0]);
-#pragma unroll
+#pragma unroll 2
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(sum_addr + c * 32, r);
