@@ -42,13 +42,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram bytes per launch from an ncu capture, keyed by kernel; only used while the kernel
 # source still hashes to the value recorded with it.
 NCU_TRAFFIC = {
-    # ncu --set full, one launch of the dit512 shape after 3 warm-ups (profiles/)
-    "gemm_fc2_gate": {"bytes": 136698880 + 17368576, "src": "gemm_tc.cu",
-                      "src_sha": "85fffcd9e59c9ba3"},
-    "gemm_out_gate": {"bytes": 38648832 + 1331968, "src": "gemm_tc.cu",
-                      "src_sha": "85fffcd9e59c9ba3"},
-    "gemm_fc1_gelu": {"bytes": 85517824 + 18561280, "src": "gemm_tc.cu",
-                      "src_sha": "85fffcd9e59c9ba3"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch, ncu --set full, the dit512
+    # shape after 3 warm-ups (`bench.py --kernel <name> --reps 3`; profiles/), valid while the
+    # kernel's source file hashes to src_sha
+    "gemm_fc1_gelu": {"bytes": 85718784 + 18778112, "src": "gemm_tc.cu",
+                      "src_sha": "00a7f8e4ade88b1c"},
+    "gemm_fc2_gate": {"bytes": 137048064 + 17270272, "src": "gemm_tc.cu",
+                      "src_sha": "00a7f8e4ade88b1c"},
+    "gemm_qkv_rope": {"bytes": 67601152 + 8299776, "src": "gemm_tc.cu",
+                      "src_sha": "00a7f8e4ade88b1c"},
+    "gemm_out_gate": {"bytes": 38612736 + 1557504, "src": "gemm_tc.cu",
+                      "src_sha": "00a7f8e4ade88b1c"},
+    "attention": {"bytes": 29564160 + 41984, "src": "attention_tc.cu",
+                  "src_sha": "e705e139b6351063"},
 }
 
 
