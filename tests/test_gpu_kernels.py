@@ -223,10 +223,13 @@ def test_gemm_rope_epilogue(grid, n_audio, heads, hd, split):
 # (tokens, heads, head_dim, q/k/v std).  With the scratch, the (head, 128-query tile)
 # units are split over one CTA per SM once there are more units than SMs: the last four
 # cases have 312, 240, 200 and 200 units (ragged key tiles, cut units merged across CTAs;
-# the 100-token case has one key tile per unit, so nothing can be cut).
+# the 100-token case has one key tile per unit, so nothing can be cut; at 1,600, 1,650 and
+# 2,900 tokens the last 256-query block of each head has one tile and the two-tile form
+# cuts the CTA ranges by work, such blocks' steps weighing 5/8 of the others).
 ATTN_CASES = [(40, 4, 64, 1.2), (1, 2, 128, 1.0), (128, 1, 128, 1.2), (129, 2, 64, 1.2),
               (300, 2, 128, 1.2), (300, 2, 128, 3.0), (700, 3, 64, 2.0), (1600, 24, 128, 1.2),
-              (300, 80, 64, 1.2), (520, 40, 128, 2.0), (100, 200, 64, 1.2)]
+              (300, 80, 64, 1.2), (520, 40, 128, 2.0), (100, 200, 64, 1.2),
+              (1650, 32, 128, 1.2), (2900, 16, 64, 1.5)]
 
 
 def _worst_unit_rel_l2(got, want, heads, hd):

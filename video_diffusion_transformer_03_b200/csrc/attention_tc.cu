@@ -606,6 +606,9 @@ struct Attn2Cfg {
 struct Attn2Params {
   int n, d, n_kv, n_qb;  // tokens, n_heads * head_dim, key tiles, 256-query blocks per head
   long long steps;       // units * n_kv
+  long long work;        // the steps weighted by their cost (see work_to_step)
+  int half_last;         // 1: the last block of each head has one query tile
+  int weighted;          // CTA ranges cut by work instead of steps
   float scale_log2;
   bf16* out;
   uint4* part_o;         // [gridDim.x][2 tiles][head_dim / 8][128] uint4 (8 bf16)
@@ -615,10 +618,37 @@ struct Attn2Params {
   uint32_t* err;
 };
 
+// Relative cost of a key-tile step of a block with two query tiles and of one whose second
+// tile is empty (the last block of each head when n % 256 is in (0, 128]): the second runs
+// one softmax warp per SMSP instead of two, which takes ~63% of the time, not half
+// (measured on B200: CTAs holding such a block finished 30% before the others).
+constexpr long long kWorkFull = 8, kWorkHalf = 5;
+
+// The first step (u * n_kv + j) whose work starts at or after work position P.
+__host__ __device__ inline long long work_to_step(const Attn2Params& p, long long P) {
+  const long long nkv = p.n_kv, h1 = p.half_last;
+  const long long per_head = (kWorkFull * (p.n_qb - h1) + kWorkHalf * h1) * nkv;
+  const long long head = P / per_head;
+  const long long r = P - head * per_head;
+  long long qb = r / (kWorkFull * nkv);
+  if (qb > p.n_qb - 1) qb = p.n_qb - 1;
+  const long long wu = (h1 && qb == p.n_qb - 1) ? kWorkHalf : kWorkFull;
+  const long long j = (r - qb * kWorkFull * nkv + wu - 1) / wu;
+  return (head * p.n_qb + qb) * nkv + j;
+}
+
+// This CTA's steps.  Cut by work where every range still holds at least n_kv steps (a unit
+// is then cut at most once, between two neighbouring CTAs), else by steps.
 __device__ __forceinline__ Range cta_range2(const Attn2Params& p) {
   Range r;
-  r.begin = p.steps * static_cast<long long>(blockIdx.x) / static_cast<long long>(gridDim.x);
-  r.end = p.steps * static_cast<long long>(blockIdx.x + 1) / static_cast<long long>(gridDim.x);
+  const long long b = blockIdx.x, g = gridDim.x;
+  if (p.weighted) {
+    r.begin = work_to_step(p, p.work * b / g);
+    r.end = work_to_step(p, p.work * (b + 1) / g);
+  } else {
+    r.begin = p.steps * b / g;
+    r.end = p.steps * (b + 1) / g;
+  }
   r.u_first = static_cast<int>(r.begin / p.n_kv);
   r.u_last = static_cast<int>((r.end - 1) / p.n_kv);
   return r;
@@ -1138,6 +1168,9 @@ int launch_hd2(const DevCtx& ctx, const bf16* qkv, int n, int heads, bf16* out, 
     p.seq = next_scratch_seq();
   }
   if (grid > 0x7fffffffll) return set_error(-1, "attention: %lld units", units);
+  p.half_last = (n % 256 != 0 && n % 256 <= 128) ? 1 : 0;
+  p.work = (kWorkFull * (p.n_qb - p.half_last) + kWorkHalf * p.half_last) * heads * p.n_kv;
+  p.weighted = p.half_last && p.work >= kWorkFull * p.n_kv * grid;
   kernel<<<static_cast<unsigned>(grid), 384, Cfg::kSmem, stream>>>(tm, p);
   return check_launch("attention");
 }
