@@ -459,19 +459,21 @@ __device__ __forceinline__ uint4* sk_slot(const GemmParams& p, int slot_id) {
   return reinterpret_cast<uint4*>(p.sk_slots) + size_t(slot_id) * (BN / 4) * kBM;
 }
 
-// Park a 128 x BN partial accumulator (this thread's row from TMEM) in a slot.
+// Park a 128 x BN partial accumulator (this thread's row from TMEM) in a slot: the
+// 32-column chunks [c_first, c_first + nchunks) of the tile; tbase addresses chunk c_first.
 template <int BN>
 __device__ __forceinline__ void sk_park(const GemmParams& p, int slot_id, uint32_t tbase,
-                                        int row_in_tile) {
+                                        int row_in_tile, int c_first = 0,
+                                        int nchunks = BN / 32) {
   uint4* slot = sk_slot<BN>(p, slot_id) + row_in_tile;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = 0; c < nchunks; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
     tmem_wait_ld(r);
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      __stcg(slot + size_t(c * 8 + i) * kBM,
+      __stcg(slot + size_t((c_first + c) * 8 + i) * kBM,
              make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
   }
 }
@@ -825,63 +827,70 @@ __device__ __forceinline__ void epilogue_block(const GemmEpilogue& e, int row0, 
 // accumulator from TMEM, plus the partial tiles parked by units [src_lo, src_hi) (slot
 // src * stride + off), then the staged epilogue chunk by chunk.  The next chunk's global
 // inputs and first partial are fetched while the current chunk is finished.
-template <int BN, bool INT8, int EPI>
-__device__ __forceinline__ void epilogue_unit_pair(const GemmParams& p, uint32_t tbase,
-                                                   int row0, int row_in_tile, int col0,
-                                                   int src_lo, int src_hi, int stride,
-                                                   int off, uint4* blk, const float* vec,
-                                                   int lane, LnRow ln) {
-  constexpr int NC = BN / 32;
+template <int BN, bool INT8, int EPI, int NCW>
+__device__ __forceinline__ StatAcc epilogue_unit_pair(const GemmParams& p, uint32_t tbase,
+                                                      int row0, int row_in_tile, int col0,
+                                                      int c_first, int src_lo, int src_hi,
+                                                      int stride, int off, uint4* blk,
+                                                      const float* vec, int lane, LnRow ln) {
+  // NCW 32-column chunks of the tile, [c_first, c_first + NCW): tbase, col0 and vec address
+  // the first of them; the partial slots hold the whole tile.  Returns this row's output
+  // statistics over those columns (when the epilogue keeps them).
   const int nrows = p.M - row0;
   const bool has_part = src_lo < src_hi;
-  const uint4* first = has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile : nullptr;
+  const uint4* first =
+      has_part ? sk_slot<BN>(p, src_lo * stride + off) + row_in_tile + size_t(c_first) * 8 * kBM
+               : nullptr;
   StatAcc sa{0.f, 0.f, 0.f};
   const bool want_stats =
       (EPI == kEpiGateResid || EPI == kEpiBias) && BN == 256 && p.epi.stats_out != nullptr;
   float qks[4] = {1.f, 1.f, 1.f, 1.f};
   if constexpr (epi_base(EPI) == kEpiRope) {
     if (p.epi.q_gain != nullptr && col0 < p.epi.rope_cols)
-      qk_rms_pass<BN, EPI>(p.epi, tbase, vec, ln, qks);
+      qk_rms_pass<NCW * 32, EPI>(p.epi, tbase, vec, ln, qks);
   }
-  // The chunk loop is unrolled by two only (the double buffers alternate at even and odd
-  // chunks): fully unrolled, the epilogue of a 256-wide tile is large enough that its warps
+  // Each chunk's global inputs are fetched while its accumulator columns come out of
+  // tensor memory (two epilogue warps per SMSP hide the rest of the latency; double
+  // buffering them would not fit the registers of a 10-warp CTA).  The loop is unrolled by
+  // two only: fully unrolled, a 256-wide tile's epilogue is large enough that its warps
   // stall on instruction fetch.
-  RowIn in[2];
-  uint4 part[2][8];
-  load_block_in<EPI>(p.epi, row0, nrows, col0, lane, in[0]);
-  if (has_part) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) part[0][i] = __ldcg(first + size_t(i) * kBM);
-  }
 #pragma unroll 2
-  for (int c = 0; c < NC; ++c) {
+  for (int c = 0; c < NCW; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
-    if (c + 1 < NC) {
-      load_block_in<EPI>(p.epi, row0, nrows, col0 + (c + 1) * 32, lane, in[(c + 1) & 1]);
-      if (has_part) {
+    RowIn in;
+    load_block_in<EPI>(p.epi, row0, nrows, col0 + c * 32, lane, in);
+    uint4 part[8];
+    if (has_part) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          part[(c + 1) & 1][i] = __ldcg(first + size_t((c + 1) * 8 + i) * kBM);
-      }
+      for (int i = 0; i < 8; ++i) part[i] = __ldcg(first + size_t(c * 8 + i) * kBM);
     }
     tmem_wait_ld(r);
     if (has_part) {
-      add_part<INT8>(r, part[c & 1]);
+      add_part<INT8>(r, part);
       for (int src = src_lo + 1; src < src_hi; ++src) {
         const uint4* ps = sk_slot<BN>(p, src * stride + off) + row_in_tile;
         uint4 more[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) more[i] = __ldcg(ps + size_t(c * 8 + i) * kBM);
+        for (int i = 0; i < 8; ++i) more[i] = __ldcg(ps + size_t((c_first + c) * 8 + i) * kBM);
         add_part<INT8>(r, more);
       }
     }
-    epilogue_block<EPI>(p.epi, row0, nrows, col0 + c * 32, r, in[c & 1], blk, vec + c * 32,
-                        lane, ln, want_stats ? &sa : nullptr, c == 0,
+    epilogue_block<EPI>(p.epi, row0, nrows, col0 + c * 32, r, in, blk, vec + c * 32, lane, ln,
+                        want_stats ? &sa : nullptr, c == 0,
                         pick4(qks, (c * 32) / p.epi.head_dim));
   }
-  if (want_stats && lane < nrows)
-    p.epi.stats_out[size_t(row0 + lane) * (p.epi.ld_out / 256) + col0 / 256] = stat_final(sa);
+  return sa;
+}
+
+// Group statistics (mean, M2) of a row's 256 columns from two halves of 128 columns, each
+// kept as shifted sums (StatAcc) by its own warp (Chan et al.'s pairwise combination).
+__device__ __forceinline__ float2 stat_half(const StatAcc& a) {
+  return make_float2(a.k + a.s1 * (1.0f / 128.0f), a.s2 - a.s1 * a.s1 * (1.0f / 128.0f));
+}
+__device__ __forceinline__ float2 stat_combine(float2 a, float2 b) {
+  const float d = b.x - a.x;
+  return make_float2(0.5f * (a.x + b.x), a.y + b.y + 64.0f * d * d);
 }
 
 // Epilogue of the transposed pair kernel (A = weights, B = activations, so the TMEM lane
@@ -895,16 +904,13 @@ __device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_
                                                     const float* vec) {
   constexpr int NC = BN / 32;
   float* stage = reinterpret_cast<float*>(blk);
-  RowIn in[2];
-  load_block_in<EPI>(p.epi, tok0, p.tokens - tok0, feat0, lane, in[0]);
 #pragma unroll 2
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
     const int row0 = tok0 + c * 32;
-    if (c + 1 < NC)
-      load_block_in<EPI>(p.epi, row0 + 32, p.tokens - row0 - 32, feat0, lane,
-                         in[(c + 1) & 1]);
+    RowIn in;
+    load_block_in<EPI>(p.epi, row0, p.tokens - row0, feat0, lane, in);
     tmem_wait_ld(r);
 #pragma unroll
     for (int t = 0; t < 32; ++t) stage[t * 32 + ((lane + t) & 31)] = __uint_as_float(r[t]);
@@ -912,7 +918,7 @@ __device__ __forceinline__ void epilogue_unit_trans(const GemmParams& p, uint32_
     uint32_t v[32];
 #pragma unroll
     for (int f = 0; f < 32; ++f) v[f] = __float_as_uint(stage[lane * 32 + ((f + lane) & 31)]);
-    epilogue_block<EPI>(p.epi, row0, p.tokens - row0, feat0, v, in[c & 1], blk, vec, lane,
+    epilogue_block<EPI>(p.epi, row0, p.tokens - row0, feat0, v, in, blk, vec, lane,
                         LnRow{0.f, 1.f}, nullptr, false);
   }
 }
@@ -1134,23 +1140,37 @@ __global__ void __launch_bounds__(192, 1)
 // single-CTA 128 x 256 tile and the ring holds 6 stages.  The even CTA issues the MMAs
 // (M = 256) and signals both CTAs; each CTA's epilogue reads its own 128 accumulator
 // lanes.  Work units (tiles or stream-K ranges) are scheduled per pair.
-#ifndef H3B_PAIR_STAGES
-#define H3B_PAIR_STAGES 6
-#endif
-template <int BN, bool TRANS = false>
+// 256-wide tiles (not transposed) get eight epilogue warps, two per TMEM lane quarter,
+// each taking one 128-column half: one warp per SMSP was slow enough that the last tile's
+// epilogue and the stream-K merges stood out at the end of the kernel.  Narrower and
+// transposed tiles keep four.  Flags are laid out for eight either way.
+constexpr int kPairEpiWarps = 8;
+template <int BN, bool TRANS>
+constexpr int pair_epi_warps() { return BN == 256 && !TRANS ? 8 : 4; }
+// Row statistics of the two halves meet in shared memory: [2 accumulators][4 quarters][32].
+constexpr uint32_t kPairStatBytes = 2 * 4 * 32 * sizeof(float2);
+
+template <int BN, bool TRANS = false, int EPIW = pair_epi_warps<BN, TRANS>()>
 struct PairCfg {
-  static constexpr int kStages = BN == 256 ? H3B_PAIR_STAGES : BN == 160 ? 7 : 8;
+  static constexpr int kEpiWarps = EPIW;
+  static constexpr int kThreads = 64 + 32 * EPIW;
   static constexpr uint32_t kABytes = 128 * kTileBytesK;       // this CTA's 128 rows of A
   static constexpr uint32_t kBBytes = (BN / 2) * kTileBytesK;  // this CTA's half of B
   static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;  // two accumulators
-  static constexpr uint32_t kStageOut = 4 * kWarpStage;  // the 4 epilogue warps' staging
+  static constexpr uint32_t kStageOut = EPIW * kWarpStage + kPairStatBytes;
+  // as many stages as fit (5 at BN 256: one fewer than with four epilogue warps measured
+  // no slower on the block shapes), at most 8
+  static constexpr int kFit =
+      static_cast<int>((232448 - 1024 - 512 - kStageOut) / (kABytes + kBBytes));
+  static constexpr int kStages = kFit < 8 ? kFit : 8;
   static constexpr size_t kSmem =
-      1024 + size_t(kStages) * (kABytes + kBBytes) + kStageOut + 256;
+      1024 + size_t(kStages) * (kABytes + kBBytes) + kStageOut + 512;
+  static_assert(kStages >= 4, "pair kernel ring below 4 stages");
   static_assert(kSmem <= 232448, "pair kernel shared memory above the 227 KB limit");
 };
 
 template <int BN, bool INT8, int EPI, bool TRANS>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<BN, TRANS>::kThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams p) {
   using Cfg = PairCfg<BN, TRANS>;
@@ -1168,12 +1188,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * HA;
   uint8_t* sEpi = sB + STAGES * HB;  // epilogue staging, kWarpStage per epilogue warp
+  float2* sStat = reinterpret_cast<float2*>(sEpi + Cfg::kEpiWarps * kWarpStage);
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * HB + Cfg::kStageOut);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stat_bar = drain + 1;  // [2 accumulators][4 quarters]: the second half's
+                                   // statistics of the tile are in sStat
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stat_bar + 8);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
@@ -1189,9 +1212,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);  // four epilogue warps in each CTA of the pair
+      mbar_init(&tempty[b], 2 * Cfg::kEpiWarps);  // every epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < 8; ++q) mbar_init(&stat_bar[q], 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -1291,27 +1315,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both)
+    // Warp 2 + e: TMEM lane quarter (2 + e) & 3, column half e >> 2 of a 256-wide tile
+    // (with a narrower or transposed tile the second four warps only keep the tile count).
+    constexpr bool kSplit = Cfg::kEpiWarps == 8;
+    constexpr int NCW = kSplit ? BN / 64 : BN / 32;  // 32-column chunks per warp
+    const int ew = warp - 2;
+    const int half = ew >> 2;
+    const bool worker = kSplit || half == 0;
+    const int ch0 = kSplit ? half * (BN / 2) : 0;  // the warp's first column in the tile
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int slot_id = pair * 2 + static_cast<int>(rank);
-    uint4* blk = reinterpret_cast<uint4*>(sEpi + quarter * kWarpStage);
-    float* vec = reinterpret_cast<float*>(sEpi + quarter * kWarpStage + 4096);
+    uint4* blk = reinterpret_cast<uint4*>(sEpi + ew * kWarpStage);
+    float* vec = reinterpret_cast<float*>(sEpi + ew * kWarpStage + 4096);
     int local = 0;
+    int n_stats[2] = {0, 0};  // per accumulator: tiles whose statistics the halves combined
     Sched sc;
     sched_init(p, sc, pair, npairs);
     int tile, kb0, kb1;
+    auto release_acc = [&](int buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&tempty[buf]);
+        else
+          mbar_arrive_cluster(tempty0 + buf * 8);
+      }
+    };
     for (; sched_next(p, sc, tile, kb0, kb1); ++local) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
+      if (!worker) {
+        // paced by the accumulator like the workers, so its arrival counts for this tile
+        const bool ok = __all_sync(0xffffffffu,
+                                   wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait));
+        if (!ok) break;
+        release_acc(buf);
+        continue;
+      }
       // the tile's column vectors, fetched while the accumulator is being computed
       if constexpr (TRANS)
         stage_vectors<EPI, 32>(p.epi, mb * 256 + static_cast<int>(rank) * 128 + quarter * 32,
                                vec, lane);
       else
-        stage_vectors<EPI, BN>(p.epi, nb * BN, vec, lane);
+        stage_vectors<EPI, NCW * 32>(p.epi, nb * BN + ch0, vec, lane);
       const int row_pre = mb * 256 + static_cast<int>(rank) * 128 + row_in_tile;
       const LnRow ln_pre = row_scalars<EPI>(p.epi, row_pre, !TRANS && row_pre < p.M);
       bool ok = wait_bar(&tfull[buf], use & 1u, abort_flag, p.err, kErrGemmWait);
@@ -1319,27 +1370,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       if (!ok) break;
       tc_fence_after();
       const int row = mb * 256 + static_cast<int>(rank) * 128 + row_in_tile;
-      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN);
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * BN + ch0);
       if (kb1 < p.k_blocks) {
-        // stream-K contributor: park this CTA's half of the partial tile in its slot
-        sk_park<BN>(p, slot_id, tbase, row_in_tile);
+        // stream-K contributor: park this warp's part of the partial tile in its slot
+        sk_park<BN>(p, slot_id, tbase, row_in_tile, ch0 / 32, NCW);
         __threadfence();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (rank == 0)
-            mbar_arrive(&tempty[buf]);
-          else
-            mbar_arrive_cluster(tempty0 + buf * 8);
-          st_release_u64(p.sk_flags + slot_id * 4 + quarter, p.sk_seq);
-        }
+        release_acc(buf);
+        if (lane == 0) st_release_u64(p.sk_flags + slot_id * kPairEpiWarps + ew, p.sk_seq);
         continue;
       }
       int c_lo = pair;
       if (kb0 > 0) {
         c_lo = sk_owner(p, static_cast<long long>(tile - p.sk_tile0) * p.k_blocks, npairs);
         for (int c = c_lo; c < pair && ok; ++c) {
-          const unsigned long long* f = p.sk_flags + (c * 2 + static_cast<int>(rank)) * 4 + quarter;
+          const unsigned long long* f =
+              p.sk_flags + (c * 2 + static_cast<int>(rank)) * kPairEpiWarps + ew;
           bool seen = ld_acquire_u64(f) == p.sk_seq;
           if (!seen) {
             const uint64_t t0 = global_timer_ns();
@@ -1356,25 +1401,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
       __syncwarp();  // staged vectors visible to every lane
+      StatAcc sa{0.f, 0.f, 0.f};
       if constexpr (TRANS)
         epilogue_unit_trans<BN, EPI>(p, tbase, lane, mb * 256 + static_cast<int>(rank) * 128 +
                                      quarter * 32, nb * BN, blk, vec);
       else
-        epilogue_unit_pair<BN, INT8, EPI>(p, tbase, row - lane, row_in_tile, nb * BN, c_lo,
-                                          pair, 2, static_cast<int>(rank), blk, vec, lane,
-                                          ln_pre);
+        sa = epilogue_unit_pair<BN, INT8, EPI, NCW>(p, tbase, row - lane, row_in_tile,
+                                                    nb * BN + ch0, ch0 / 32, c_lo, pair, 2,
+                                                    static_cast<int>(rank), blk, vec, lane,
+                                                    ln_pre);
       __syncwarp();
       if (lane == 0)
         for (int src = c_lo; src < pair; ++src)
-          p.sk_flags[(src * 2 + static_cast<int>(rank)) * 4 + quarter] = 0ull;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (rank == 0)
-          mbar_arrive(&tempty[buf]);
-        else
-          mbar_arrive_cluster(tempty0 + buf * 8);
+          p.sk_flags[(src * 2 + static_cast<int>(rank)) * kPairEpiWarps + ew] = 0ull;
+      if constexpr (kSplit && (EPI == kEpiGateResid || EPI == kEpiBias)) {
+        if (p.epi.stats_out != nullptr) {
+          // the row's statistics over the tile's 256 columns: the second half hands its
+          // 128 to the first, which combines and stores them
+          // (one barrier per accumulator: the second half can be a tile ahead, never two
+          // on the same accumulator, which waits for the first half's release)
+          float2* xs = sStat + (buf * 4 + quarter) * 32;
+          const int ns = buf ? n_stats[1] : n_stats[0];
+          if (half == 1) {
+            xs[lane] = stat_half(sa);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&stat_bar[buf * 4 + quarter]);
+          } else {
+            ok = __all_sync(0xffffffffu, wait_bar(&stat_bar[buf * 4 + quarter],
+                                                  static_cast<uint32_t>(ns) & 1u, abort_flag,
+                                                  p.err, kErrGemmWait));
+            if (ok && row < p.M)
+              p.epi.stats_out[size_t(row) * (p.epi.ld_out / 256) + nb] =
+                  stat_combine(stat_half(sa), xs[lane]);
+          }
+          if (buf)
+            ++n_stats[1];
+          else
+            ++n_stats[0];
+        }
       }
+      release_acc(buf);
+      if (!ok) break;
     }
   }
 
@@ -1405,7 +1472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_gemm_pair_grouped(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
   constexpr int BN = 128;
-  using Cfg = PairCfg<BN>;
+  using Cfg = PairCfg<BN, false, 4>;
   constexpr int STAGES = Cfg::kStages;
   constexpr uint32_t HA = Cfg::kABytes;
   constexpr uint32_t HB = Cfg::kBBytes;
@@ -1804,11 +1871,11 @@ int launch_pair(const DevCtx& ctx, const void* A, const void* B, int M, int N, i
         reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kSkFlagsOffset);
     q.sk_seq = next_sk_seq();
     // never more pairs than can be resident at once (occupancy query above)
-    kernel<<<2 * sk_pairs, 192, Cfg::kSmem, stream>>>(ta, tb, q);
+    kernel<<<2 * sk_pairs, Cfg::kThreads, Cfg::kSmem, stream>>>(ta, tb, q);
     *rc = check_launch("gemm_pair");
     return 0;
   }
-  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  kernel<<<2 * std::min(tiles, cap), Cfg::kThreads, Cfg::kSmem, stream>>>(ta, tb, p);
   *rc = check_launch("gemm_pair");
   return 0;
 }
@@ -1856,7 +1923,7 @@ int launch_pair_trans(const DevCtx& ctx, const bf16* X, const bf16* W, int M, in
   if (trace_gemm())
     std::fprintf(stderr, "h3b gemm pair transposed BN=%d M=%d N=%d K=%d tiles=%d cap=%d\n", BN,
                  M, N, K, tiles, cap);
-  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  kernel<<<2 * std::min(tiles, cap), Cfg::kThreads, Cfg::kSmem, stream>>>(ta, tb, p);
   *rc = check_launch("gemm_pair_trans");
   return 0;
 }
@@ -2113,7 +2180,7 @@ int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, 
   if (M <= 0) return 0;
   if (epi.kind != kEpiI8GroupGate || K % kGroupK || N % 128)
     return set_error(-1, "gemm_i8_grouped: K=%d must be a multiple of %d, N=%d of 128", K, kGroupK, N);
-  using Cfg = PairCfg<128>;
+  using Cfg = PairCfg<128, false, 4>;
   auto kernel = k_gemm_pair_grouped<kEpiI8GroupGate>;
   static std::atomic<uint32_t> attr_done{0};
   const uint32_t bit = 1u << (ctx.device & 31);

@@ -103,13 +103,13 @@ struct GemmEpilogue {
 //                                       ([CTA][128][256] words), or the attention's split
 //                                       query tiles ([CTA][head_dim/4][128] float4, then
 //                                       [CTA][128] (m, l) pairs)
-//   [kSkFlagsOffset, kAttnFlagsOffset)  GEMM flags, [CTA][4 epilogue warps]
+//   [kSkFlagsOffset, kAttnFlagsOffset)  GEMM flags, [CTA][8 epilogue warps]
 //   [kAttnFlagsOffset, kScratchBytes)   attention flags, [CTA][4 softmax warps]
 // A flag holds the launch's sequence number (next_scratch_seq) once the 32 partial rows
 // of that warp are written, and is put back to zero by the reader.
 constexpr int kMaxSkCtas = 160;  // grid cap of the split schedules
 constexpr size_t kSkFlagsOffset = size_t(kMaxSkCtas) * 128 * 256 * 4;
-constexpr size_t kAttnFlagsOffset = kSkFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
+constexpr size_t kAttnFlagsOffset = kSkFlagsOffset + size_t(kMaxSkCtas) * 8 * 8;
 constexpr size_t kScratchBytes = kAttnFlagsOffset + size_t(kMaxSkCtas) * 4 * 8;
 
 // Bytes of kernel scratch (kScratchBytes).
