@@ -45,16 +45,16 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch, ncu --set full, the dit512
     # shape after 3 warm-ups (`bench.py --kernel <name> --reps 3`; profiles/), valid while the
     # kernel's source file hashes to src_sha
-    "gemm_fc1_gelu": {"bytes": 85718784 + 18778112, "src": "gemm_tc.cu",
-                      "src_sha": "00a7f8e4ade88b1c"},
-    "gemm_fc2_gate": {"bytes": 137048064 + 17270272, "src": "gemm_tc.cu",
-                      "src_sha": "00a7f8e4ade88b1c"},
-    "gemm_qkv_rope": {"bytes": 67601152 + 8299776, "src": "gemm_tc.cu",
-                      "src_sha": "00a7f8e4ade88b1c"},
-    "gemm_out_gate": {"bytes": 38612736 + 1557504, "src": "gemm_tc.cu",
-                      "src_sha": "00a7f8e4ade88b1c"},
-    "attention": {"bytes": 29564160 + 41984, "src": "attention_tc.cu",
-                  "src_sha": "e705e139b6351063"},
+    "gemm_fc1_gelu": {"bytes": 85656832 + 19310592, "src": "gemm_tc.cu",
+                      "src_sha": "25d03fdf1a80a848"},
+    "gemm_fc2_gate": {"bytes": 137484032 + 17345536, "src": "gemm_tc.cu",
+                      "src_sha": "25d03fdf1a80a848"},
+    "gemm_qkv_rope": {"bytes": 67651328 + 9941760, "src": "gemm_tc.cu",
+                      "src_sha": "25d03fdf1a80a848"},
+    "gemm_out_gate": {"bytes": 38612736 + 1211392, "src": "gemm_tc.cu",
+                      "src_sha": "25d03fdf1a80a848"},
+    "attention": {"bytes": 29571328 + 206848, "src": "attention_tc.cu",
+                  "src_sha": "83cba2667860a7ac"},
 }
 
 
