@@ -88,8 +88,13 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        peaks = dict(FALLBACK_PEAKS)
+        peaks.update({k: float(d[k]) for k in FALLBACK_PEAKS if k in d})
+        peaks["source"] = "MEASURED_PEAKS.json"
+        return peaks, "measured"
+    peaks = dict(FALLBACK_PEAKS)
+    peaks["source"] = "the fallback figures (MEASURED_PEAKS.json absent)"
+    return peaks, "fallback"
 
 
 def block_flops(n, d, f):
@@ -626,7 +631,9 @@ def time_int8_fc2(dev, peaks, reps=10):
            "quantize_cold_hbm_frac": q_bytes / (q_cold * 1e-3) / 1e9 / peaks["hbm_gbs"],
            "int8_gemm_tops": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12,
            "int8_gemm_frac": 2 * M * N * K / (gemm_ms * 1e-3) / 1e12 / int8_peak,
-           "int8_peak_tops": int8_peak, "int8_peak_note": "measured bf16 burst x 2 (nominal ratio)"}
+           "int8_peak_tops": int8_peak,
+           "int8_peak_note": "bf16 burst peak x 2 (nominal ratio); bf16 peak from "
+                             + peaks.get("source", "MEASURED_PEAKS.json or the fallback")}
     del inp, wq, aq, resid
     torch.cuda.empty_cache()
     return res
