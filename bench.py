@@ -429,6 +429,73 @@ def time_gemm_widths(dev, peaks, reps=10):
     return res
 
 
+def time_library_same_shapes(model, cfg, dev, reps=20):
+    """Context for the breakdown: the vendor libraries on the block's shapes, timed the same
+    way (CUDA events around a CUDA-graph replay of `reps` launches, weights rotated over the
+    blocks).  cuBLAS through torch's bf16 linear (no epilogue: no bias, LayerNorm fold, RoPE,
+    GELU or gate), and torch's scaled-dot-product attention on its cuDNN backend where it
+    is available (else torch's own choice, named)."""
+    import torch
+    import torch.nn.functional as F
+    n, d, f, hd, H = cfg.n_tokens, cfg.d, cfg.d_ff, cfg.head_dim, cfg.n_heads
+    P = model.params
+    nb = len(P)
+    g = torch.Generator(device=dev).manual_seed(9)
+    rnd = lambda *s: torch.randn(*s, generator=g, device=dev).to(torch.bfloat16)
+    x, gbuf = rnd(n, d), rnd(n, f)
+    gemms = {"gemm_qkv_rope": (x, "w_qkv", 2 * n * d * 3 * d),
+             "gemm_out_gate": (x, "w_o", 2 * n * d * d),
+             "gemm_fc1_gelu": (x, "w_fc1", 2 * n * d * f),
+             "gemm_fc2_gate": (gbuf, "w_fc2", 2 * n * f * d)}
+
+    def graph_ms(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(reps):
+                fn(i)
+        graph.replay()
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del graph
+        return e0.elapsed_time(e1) / reps
+
+    out = {}
+    for name, (a, w, flops) in gemms.items():
+        ms = graph_ms(lambda i: F.linear(a, P[i % nb][w]))
+        out[name] = {"library": "cuBLAS (torch bf16 linear, no epilogue)", "ms": ms,
+                     "tflops": flops / (ms * 1e-3) / 1e12}
+    q, k, v = (rnd(1, H, n, hd) for _ in range(3))
+    backend = "torch default"
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            F.scaled_dot_product_attention(q, k, v)
+            torch.cuda.synchronize(dev)
+        backend = "cuDNN"
+    except Exception:  # noqa: BLE001  (backend unavailable on this build)
+        pass
+
+    def sdpa(i):
+        if backend == "cuDNN":
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+                return F.scaled_dot_product_attention(q, k, v)
+        return F.scaled_dot_product_attention(q, k, v)
+    ms = graph_ms(sdpa)
+    out["attention"] = {"library": f"torch scaled_dot_product_attention ({backend})", "ms": ms,
+                        "tflops": 4 * n * n * d / (ms * 1e-3) / 1e12}
+    del x, gbuf, q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_reuse(cfg_name, dev, reps=10):
     """Whole denoises under the reuse policies (host loop over the C ABI captured as one
     CUDA graph): ms per denoise and fresh model evaluations, for whole-velocity and
@@ -865,6 +932,7 @@ def run_gpu(args):
         also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
         also["gemm_widths"] = time_gemm_widths(dev, peaks)
+        also["libraries_same_shapes"] = time_library_same_shapes(model, cfg, dev)
         line["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)

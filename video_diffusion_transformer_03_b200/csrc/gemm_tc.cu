@@ -853,8 +853,10 @@ __device__ __forceinline__ StatAcc epilogue_unit_pair(const GemmParams& p, uint3
   // tensor memory (two epilogue warps per SMSP hide the rest of the latency; double
   // buffering them would not fit the registers of a 10-warp CTA).  The loop is unrolled by
   // two only: fully unrolled, a 256-wide tile's epilogue is large enough that its warps
-  // stall on instruction fetch.
-#pragma unroll 2
+  // stall on instruction fetch.  With RoPE (32 more registers of (cos, sin) per chunk) two
+  // chunks in flight overflow the 168 registers, so one.
+  constexpr int kUnroll = epi_base(EPI) == kEpiRope ? 1 : 2;
+#pragma unroll kUnroll
   for (int c = 0; c < NCW; ++c) {
     uint32_t r[32];
     tmem_ld32(tbase + c * 32, r);
@@ -1795,7 +1797,7 @@ int pair_capacity(const DevCtx& ctx) {
   if (c > 0) return c;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (ctx.num_sms / 2));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(PairCfg<BN, TRANS>::kThreads);
   cfg.dynamicSmemBytes = PairCfg<BN, TRANS>::kSmem;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, k_gemm_pair<BN, INT8, EPI, TRANS>, &cfg) !=
