@@ -42,17 +42,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram bytes per launch from an ncu capture, keyed by kernel; only used while the kernel
 # source still hashes to the value recorded with it.
 NCU_TRAFFIC = {
-    # dram__bytes_read.sum + dram__bytes_write.sum of one launch, ncu --set full, the dit512
-    # shape after 3 warm-ups (`bench.py --kernel <name> --reps 3`; profiles/), valid while the
-    # kernel's source file hashes to src_sha
-    "gemm_fc1_gelu": {"bytes": 85656832 + 19310592, "src": "gemm_tc.cu",
-                      "src_sha": "25d03fdf1a80a848"},
-    "gemm_fc2_gate": {"bytes": 137484032 + 17345536, "src": "gemm_tc.cu",
-                      "src_sha": "25d03fdf1a80a848"},
-    "gemm_qkv_rope": {"bytes": 67651328 + 9941760, "src": "gemm_tc.cu",
-                      "src_sha": "25d03fdf1a80a848"},
-    "gemm_out_gate": {"bytes": 38612736 + 1211392, "src": "gemm_tc.cu",
-                      "src_sha": "25d03fdf1a80a848"},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch on the dit512 shape after 3
+    # warm-ups (`bench.py --kernel <name> --reps 3`, ncu --metrics dram__bytes_read.sum,
+    # dram__bytes_write.sum; profiles/), valid while the kernel's source file hashes to src_sha
+    "gemm_fc1_gelu": {"bytes": 85663744 + 18824704, "src": "gemm_tc.cu",
+                      "src_sha": "664c8528af8df287"},
+    "gemm_fc2_gate": {"bytes": 137369600 + 18102016, "src": "gemm_tc.cu",
+                      "src_sha": "664c8528af8df287"},
+    "gemm_qkv_rope": {"bytes": 67641856 + 9009920, "src": "gemm_tc.cu",
+                      "src_sha": "664c8528af8df287"},
+    "gemm_out_gate": {"bytes": 38618880 + 541952, "src": "gemm_tc.cu",
+                      "src_sha": "664c8528af8df287"},
     "attention": {"bytes": 29571328 + 206848, "src": "attention_tc.cu",
                   "src_sha": "83cba2667860a7ac"},
 }
