@@ -1575,6 +1575,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       uint32_t phase = 0;
       bool ok = true;
       int gi = 0;  // groups issued by this pair so far
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 16, 1024);
       for (int tile = pair; tile < tiles && ok; tile += npairs) {
         for (int g = 0; g < groups && ok; ++g, ++gi) {
           const int buf = gi & 1;
@@ -1585,21 +1587,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-          for (int kb = 0; kb < KB_PER_GROUP; ++kb) {
-            if (!wait_bar(&full[stage], phase, abort_flag, p.err, kErrGemmWait)) {
+          // two stages per step: their eight K steps from one asm block (a 256 x 128 int8
+          // MMA is short, and what the thread issues between MMAs idles the tensor pipe)
+          static_assert(K_STEPS == 4, "one stage is four K steps of 32 bytes");
+          static_assert(STAGES % 2 == 0 && KB_PER_GROUP % 2 == 0, "stages taken in pairs");
+          for (int kb = 0; kb < KB_PER_GROUP; kb += 2) {
+            if (!wait_bar(&full[stage], phase, abort_flag, p.err, kErrGemmWait) ||
+                !wait_bar(&full[stage + 1], phase, abort_flag, p.err, kErrGemmWait)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA + stage * HA);
-            const uint32_t b0 = smem_u32(sB + stage * HB);
-#pragma unroll
-            for (int k = 0; k < K_STEPS; ++k)
-              umma_i8_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024),
-                           sdesc_sw128(b0 + k * 32, 16, 1024), IDESC,
-                           (kb > 0 || k > 0) ? 1u : 0u);
+            umma_pair_i8_x8<(HA >> 4), (HB >> 4)>(
+                d_tmem, a_desc0 + static_cast<uint64_t>(stage) * (HA >> 4),
+                b_desc0 + static_cast<uint64_t>(stage) * (HB >> 4), IDESC, kb > 0 ? 1u : 0u);
             tc_commit_pair_mc(&empty[stage], 0x3);
-            if (++stage == STAGES) {
+            tc_commit_pair_mc(&empty[stage + 1], 0x3);
+            stage += 2;
+            if (stage == STAGES) {
               stage = 0;
               phase ^= 1u;
             }

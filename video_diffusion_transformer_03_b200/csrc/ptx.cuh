@@ -354,28 +354,6 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
                : "memory");
 }
 
-// Pair MMA (issued by the even CTA): D (128 lanes in each CTA) (+)= A[256 x K] B[N x K]^T,
-// A rows 0..127 / B rows 0..N/2-1 from the even CTA's shared memory and the rest from the
-// odd CTA's, both at the descriptors' offsets.
-__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Four K steps of a pair MMA (both operands K-major, 128B swizzle: each step advances the
 // descriptors by 32 B) from one asm block, so that the issuing thread puts nothing between
 // them.  KIND_I8 selects kind::i8, else kind::f16.  acc_first: accumulate on the first step.
@@ -409,6 +387,35 @@ __device__ __forceinline__ void umma_pair_x4(uint32_t d_tmem, uint64_t a_desc, u
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first)
         : "memory");
   }
+}
+
+// Two stages of four K steps each (the second stage's descriptors ASTRIDE / BSTRIDE
+// 16-byte units on), eight kind::i8 pair MMAs from one asm block.
+template <uint32_t ASTRIDE, uint32_t BSTRIDE>
+__device__ __forceinline__ void umma_pair_i8_x8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %6;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %8;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %9;\n\tadd.s64 b, %2, %10;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, %11;\n\tadd.s64 b, %2, %12;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], a, b, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first), "n"(ASTRIDE), "n"(BSTRIDE),
+      "n"(ASTRIDE + 2), "n"(BSTRIDE + 2), "n"(ASTRIDE + 4), "n"(BSTRIDE + 4), "n"(ASTRIDE + 6),
+      "n"(BSTRIDE + 6)
+      : "memory");
 }
 
 // Arrive on the mbarrier at this offset in every CTA of `cta_mask` once the pair MMAs
