@@ -45,14 +45,14 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch on the dit512 shape after 3
     # warm-ups (`bench.py --kernel <name> --reps 3`, ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum; profiles/), valid while the kernel's source file hashes to src_sha
-    "gemm_fc1_gelu": {"bytes": 85663744 + 18824704, "src": "gemm_tc.cu",
-                      "src_sha": "664c8528af8df287"},
-    "gemm_fc2_gate": {"bytes": 137369600 + 18102016, "src": "gemm_tc.cu",
-                      "src_sha": "664c8528af8df287"},
-    "gemm_qkv_rope": {"bytes": 67641856 + 9009920, "src": "gemm_tc.cu",
-                      "src_sha": "664c8528af8df287"},
-    "gemm_out_gate": {"bytes": 38618880 + 541952, "src": "gemm_tc.cu",
-                      "src_sha": "664c8528af8df287"},
+    "gemm_fc1_gelu": {"bytes": 85666816 + 18485504, "src": "gemm_tc.cu",
+                      "src_sha": "20099420c547b638"},
+    "gemm_fc2_gate": {"bytes": 137475584 + 16809472, "src": "gemm_tc.cu",
+                      "src_sha": "20099420c547b638"},
+    "gemm_qkv_rope": {"bytes": 67651072 + 9171968, "src": "gemm_tc.cu",
+                      "src_sha": "20099420c547b638"},
+    "gemm_out_gate": {"bytes": 38619392 + 524288, "src": "gemm_tc.cu",
+                      "src_sha": "20099420c547b638"},
     "attention": {"bytes": 29571328 + 206848, "src": "attention_tc.cu",
                   "src_sha": "83cba2667860a7ac"},
 }
