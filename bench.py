@@ -69,7 +69,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--kernel", default=None,
                     help="time one kernel of the block alone on the workload shapes, or the "
-                         "fc2_int8_row / token_pairing workload (for ncu)")
+                         "fc2_int8_row / token_pairing / grouped_fc2_int8 workload (for ncu)")
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--no-also", action="store_true",
                     help="skip the secondary measurements of the other workloads")
@@ -706,6 +706,47 @@ def time_int8_fc2(dev, peaks, reps=10):
     return res
 
 
+def time_grouped_fc2(dev, peaks, reps=20):
+    """The int8 MLP's FC2 at the 512x512 shape (M = 1600 tokens, K = 12288, N = 3072): the
+    grouped int8 GEMM alone (h3b_gemm_i8_grouped; activations quantised per row and 1024
+    channels, weights per output channel) with the gated-residual epilogue, CUDA events
+    around `reps` launches."""
+    import torch
+    from video_diffusion_transformer_03_b200 import h3b
+    M, K, N = 1600, 12288, 3072
+    g = torch.Generator(device=dev).manual_seed(5)
+    a = torch.nn.functional.gelu(torch.randn(M, K, generator=g, device=dev),
+                                 approximate="tanh").to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    asc = torch.empty((M, K // 1024), dtype=torch.float32, device=dev)
+    h3b.quantize_groups(a, aq, asc)
+    wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+    wsc = torch.empty((N,), dtype=torch.float32, device=dev)
+    h3b.quantize_rows(w, wq, wsc)
+    bias = torch.zeros(N, dtype=torch.bfloat16, device=dev)
+    gate = torch.ones(N, device=dev)
+    resid = torch.randn(M, N, generator=g, device=dev).to(torch.bfloat16)
+    run = lambda: h3b.gemm_i8_grouped(aq, asc, wq, wsc, bias, gate, resid)
+    for _ in range(3):
+        run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    h3b.sync_status()
+    ms = e0.elapsed_time(e1) / reps
+    tops = 2 * M * N * K / (ms * 1e-3) / 1e12
+    res = {"workload": f"grouped int8 FC2 M={M} K={K} N={N}", "us": ms * 1e3, "tops": tops,
+           "frac_int8": tops / (2 * peaks["bf16_tflops"])}
+    del a, w, aq, wq, resid
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_token_pairing(dev, peaks, reps=20):
     import torch
     from video_diffusion_transformer_03_b200 import h3b, synth
@@ -798,9 +839,9 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     if args.attn_variant:
         h3b.set_attention_variant(args.attn_variant)
-    if args.kernel in ("fc2_int8_row", "token_pairing"):  # workloads outside the block
-        res = (time_int8_fc2(dev, peaks, reps=args.reps) if args.kernel == "fc2_int8_row"
-               else time_token_pairing(dev, peaks, reps=args.reps))
+    if args.kernel in ("fc2_int8_row", "token_pairing", "grouped_fc2_int8"):  # outside the block
+        res = {"fc2_int8_row": time_int8_fc2, "token_pairing": time_token_pairing,
+               "grouped_fc2_int8": time_grouped_fc2}[args.kernel](dev, peaks, reps=args.reps)
         if rank == 0:
             print(json.dumps({"kernel_only": args.kernel, **res}), flush=True)
         return
@@ -930,6 +971,7 @@ def run_gpu(args):
         also["int8_block_dit512"] = time_int8_block(dev, peaks)
         also["attention_forms"] = time_attention_forms(dev, peaks)
         also["fc2_int8_row"] = time_int8_fc2(dev, peaks)
+        also["grouped_fc2_int8"] = time_grouped_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
         also["gemm_widths"] = time_gemm_widths(dev, peaks)
         also["libraries_same_shapes"] = time_library_same_shapes(model, cfg, dev)
