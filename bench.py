@@ -974,7 +974,10 @@ def run_gpu(args):
         also["grouped_fc2_int8"] = time_grouped_fc2(dev, peaks)
         also["token_pairing"] = time_token_pairing(dev, peaks)
         also["gemm_widths"] = time_gemm_widths(dev, peaks)
-        also["libraries_same_shapes"] = time_library_same_shapes(model, cfg, dev)
+        try:  # context only: a library that cannot run here must not cost the bench line
+            also["libraries_same_shapes"] = time_library_same_shapes(model, cfg, dev)
+        except Exception as exc:  # noqa: BLE001
+            also["libraries_same_shapes"] = {"error": f"{type(exc).__name__}: {exc}"}
         line["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_sample(cfg)
