@@ -708,9 +708,9 @@ def time_int8_fc2(dev, peaks, reps=10):
 
 def time_grouped_fc2(dev, peaks, reps=20):
     """The int8 MLP's FC2 at the 512x512 shape (M = 1600 tokens, K = 12288, N = 3072): the
-    grouped int8 GEMM alone (h3b_gemm_i8_grouped; activations quantised per row and 1024
-    channels, weights per output channel) with the gated-residual epilogue, CUDA events
-    around `reps` launches."""
+    grouped int8 GEMM alone (h3b_gemm_i8_grouped with the kernel scratch, as the int8 block
+    runs it; activations quantised per row and 1024 channels, weights per output channel)
+    with the gated-residual epilogue, CUDA events around `reps` launches."""
     import torch
     from video_diffusion_transformer_03_b200 import h3b
     M, K, N = 1600, 12288, 3072
@@ -727,7 +727,8 @@ def time_grouped_fc2(dev, peaks, reps=20):
     bias = torch.zeros(N, dtype=torch.bfloat16, device=dev)
     gate = torch.ones(N, device=dev)
     resid = torch.randn(M, N, generator=g, device=dev).to(torch.bfloat16)
-    run = lambda: h3b.gemm_i8_grouped(aq, asc, wq, wsc, bias, gate, resid)
+    scratch = torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=dev)
+    run = lambda: h3b.gemm_i8_grouped(aq, asc, wq, wsc, bias, gate, resid, ws=scratch)
     for _ in range(3):
         run()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

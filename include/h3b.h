@@ -504,10 +504,14 @@ int h3b_quantize_groups(const h3b_bf16* a, int rows, int cols, int8_t* q, float*
  *   resid = bf16(resid + gate (w_scale[n] sum_g a_scale[m, g] acc_g[m, n] + bias[n])),
  *   acc_g = the exact int32 product of group g (1024 K columns) of A [M, K] and w_q [N, K].
  * a_scale [M, K / 1024], w_scale, gate [N] fp32; bias [N] bf16 or NULL; resid [M, N]
- * bf16 in/out.  All device.  K % 1024 == 0, N % 128 == 0. */
+ * bf16 in/out.  All device.  K % 1024 == 0, N % 128 == 0.  ws: NULL, or ws_bytes >=
+ * h3b_gemm_workspace_size() of device scratch, which lets a partial last wave of tiles run
+ * stream-K over the groups (the same sums, added in a fixed order); one call at a time per
+ * scratch. */
 int h3b_gemm_i8_grouped(const int8_t* A, const float* a_scale, int M, int K, int N,
                         const int8_t* w_q, const float* w_scale, const h3b_bf16* bias,
-                        const float* gate, h3b_bf16* resid, void* stream);
+                        const float* gate, h3b_bf16* resid, void* ws, size_t ws_bytes,
+                        void* stream);
 
 /* ---------------------------------------------------------------- single kernels */
 /* The projection GEMM used by the block: out = A B^T with an epilogue.

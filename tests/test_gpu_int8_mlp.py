@@ -50,8 +50,13 @@ def test_quantize_groups_bit_exact(rows, cols):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
-@pytest.mark.parametrize("M,K,N", [(1600, 12288, 3072), (40, 1024, 256), (300, 2048, 640)])
-def test_grouped_int8_gemm_vs_oracle(M, K, N):
+# With the scratch, a partial last wave of 256 x 128 tiles runs stream-K over the 1024-column
+# groups: at 1,600 x 3,072 x 12,288, 20 of 168 tiles split over 74 pairs; at 2,048 x 3,072 x
+# 8,192, 44 of 192 tiles of 8 groups.  The small shapes stay data-parallel either way.
+@pytest.mark.parametrize("use_ws", [False, True])
+@pytest.mark.parametrize("M,K,N", [(1600, 12288, 3072), (2048, 8192, 3072), (40, 1024, 256),
+                                   (300, 2048, 640)])
+def test_grouped_int8_gemm_vs_oracle(M, K, N, use_ws):
     z = rnd((M, K), 1.0, seed=M, dtype=torch.float32)
     a = torch.nn.functional.gelu(z, approximate="tanh").to(torch.bfloat16)
     w = rnd((N, K), 0.02, seed=M + 1)
@@ -65,8 +70,15 @@ def test_grouped_int8_gemm_vs_oracle(M, K, N):
     ws = torch.empty((N,), dtype=torch.float32, device=DEV)
     h3b.quantize_rows(w.to(DEV), wq, ws)
     out = resid.to(DEV)
-    h3b.gemm_i8_grouped(aq, asc, wq, ws, bias.to(DEV), gate.to(DEV), out)
+    scratch = (torch.empty(h3b.gemm_workspace_size(), dtype=torch.uint8, device=DEV)
+               if use_ws else None)
+    h3b.gemm_i8_grouped(aq, asc, wq, ws, bias.to(DEV), gate.to(DEV), out, ws=scratch)
     h3b.sync_status()
+    if use_ws:  # the split sums are added in a fixed order: a second call gives the same bits
+        again = resid.to(DEV)
+        h3b.gemm_i8_grouped(aq, asc, wq, ws, bias.to(DEV), gate.to(DEV), again, ws=scratch)
+        h3b.sync_status()
+        assert torch.equal(again, out)
     qo, so = O.quantize_groups(a.float().numpy(), 1024)
     wqo, wso = O.quantize_rows(w.float().numpy())
     y = O.int8_grouped_matmul(qo, so, wqo, wso, 1024) + np64(bias)[None, :]

@@ -1503,8 +1503,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int groups = p.k_blocks / KB_PER_GROUP;
+  // the schedule counts K in groups (p.k_blocks = groups of kGroupK columns), so that a
+  // stream-K cut always falls between two groups
+  const int groups = p.k_blocks;
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < STAGES; ++st) {
@@ -1543,10 +1544,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
       for (int st = 0; st < STAGES; ++st) armed[st] = -1;
       bool ok = true;
-      for (int tile = pair; tile < tiles && ok; tile += npairs) {
+      Sched sc;
+      sched_init(p, sc, pair, npairs);
+      int tile, g0, g1;
+      while (ok && sched_next(p, sc, tile, g0, g1)) {
         int mb, nb;
         tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = g0 * KB_PER_GROUP; kb < g1 * KB_PER_GROUP; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1u, abort_flag, p.err, kErrGemmWait)) {
             ok = false;
             break;
@@ -1577,8 +1581,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       int gi = 0;  // groups issued by this pair so far
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 16, 1024);
       const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 16, 1024);
-      for (int tile = pair; tile < tiles && ok; tile += npairs) {
-        for (int g = 0; g < groups && ok; ++g, ++gi) {
+      Sched sc;
+      sched_init(p, sc, pair, npairs);
+      int tile, g0, g1;
+      while (ok && sched_next(p, sc, tile, g0, g1)) {
+        for (int g = g0; g < g1 && ok; ++g, ++gi) {
           const int buf = gi & 1;
           const uint32_t use = static_cast<uint32_t>(gi >> 1);
           if (!wait_bar(&gempty[buf], (use & 1u) ^ 1u, abort_flag, p.err, kErrGemmWait)) {
@@ -1623,14 +1630,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     float* vec = reinterpret_cast<float*>(sEpi + quarter * kWarpStage + 4096);
     int gi = 0;
     bool ok = true;
-    for (int tile = pair; tile < tiles && ok; tile += npairs) {
+    const int ew = warp - 2;  // epilogue warp 0..3 (its flag in the slot's flag row)
+    const int slot_id = pair * 2 + static_cast<int>(rank);
+    const int row_in_tile = quarter * 32 + lane;
+    Sched sc;
+    sched_init(p, sc, pair, npairs);
+    int tile, g0, g1;
+    while (ok && sched_next(p, sc, tile, g0, g1)) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       stage_vectors<EPI, BN>(p.epi, nb * BN, vec, lane);
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
       const int row = row0 + lane;
       const uint32_t sum_addr = tmem_base + lane_addr + kSumCol;
-      for (int g = 0; g < groups; ++g, ++gi) {
+      for (int g = g0; g < g1; ++g, ++gi) {
         const int buf = gi & 1;
         const uint32_t use = static_cast<uint32_t>(gi >> 1);
         ok = __all_sync(0xffffffffu,
@@ -1645,7 +1658,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           tmem_ld32(acc_addr + c * 32, a);
           tmem_wait_ld(a);
           uint32_t sm[32];
-          if (g > 0) {
+          if (g > g0) {
             tmem_ld32(sum_addr + c * 32, sm);
             tmem_wait_ld(sm);
 #pragma unroll
@@ -1670,6 +1683,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
       }
       if (!ok) break;
+      if (g1 < groups) {
+        // stream-K contributor: park this warp's rows of the running sum in its slot (the
+        // sum is rewritten only by this warp's next fold, after the stores have read it)
+        tc_fence_after();
+        sk_park<BN>(p, slot_id, sum_addr, row_in_tile);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_u64(p.sk_flags + slot_id * kPairEpiWarps + ew, p.sk_seq);
+        tc_fence_before();
+        __syncwarp();
+        continue;
+      }
+      int c_lo = pair;
+      if (g0 > 0) {
+        // the tile's earlier groups were summed by the units below: wait for their parks
+        c_lo = sk_owner(p, static_cast<long long>(tile - p.sk_tile0) * p.k_blocks, npairs);
+        for (int c = c_lo; c < pair && ok; ++c) {
+          const unsigned long long* f =
+              p.sk_flags + (c * 2 + static_cast<int>(rank)) * kPairEpiWarps + ew;
+          bool seen = ld_acquire_u64(f) == p.sk_seq;
+          if (!seen) {
+            const uint64_t t0 = global_timer_ns();
+            while (!seen) {
+              seen = ld_acquire_u64(f) == p.sk_seq;
+              if (!seen && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
+                *abort_flag = 1u;
+                atomicCAS(p.err, 0u, kErrGemmWait);
+                break;
+              }
+            }
+          }
+          ok = __all_sync(0xffffffffu, seen);
+        }
+        if (!ok) break;
+      }
       __syncwarp();  // staged vectors visible to every lane
       const int nrows = p.M - row0;
       RowIn in[2];
@@ -1680,9 +1728,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         tmem_ld32(sum_addr + c * 32, r);
         if (c + 1 < BN / 32) load_block_in<EPI>(p.epi, row0, nrows, nb * BN + (c + 1) * 32, lane, in[(c + 1) & 1]);
         tmem_wait_ld(r);
+        for (int src = c_lo; src < pair; ++src) {  // the parked partial sums, fp32
+          const uint4* ps = sk_slot<BN>(p, src * 2 + static_cast<int>(rank)) + row_in_tile;
+          uint4 part[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) part[i] = __ldcg(ps + size_t(c * 8 + i) * kBM);
+          add_part<false>(r, part);
+        }
         epilogue_block<EPI>(p.epi, row0, nrows, nb * BN + c * 32, r, in[c & 1], blk, vec + c * 32,
                             lane, LnRow{0.f, 1.f}, nullptr, false);
       }
+      if (lane == 0)
+        for (int src = c_lo; src < pair; ++src)
+          p.sk_flags[(src * 2 + static_cast<int>(rank)) * kPairEpiWarps + ew] = 0ull;
       tc_fence_before();
       __syncwarp();
     }
@@ -2183,7 +2241,8 @@ int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, i
 }
 
 int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N,
-                           int K, const GemmEpilogue& epi, cudaStream_t stream) {
+                           int K, const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                           cudaStream_t stream) {
   if (M <= 0) return 0;
   if (epi.kind != kEpiI8GroupGate || K % kGroupK || N % 128)
     return set_error(-1, "gemm_i8_grouped: K=%d must be a multiple of %d, N=%d of 128", K, kGroupK, N);
@@ -2222,16 +2281,37 @@ int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, 
   GemmParams p{};
   p.M = M;
   p.N = N;
-  p.k_blocks = K / 128;
+  p.k_blocks = K / kGroupK;  // the kernel schedules K in groups
   p.m_tiles = (M + 255) / 256;
   p.n_tiles = N / 128;
   p.epi = epi;
   p.err = ctx.err_flag;
   const int tiles = p.m_tiles * p.n_tiles;
+  // A last wave that would leave pairs idle is split stream-K by groups over all pairs,
+  // ahead of the whole waves (which run data-parallel): every pair gets at least one group
+  // of it, the units below a split tile park their fp32 sums, the one holding its last group
+  // adds them in its epilogue.
+  const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
+  const int sk_tile0 = (tiles / sk_pairs) * sk_pairs;
+  const long long iters = static_cast<long long>(tiles - sk_tile0) * p.k_blocks;
+  const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
+                      tiles > sk_pairs && iters >= sk_pairs && forced_sched() != 0;
   if (trace_gemm())
-    std::fprintf(stderr, "h3b gemm i8 grouped M=%d N=%d K=%d tiles=%d cap=%d\n", M, N, K, tiles,
-                 cap);
-  kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+    std::fprintf(stderr, "h3b gemm i8 grouped M=%d N=%d K=%d tiles=%d cap=%d -> %s sk_tile0=%d\n",
+                 M, N, K, tiles, cap, use_sk ? "hybrid stream-K" : "data-parallel",
+                 use_sk ? sk_tile0 : 0);
+  if (use_sk) {
+    p.sk = 1;
+    p.sk_tile0 = sk_tile0;
+    p.sk_iters = iters;
+    p.sk_slots = static_cast<uint32_t*>(scratch);
+    p.sk_flags =
+        reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(scratch) + kSkFlagsOffset);
+    p.sk_seq = next_sk_seq();
+    kernel<<<2 * sk_pairs, 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  } else {
+    kernel<<<2 * std::min(tiles, cap), 192, Cfg::kSmem, stream>>>(ta, tb, p);
+  }
   return check_launch("gemm_i8_grouped");
 }
 

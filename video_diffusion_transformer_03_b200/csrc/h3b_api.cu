@@ -404,7 +404,8 @@ int block_forward_int8_impl(const DevCtx& ctx, const h3b_dims* d, const h3b_bloc
   e.gate = mod + 5 * D;
   e.out = x;
   e.ld_out = D;
-  return launch_gemm_i8_grouped(ctx, ib.gq, q->w_fc2_q, n, D, d->d_ff, e, s);
+  return launch_gemm_i8_grouped(ctx, ib.gq, q->w_fc2_q, n, D, d->d_ff, e, b.gemm_scratch,
+                                gemm_scratch_bytes(), s);
 }
 
 // Workspace of one denoise step.
@@ -879,7 +880,8 @@ int h3b_ln_modulate_q8(const h3b_bf16* x, int n_tokens, int d, float eps, const 
 
 int h3b_gemm_i8_grouped(const int8_t* A, const float* a_scale, int M, int K, int N,
                         const int8_t* w_q, const float* w_scale, const h3b_bf16* bias,
-                        const float* gate, h3b_bf16* resid, void* stream) {
+                        const float* gate, h3b_bf16* resid, void* ws, size_t ws_bytes,
+                        void* stream) {
   if (M < 0 || K <= 0 || K % 1024 || N <= 0 || N % 128)
     return set_error(H3B_EINVAL, "gemm_i8_grouped: K=%d must be a multiple of 1024, N=%d of 128", K, N);
   const void* ptrs[6] = {A, a_scale, w_q, w_scale, gate, resid};
@@ -897,7 +899,8 @@ int h3b_gemm_i8_grouped(const int8_t* A, const float* a_scale, int M, int K, int
   e.gate = gate;
   e.out = reinterpret_cast<bf16*>(resid);
   e.ld_out = N;
-  return launch_gemm_i8_grouped(ctx, A, w_q, M, N, K, e, static_cast<cudaStream_t>(stream));
+  return launch_gemm_i8_grouped(ctx, A, w_q, M, N, K, e, ws, ws ? ws_bytes : 0,
+                                static_cast<cudaStream_t>(stream));
 }
 
 int h3b_block_forward_noalloc(const h3b_dims* dims, const h3b_block_weights* w,

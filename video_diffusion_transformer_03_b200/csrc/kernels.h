@@ -134,9 +134,11 @@ int launch_gemm_i8(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, i
                    const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
                    cudaStream_t stream);
 // Grouped int8 product (kEpiI8GroupGate): one A scale per row and 1024-column group.
-// K % 1024 == 0, N % 128 == 0.
+// K % 1024 == 0, N % 128 == 0.  scratch (>= gemm_scratch_bytes(), or null) lets a partial
+// last wave run stream-K over groups.
 int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, int M, int N,
-                           int K, const GemmEpilogue& epi, cudaStream_t stream);
+                           int K, const GemmEpilogue& epi, void* scratch, size_t scratch_bytes,
+                           cudaStream_t stream);
 
 // ---------------------------------------------------------------- attention (tcgen05)
 // scratch (>= gemm_scratch_bytes(), or null) enables the persistent split schedule:

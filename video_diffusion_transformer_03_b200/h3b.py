@@ -107,7 +107,7 @@ _SIGS = {
                                     ctypes.POINTER(Int8Block), _P, _P, _I, _P, _P, _SZ, _P]),
     "h3b_ln_modulate_q8": (_I, [_P, _I, _I, _F, _P, _P, _P, _P, _P]),
     "h3b_quantize_groups": (_I, [_P, _I, _I, _P, _P, _P]),
-    "h3b_gemm_i8_grouped": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "h3b_gemm_i8_grouped": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "h3b_reuse_schedule": (_I, [_I, _I, _P]),
     "h3b_denoise_step_keep": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Grid), _I,
                                    ctypes.POINTER(BlockWeights), _P, _P, _P, _I, _I, _F, _F, _P,
@@ -477,11 +477,15 @@ def quantize_groups(a, q, scale, stream=None) -> None:
                                    _stream(stream)))
 
 
-def gemm_i8_grouped(A, a_scale, w_q, w_scale, bias, gate, resid, stream=None) -> None:
+def gemm_i8_grouped(A, a_scale, w_q, w_scale, bias, gate, resid, ws=None,
+                    stream=None) -> None:
+    """ws: None (data-parallel) or a device buffer of gemm_workspace_size() bytes (a partial
+    last wave of tiles runs stream-K over the 1024-column groups)."""
     _dev(A, torch.int8, "A"); _dev(w_q, torch.int8, "w_q"); _dev(resid, torch.bfloat16, "resid")
     M, K = A.shape
     _check(lib.h3b_gemm_i8_grouped(_ptr(A), _ptr(a_scale), M, K, w_q.shape[0], _ptr(w_q),
                                    _ptr(w_scale), _ptr(bias), _ptr(gate), _ptr(resid),
+                                   _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                    _stream(stream)))
 
 
