@@ -45,14 +45,14 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch on the dit512 shape after 3
     # warm-ups (`bench.py --kernel <name> --reps 3`, ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum; profiles/), valid while the kernel's source file hashes to src_sha
-    "gemm_fc1_gelu": {"bytes": 85666816 + 18485504, "src": "gemm_tc.cu",
-                      "src_sha": "20099420c547b638"},
-    "gemm_fc2_gate": {"bytes": 137475584 + 16809472, "src": "gemm_tc.cu",
-                      "src_sha": "20099420c547b638"},
-    "gemm_qkv_rope": {"bytes": 67651072 + 9171968, "src": "gemm_tc.cu",
-                      "src_sha": "20099420c547b638"},
-    "gemm_out_gate": {"bytes": 38619392 + 524288, "src": "gemm_tc.cu",
-                      "src_sha": "20099420c547b638"},
+    "gemm_fc1_gelu": {"bytes": 85670144 + 18355200, "src": "gemm_tc.cu",
+                      "src_sha": "665f04dfed9c3e04"},
+    "gemm_fc2_gate": {"bytes": 137548544 + 17156096, "src": "gemm_tc.cu",
+                      "src_sha": "665f04dfed9c3e04"},
+    "gemm_qkv_rope": {"bytes": 67616512 + 9027072, "src": "gemm_tc.cu",
+                      "src_sha": "665f04dfed9c3e04"},
+    "gemm_out_gate": {"bytes": 38624512 + 1132032, "src": "gemm_tc.cu",
+                      "src_sha": "665f04dfed9c3e04"},
     "attention": {"bytes": 29571328 + 206848, "src": "attention_tc.cu",
                   "src_sha": "83cba2667860a7ac"},
 }
