@@ -1460,13 +1460,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<BN, TRANS>::
 // ---------------------------------------------------------------------------------------
 // Grouped int8 pair GEMM: the A operand carries one scale per row and per group of 1024 K
 // columns (the int8 MLP's FC2 input), so the group products cannot share one integer
-// accumulator.  Pair tiles of 256 x 128, data-parallel.  TMEM (per CTA, 128 lanes): two
-// int32 group accumulators (columns 0-127 and 128-255) and the fp32 running sum (256-383).
-// The MMA issuer fills accumulator g & 1 with group g's products (the accumulation
-// restarts at each group) and signals gfull; the epilogue warps fold it into the sum,
-// sum += float(acc_g) * s_a[row, g], and hand the accumulator back (gempty), so the fold
-// of group g overlaps the products of group g + 1.  After a tile's last group the same
-// warps run the staged epilogue on the sum.
+// accumulator.  Pair tiles of 256 x 128; with the scratch, the tiles past the whole waves
+// are split stream-K in groups (lower units park their fp32 sums, the owner adds them).
+// TMEM (per CTA, 128 lanes): two int32 group accumulators (columns 0-127, 128-255) and the
+// fp32 running sum (256-383).  The MMA issuer fills accumulator g & 1 with group g's
+// products and signals gfull; the epilogue warps fold it into the sum, sum += float(acc_g)
+// * s_a[row, g], and hand it back (gempty), so the fold of group g overlaps the products
+// of group g + 1.  After a tile's last group the same warps run the staged epilogue.
 constexpr int kGroupK = 1024;
 
 template <int EPI>
