@@ -1,19 +1,19 @@
-// Persistent, warp-specialised tcgen05 GEMM for the block's projections (QKV, out-proj,
-// FC1, FC2) and the int8 row-scaled FC2:  out = A[M, K] * B[N, K]^T  with a fused
-// epilogue.
+// Persistent, warp-specialised tcgen05 GEMMs for the block's projections (QKV, out-proj,
+// FC1, FC2) and the int8 row-scaled and grouped FC2:  out = A[M, K] * B[N, K]^T  with a
+// fused epilogue.
 //
-// Roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: 128-byte-swizzled [128 x 128 B] A tiles and [BN x 128 B] B
-//               tiles into a STAGES-deep shared-memory ring;
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma per stage,
-//               accumulating a 128 x BN fp32 / int32 tile in tensor memory; two
-//               accumulator buffers so the epilogue of tile i overlaps the MMAs of
-//               tile i + 1;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = row, 32 columns per
-//               load), bias / GELU / RoPE / gated residual / int8 dequant, 16-byte
-//               global stores.
-// Tiles are visited in groups of 16 M-tiles (M fastest) so that CTAs running together
-// share weight tiles in L2.
+// Main form, a CTA pair (cluster of 2, cta_group::2) per 256 x BN tile:
+//   warp 0      TMA producer: 128-byte-swizzled [128 x 128 B] A tiles and [BN/2 x 128 B]
+//               B tiles into a STAGES-deep shared-memory ring in each CTA;
+//   warp 1      TMEM allocator; in the even CTA the MMA issuer (one thread): 4 x
+//               tcgen05.mma per stage into a 256 x BN fp32 / int32 accumulator; two
+//               accumulator buffers, so the epilogue of tile i overlaps tile i + 1's MMAs;
+//   warps 2..   epilogue (4 warps, 8 for 256-wide tiles): tcgen05.ld of the accumulator
+//               (thread = row, 32 columns per load), bias / LayerNorm fold / GELU / RoPE /
+//               gated residual / int8 dequant, staged through shared memory, coalesced.
+// Single-CTA 128 x BN tiles (192 threads) serve M < 256.  Tiles are visited in groups of
+// 16 M-tiles (M fastest) so that CTAs running together share weight tiles in L2; schedules
+// data-parallel, stream-K or both (a cost model picks), all waits bounded.
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.h"
