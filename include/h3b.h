@@ -160,14 +160,17 @@ size_t h3b_denoise_workspace_size(const h3b_dims* dims, const h3b_grid* grid, in
  * pair kernel, a CTA of the single-SM kernel) out of `units`, for `tiles` output tiles of
  * `k_blocks` K slices each.  mode: 0 data-parallel; 1 hybrid stream-K (the pair kernel's
  * form: whole waves but the last data-parallel, the rest split evenly); 2 stream-K over
- * every tile (the single-SM kernel's form).  Item i goes to items[4 i .. 4 i + 3] (host,
+ * every tile (the single-SM kernel's form); 3 remainder stream-K (the grouped int8 kernel's
+ * form, K slices being its 1024-column groups: every whole wave data-parallel, the tiles
+ * past them split evenly).  Item i goes to items[4 i .. 4 i + 3] (host,
  * caller-owned) as (tile, first K slice, end K slice, merge), in processing order: merge
  * is -1 for a partial tile the unit parks for a higher unit, else the first unit whose
  * parked partial the item's epilogue adds (the unit itself when it adds none).  At most
  * max_items items are written.  Returns the number of items, or H3B_EINVAL for
- * non-positive sizes, a unit outside [0, units), a mode outside 0-2, a missing buffer, or
- * a stream-K mode with fewer than 4 split K slices per unit (the GEMM calls run those
- * shapes data-parallel). */
+ * non-positive sizes, a unit outside [0, units), a mode outside 0-3, a missing buffer, or
+ * a stream-K mode with fewer than 4 split K slices per unit (mode 3: fewer than one, or
+ * no partial wave past at least one whole one); the GEMM calls run those shapes
+ * data-parallel. */
 int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, int* items,
                       int max_items);
 

@@ -1,6 +1,6 @@
-"""The GEMM kernels' work schedule (data-parallel, hybrid stream-K, stream-K), enumerated on
-the host by the functions the kernels run (h3b_gemm_schedule), against the properties the
-kernels rely on: every (tile, K slice) is computed exactly once; each tile is finished by
+"""The GEMM kernels' work schedule (data-parallel, hybrid stream-K, stream-K, and the grouped
+int8 kernel's remainder stream-K), enumerated on the host by the functions the kernels run
+(h3b_gemm_schedule), against the properties the kernels rely on: every (tile, K slice) is computed exactly once; each tile is finished by
 the unit holding its last K slice, which adds the partials of exactly the lower units that
 computed the rest; a unit parks at most one partial, as its first item, so its slot and
 flag are written once and every wait points at work done before anything else.  No GPU."""
@@ -28,9 +28,24 @@ def hybrid_tile0(tiles, units):
     return max(0, tiles // units - 1) * units
 
 
+def remainder_tile0(tiles, units):
+    return tiles // units * units
+
+
 def split_iters(tiles, kb, units, mode):
-    tile0 = hybrid_tile0(tiles, units) if mode == h3b.SCHED_HYBRID_STREAM_K else 0
+    tile0 = (hybrid_tile0(tiles, units) if mode == h3b.SCHED_HYBRID_STREAM_K else
+             remainder_tile0(tiles, units) if mode == h3b.SCHED_REMAINDER_STREAM_K else 0)
     return (tiles - tile0) * kb
+
+
+def runs_split(tiles, kb, units, mode):
+    """Whether the GEMM calls split this shape in this mode (else they run it
+    data-parallel): a unit with an empty range would never publish the flag its tile's
+    owner waits for, so the pair kernels want 4 K slices per unit, the grouped kernel one
+    group per unit and a partial wave past whole ones."""
+    if mode == h3b.SCHED_REMAINDER_STREAM_K:
+        return tiles > units and split_iters(tiles, kb, units, mode) >= units
+    return split_iters(tiles, kb, units, mode) >= 4 * units
 
 
 def check_schedule(tiles, kb, units, mode):
@@ -66,13 +81,18 @@ def check_schedule(tiles, kb, units, mode):
     return per_unit
 
 
-@pytest.mark.parametrize("tiles,kb,units", SHAPES + _random_shapes(300))
+# (tiles, groups, units): the grouped int8 FC2 at 1,600 and 2,048 tokens (256 x 128 tiles,
+# 1024-column groups, 74 pairs) and edge cases of the remainder form
+GROUPED_SHAPES = [(168, 12, 74), (192, 8, 74), (75, 12, 74), (149, 1, 74), (148, 12, 74),
+                  (80, 3, 74), (7, 5, 3)]
+
+
+@pytest.mark.parametrize("tiles,kb,units", SHAPES + GROUPED_SHAPES + _random_shapes(300))
 @pytest.mark.parametrize("mode", [h3b.SCHED_DATA_PARALLEL, h3b.SCHED_HYBRID_STREAM_K,
-                                  h3b.SCHED_STREAM_K], ids=["dp", "hybrid", "sk"])
+                                  h3b.SCHED_STREAM_K, h3b.SCHED_REMAINDER_STREAM_K],
+                         ids=["dp", "hybrid", "sk", "remainder"])
 def test_schedule_properties(tiles, kb, units, mode):
-    if mode != h3b.SCHED_DATA_PARALLEL and split_iters(tiles, kb, units, mode) < 4 * units:
-        # the GEMM calls run such shapes data-parallel: a unit with an empty range would
-        # never publish the flag its tile's owner waits for
+    if mode != h3b.SCHED_DATA_PARALLEL and not runs_split(tiles, kb, units, mode):
         with pytest.raises(h3b.H3BError):
             h3b.gemm_schedule(tiles, kb, units, mode, 0)
         return
@@ -103,6 +123,25 @@ def test_hybrid_splits_only_the_last_one_to_two_waves(tiles, kb, units):
         assert units <= tiles - tile0 < 2 * units
 
 
+@pytest.mark.parametrize("tiles,kb,units", GROUPED_SHAPES + _random_shapes(100, seed=7))
+def test_remainder_splits_only_the_partial_wave(tiles, kb, units):
+    if not runs_split(tiles, kb, units, h3b.SCHED_REMAINDER_STREAM_K):
+        pytest.skip("run data-parallel by the grouped GEMM")
+    tile0 = remainder_tile0(tiles, units)
+    sk_iters = (tiles - tile0) * kb
+    for u in range(units):
+        items = h3b.gemm_schedule(tiles, kb, units, h3b.SCHED_REMAINDER_STREAM_K, u)
+        split = [it for it in items if it[0] >= tile0]
+        whole = [it for it in items if it[0] < tile0]
+        # the split items first, then every whole wave data-parallel
+        assert items == split + whole
+        assert whole == [(t, 0, kb, u) for t in range(u, tile0, units)]
+        share = sum(k1 - k0 for _, k0, k1, _ in split)
+        assert share == sk_iters * (u + 1) // units - sk_iters * u // units
+        assert share >= 1                      # every unit publishes what its owner awaits
+    assert 0 < tiles - tile0 < units
+
+
 def test_block_shapes_examples():
     # QKV at 1,600 tokens (252 tiles, 48 K slices, 74 pairs), pair 0: parks the first 19
     # slices of tile 149, finishes tile 148 alone, then data-parallel tiles 0 and 74
@@ -112,10 +151,17 @@ def test_block_shapes_examples():
     # finishes tile 5 from slice 32 after adding pair 4's partial
     assert h3b.gemm_schedule(84, 48, 74, h3b.SCHED_HYBRID_STREAM_K, 5) == [
         (6, 0, 38, -1), (5, 32, 48, 4)]
+    # grouped int8 FC2 at 1,600 tokens (168 tiles of 12 groups, 74 pairs): pair 0 parks
+    # groups 0-2 of tile 148, then runs tiles 0 and 74 whole; pair 73 finishes tile 167
+    # from group 8 after adding the sums of pairs 70-72
+    assert h3b.gemm_schedule(168, 12, 74, h3b.SCHED_REMAINDER_STREAM_K, 0) == [
+        (148, 0, 3, -1), (0, 0, 12, 0), (74, 0, 12, 0)]
+    assert h3b.gemm_schedule(168, 12, 74, h3b.SCHED_REMAINDER_STREAM_K, 73) == [
+        (167, 8, 12, 70), (73, 0, 12, 73), (147, 0, 12, 73)]
 
 
 def test_schedule_rejects_bad_arguments():
-    for args in [(0, 8, 4, 0, 0), (8, 0, 4, 0, 0), (8, 8, 0, 0, 0), (8, 8, 4, 3, 0),
-                 (8, 8, 4, 0, 4), (8, 8, 4, 0, -1)]:
+    for args in [(0, 8, 4, 0, 0), (8, 0, 4, 0, 0), (8, 8, 0, 0, 0), (8, 8, 4, 4, 0),
+                 (8, 8, 4, 0, 4), (8, 8, 4, 0, -1), (8, 8, 4, 3, 0)]:
         with pytest.raises(h3b.H3BError):
             h3b.gemm_schedule(*args)

@@ -1772,6 +1772,10 @@ unsigned long long next_sk_seq() {
 // (all tiles, when there are fewer than two waves).
 int hybrid_tile0(int tiles, int units) { return std::max(0, tiles / units - 1) * units; }
 
+// First stream-K tile of the grouped int8 kernel's schedule: every whole wave runs
+// data-parallel and only the tiles past them are split (K counted in 1024-column groups).
+int remainder_tile0(int tiles, int units) { return (tiles / units) * units; }
+
 // Schedule costs in units of one K slice of one tile on one scheduling unit.
 // Data-parallel: ceil(tiles / units) waves of k_blocks slices.  Stream-K over the tiles
 // from dp_tiles on: the whole waves before it, plus the even share of the split tiles
@@ -2080,9 +2084,13 @@ int gemm_schedule_items(int tiles, int k_blocks, int units, int mode, int unit, 
   p.n_tiles = 1;
   if (mode != 0) {
     p.sk = 1;
-    p.sk_tile0 = mode == 1 ? hybrid_tile0(tiles, units) : 0;
+    p.sk_tile0 = mode == 1 ? hybrid_tile0(tiles, units)
+                           : mode == 3 ? remainder_tile0(tiles, units) : 0;
     p.sk_iters = static_cast<long long>(tiles - p.sk_tile0) * k_blocks;
-    if (p.sk_iters < 4LL * units) return -1;
+    // the pair kernels split only with at least 4 K slices per unit; the grouped kernel
+    // with at least one group per unit, and only a partial wave past whole ones
+    if (mode == 3 ? (tiles <= units || p.sk_iters < units) : p.sk_iters < 4LL * units)
+      return -1;
   }
   Sched sc;
   sched_init(p, sc, unit, units);
@@ -2292,7 +2300,7 @@ int launch_gemm_i8_grouped(const DevCtx& ctx, const int8_t* A, const int8_t* B, 
   // of it, the units below a split tile park their fp32 sums, the one holding its last group
   // adds them in its epilogue.
   const int sk_pairs = std::min(cap, kMaxSkCtas / 2);
-  const int sk_tile0 = (tiles / sk_pairs) * sk_pairs;
+  const int sk_tile0 = remainder_tile0(tiles, sk_pairs);
   const long long iters = static_cast<long long>(tiles - sk_tile0) * p.k_blocks;
   const bool use_sk = scratch != nullptr && scratch_bytes >= kScratchBytes &&
                       tiles > sk_pairs && iters >= sk_pairs && forced_sched() != 0;

@@ -687,12 +687,13 @@ int h3b_gemm_schedule(int tiles, int k_blocks, int units, int mode, int unit, in
   if (tiles <= 0 || k_blocks <= 0 || units <= 0 || unit < 0 || unit >= units)
     return set_error(H3B_EINVAL, "gemm_schedule: tiles=%d k_blocks=%d units=%d unit=%d", tiles,
                      k_blocks, units, unit);
-  if (mode < 0 || mode > 2) return set_error(H3B_EINVAL, "gemm_schedule: mode %d", mode);
+  if (mode < 0 || mode > 3) return set_error(H3B_EINVAL, "gemm_schedule: mode %d", mode);
   if (max_items < 0 || (max_items > 0 && !items))
     return set_error(H3B_EINVAL, "gemm_schedule: items buffer");
   const int n = gemm_schedule_items(tiles, k_blocks, units, mode, unit, items, max_items);
   if (n < 0)
-    return set_error(H3B_EINVAL, "gemm_schedule: fewer than 4 split K slices per unit");
+    return set_error(H3B_EINVAL, "gemm_schedule: too few split K slices per unit for mode %d",
+                     mode);
   return n;
 }
 

@@ -212,6 +212,7 @@ def gemm_workspace_size() -> int:
 
 
 SCHED_DATA_PARALLEL, SCHED_HYBRID_STREAM_K, SCHED_STREAM_K = 0, 1, 2
+SCHED_REMAINDER_STREAM_K = 3  # h3b_gemm_schedule only: the grouped int8 kernel's form
 
 
 def gemm_schedule(tiles: int, k_blocks: int, units: int, mode: int, unit: int):
